@@ -1,0 +1,392 @@
+"""Pins of the fp64 oracle against facts it does not compute itself.
+
+Each test ties one oracle function to a closed form, a library routine, an
+invariant the pages state, or a special case that reduces to one, so that a
+dropped term, a wrong sign, a wrong index or a transposed operand fails here.
+"""
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+from oracle import dllm_oracle as O
+from diffusion_decoding_step_b200 import workload as wl
+from tests.oracle_inputs import Case, oracle_config
+
+RNG = np.random.default_rng(1234)
+
+
+# ---------------------------------------------------------------- rounding
+def test_round_bf16_matches_torch():
+    x = np.concatenate([RNG.standard_normal(20000) * 10.0 ** RNG.integers(-8, 8, 20000),
+                        [0.0, -0.0, 1.0, 1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, 65504.0]])
+    ref = torch.tensor(x, dtype=torch.float32).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(O.round_bf16(x), ref)
+
+
+def test_round_bf16_ties_to_even():
+    # 1 + 2^-8 lies halfway between bf16 neighbours 1 and 1 + 2^-7 -> even (1.0)
+    assert O.round_bf16(1.0 + 2.0 ** -8) == 1.0
+    # 1 + 3*2^-8 lies halfway between 1 + 2^-7 and 1 + 2^-6 -> even mantissa
+    assert O.round_bf16(1.0 + 3 * 2.0 ** -8) == 1.0 + 2.0 ** -6
+
+
+# ---------------------------------------------------------------- rope
+def test_rope_position_zero_is_identity():
+    x = RNG.standard_normal((5, 3, 16))
+    np.testing.assert_array_equal(O.rope(x, np.zeros(3), 1e6), x)
+
+
+def test_rope_d2_is_complex_rotation():
+    # D = 2: inv_freq = 1, so the pair (x1, x2) is the complex number x1 + i x2
+    # multiplied by exp(i * pos).
+    x = RNG.standard_normal((7, 2))
+    pos = np.arange(7) * 0.37
+    z = (x[:, 0] + 1j * x[:, 1]) * np.exp(1j * pos)
+    out = O.rope(x, pos, 10000.0)
+    np.testing.assert_allclose(out[:, 0], z.real, atol=1e-14)
+    np.testing.assert_allclose(out[:, 1], z.imag, atol=1e-14)
+
+
+def test_rope_scores_depend_on_relative_position_only():
+    D = 32
+    q = RNG.standard_normal((1, D))
+    k = RNG.standard_normal((1, D))
+    for theta in (1e4, 1e6):
+        base = (O.rope(q, np.array([11.0]), theta) @ O.rope(k, np.array([4.0]), theta).T)[0, 0]
+        shifted = (O.rope(q, np.array([511.0]), theta)
+                   @ O.rope(k, np.array([504.0]), theta).T)[0, 0]
+        assert abs(base - shifted) < 1e-10
+        # and it is not the unrotated product (the rotation does something)
+        assert abs(base - (q @ k.T)[0, 0]) > 1e-6
+
+
+def test_rope_frequency_of_last_pair():
+    # pair i = D/2 - 1 rotates by pos * theta^(-(D-2)/D)
+    D, theta, pos = 8, 100.0, 3.0
+    x = np.zeros((1, D))
+    x[0, D // 2 - 1] = 1.0
+    out = O.rope(x, np.array([pos]), theta)
+    ang = pos * theta ** (-(D - 2) / D)
+    assert abs(out[0, D // 2 - 1] - np.cos(ang)) < 1e-14
+    assert abs(out[0, D - 1] - np.sin(ang)) < 1e-14
+
+
+# ---------------------------------------------------------------- attention
+def test_attention_closed_form_weights():
+    # keys built so that q.k_i / sqrt(D) = log w_i: softmax weights are w / sum(w)
+    D = 16
+    q = RNG.standard_normal((1, D))
+    w = np.array([1.0, 2.0, 3.0, 10.0])
+    k = (np.sqrt(D) * np.log(w))[:, None] * q / (q @ q.T)
+    v = RNG.standard_normal((4, D))
+    o = O.attention(q, k, v)
+    np.testing.assert_allclose(o[0], (w / w.sum()) @ v, rtol=1e-12, atol=1e-12)
+
+
+def test_attention_single_key_returns_value():
+    q = RNG.standard_normal((3, 8))
+    k = RNG.standard_normal((1, 8))
+    v = RNG.standard_normal((1, 8))
+    np.testing.assert_allclose(O.attention(q, k, v), np.repeat(v, 3, 0), atol=1e-15)
+
+
+def test_attention_equal_scores_give_mean():
+    q = np.zeros((2, 8))
+    k = RNG.standard_normal((5, 8))
+    v = RNG.standard_normal((5, 8))
+    np.testing.assert_allclose(O.attention(q, k, v), np.repeat(v.mean(0, keepdims=True), 2, 0),
+                               atol=1e-15)
+
+
+def test_attention_key_order_irrelevant_and_rows_independent():
+    q = RNG.standard_normal((4, 8))
+    k = RNG.standard_normal((9, 8))
+    v = RNG.standard_normal((9, 8))
+    perm = RNG.permutation(9)
+    o = O.attention(q, k, v)
+    np.testing.assert_allclose(O.attention(q, k[perm], v[perm]), o, atol=1e-14)
+    np.testing.assert_allclose(O.attention(q[2:3], k, v), o[2:3], atol=1e-15)
+
+
+def test_attention_scale_is_inverse_sqrt_d():
+    # two keys with q.k difference delta: weight ratio exp(delta / sqrt(D))
+    D = 64
+    q = np.zeros((1, D)); q[0, 0] = 1.0
+    k = np.zeros((2, D)); k[1, 0] = 3.0
+    v = np.array([[0.0] * D, [1.0] * D])
+    p1 = 1.0 / (1.0 + np.exp(-3.0 / 8.0))
+    np.testing.assert_allclose(O.attention(q, k, v)[0], np.full(D, p1), rtol=1e-13)
+
+
+# ---------------------------------------------------------------- LM head
+def test_lm_head_identity_closed_form():
+    # w_lm = I  -> logits = h;  h = (0, ln 2, ln 5) -> conf = 5/8, tok = 2, gap = ln 5 - ln 2
+    h = np.array([[0.0, np.log(2.0), np.log(5.0)]])
+    c, t, g = O.lm_head_confidence(h, np.eye(3))
+    assert abs(c[0] - 5.0 / 8.0) < 1e-15 and t[0] == 2
+    assert abs(g[0] - (np.log(5.0) - np.log(2.0))) < 1e-15
+
+
+def test_lm_head_matches_scipy_softmax_and_logsumexp():
+    h = RNG.standard_normal((6, 32)) * 3
+    w = RNG.standard_normal((500, 32)) * 0.3
+    c, t, g = O.lm_head_confidence(h, w)
+    logits = h @ w.T
+    p = scipy.special.softmax(logits, axis=1)
+    np.testing.assert_allclose(p.sum(1), 1.0, atol=1e-12)
+    np.testing.assert_allclose(c, p.max(1), rtol=1e-12)
+    np.testing.assert_allclose(c, np.exp(logits.max(1) - scipy.special.logsumexp(logits, axis=1)),
+                               rtol=1e-12)
+    assert np.all(t == np.argmax(p, axis=1))
+    srt = np.sort(logits, axis=1)
+    np.testing.assert_allclose(g, srt[:, -1] - srt[:, -2], atol=1e-12)
+    assert np.all((c > 0) & (c <= 1) & (c >= 1.0 / 500 - 1e-15))
+
+
+def test_lm_head_ties_lowest_id_and_zero_gap():
+    w = np.eye(4)
+    h = np.array([[1.0, 3.0, 3.0, 0.0]])
+    c, t, g = O.lm_head_confidence(h, w)
+    assert t[0] == 1 and g[0] == 0.0
+
+
+def test_lm_head_uniform_logits_conf_is_one_over_v():
+    c, t, g = O.lm_head_confidence(np.zeros((1, 4)), RNG.standard_normal((37, 4)))
+    assert abs(c[0] - 1.0 / 37) < 1e-15 and t[0] == 0
+
+
+# ---------------------------------------------------------------- commit
+def test_commit_threshold_strict_and_forced():
+    conf = np.array([0.95, 0.9, 0.2, 0.99, 0.5])
+    masked = np.array([True, True, True, False, True])
+    c = O.threshold_commit(conf, masked, 0.9)
+    assert c.tolist() == [True, False, False, False, False]      # 0.9 does not clear 0.9
+    c = O.threshold_commit(np.array([0.1, 0.3, 0.3, 0.2]), np.ones(4, bool), 0.9)
+    assert c.tolist() == [False, True, False, False]              # forced, lowest position on tie
+
+
+def test_commit_tau_above_one_commits_exactly_one():
+    for _ in range(50):
+        conf = RNG.uniform(0, 1, 16)
+        masked = RNG.uniform(size=16) < 0.6
+        masked[RNG.integers(16)] = True
+        c = O.threshold_commit(conf, masked, 1.5)
+        assert c.sum() == 1 and masked[c].all()
+        assert np.argmax(np.where(masked, conf, -1)) == np.where(c)[0][0]
+
+
+def test_commit_tiny_tau_commits_all_masked():
+    conf = RNG.uniform(1e-3, 1, 16)
+    masked = RNG.uniform(size=16) < 0.5
+    masked[0] = True
+    c = O.threshold_commit(conf, masked, 1e-6)
+    assert np.array_equal(c, masked)
+
+
+def test_commit_nothing_masked_commits_nothing():
+    assert not O.threshold_commit(np.ones(4), np.zeros(4, bool), 0.9).any()
+
+
+# ---------------------------------------------------------------- key sets
+def test_key_positions_modes():
+    S, B, W = 100, 8, 5
+    assert O.key_positions(O.MODE_PREFIX, 40, B, S, W, 0).tolist() == list(range(48))
+    assert O.key_positions(O.MODE_NONE, 40, B, S, W, 3).tolist() == list(range(3, 48))
+    assert O.key_positions(O.MODE_DUAL, 40, B, S, W, 2).tolist() == list(range(2, 100))
+    assert O.key_positions(O.MODE_DUAL_PRUNED, 40, B, S, W, 0).tolist() == \
+        list(range(53)) + [99]
+    # window reaching the trailing position: not duplicated
+    assert O.key_positions(O.MODE_DUAL_PRUNED, 88, B, S, W, 0).tolist() == list(range(100))
+    # window clipped at S
+    assert O.key_positions(O.MODE_DUAL_PRUNED, 90, B, S, 50, 0).tolist() == list(range(100))
+    # last block: empty suffix
+    assert O.key_positions(O.MODE_DUAL_PRUNED, 92, B, S, W, 0).tolist() == list(range(100))
+
+
+def test_pruned_with_large_window_equals_dual():
+    for s in range(0, 96, 8):
+        np.testing.assert_array_equal(O.key_positions(O.MODE_DUAL_PRUNED, s, 8, 96, 96, 4),
+                                      O.key_positions(O.MODE_DUAL, s, 8, 96, 96, 4))
+
+
+# ---------------------------------------------------------------- whole decode
+TINY = wl.WORKLOADS["tiny"]
+
+
+@pytest.fixture(scope="module")
+def tiny_prefix():
+    return Case(TINY)
+
+
+def test_tiny_decode_invariants(tiny_prefix):
+    case = tiny_prefix
+    tr = case.decode()
+    B = TINY.block
+    assert not (tr.tokens[:, TINY.prompt_len:] < 0).any()
+    # never re-masked; committed tokens never change; every block commits B rows
+    seen_tok = {}
+    per_block = {}
+    for s, r in tr.steps:
+        per_block[s] = per_block.get(s, 0) + int(r.commit.sum())
+        for (bi, i) in zip(*np.where(r.commit)):
+            key = (bi, s + i)
+            assert key not in seen_tok
+            seen_tok[key] = r.tok[bi, i]
+        conf = r.conf[~np.isnan(r.conf)]
+        assert np.all((conf > 0) & (conf <= 1))
+    assert all(v == B for v in per_block.values())
+    for (bi, p), t in seen_tok.items():
+        assert tr.tokens[bi, p] == t
+    assert np.array_equal(tr.tokens[:, :TINY.prompt_len], case.tokens.numpy()[:, :TINY.prompt_len])
+    # prompt and step counts: each step commits >= 1
+    assert all(1 <= n <= B for n in tr.steps_per_block)
+
+
+def test_tiny_confidence_spread(tiny_prefix):
+    # the planted states spread confidences from ~1/V to ~1 and some clear tau
+    tr = tiny_prefix.decode()
+    c = np.concatenate([r.conf[~np.isnan(r.conf)] for _, r in tr.steps])
+    assert c.min() < 0.05 and c.max() > 0.95
+    assert (c > TINY.tau).sum() >= 3
+
+
+def test_prefix_cache_equals_no_cache_at_one_layer():
+    # one layer: keys/values of settled positions depend only on their
+    # embedding, so the cached decode must reproduce the full recompute.
+    a = Case(TINY.replace(mode=wl.MODE_PREFIX)).decode()
+    b = Case(TINY.replace(mode=wl.MODE_NONE)).decode()
+    assert np.array_equal(a.tokens, b.tokens)
+    assert a.steps_per_block == b.steps_per_block
+    for (sa, ra), (sb, rb) in zip(a.steps, b.steps):
+        assert sa == sb
+        np.testing.assert_allclose(ra.conf, rb.conf, atol=1e-12, equal_nan=True)
+        assert np.array_equal(ra.commit, rb.commit)
+
+
+def test_dual_step_equals_fresh_full_forward_at_one_layer():
+    # DualCache, first step of block 0: the cache from prefill must give the
+    # same block output as a forward over the whole sequence built from scratch
+    w = TINY.replace(mode=wl.MODE_DUAL)
+    case = Case(w)
+    cfg, W = case.cfg, case.W
+    st = O.new_state(cfg, case.tokens.numpy(), case.masked.numpy().astype(bool),
+                     case.starts.numpy())
+    O.prefill(cfg, W, st)
+    s = w.prompt_len
+    r = O.decode_step(cfg, W, st, case.plants64, s, apply=False)
+    S = w.seq_len
+    x0 = W.embed(case.tokens.numpy()[:, :S])
+    x0[:, s:s + w.block] = case.plants64[:, :w.block]
+    shape = (cfg.n_layers, 1, cfg.n_kv_heads, S, cfg.head_dim)
+    kc, vc = np.zeros(shape), np.zeros(shape)
+    x = O.forward_rows(cfg, W, x0, np.arange(S), [np.arange(S)], kc, vc, np.zeros(1, int), True)
+    np.testing.assert_allclose(r.hidden, x[:, s:s + w.block], rtol=0, atol=1e-9)
+
+
+def test_tau_above_one_takes_block_steps_in_confidence_order():
+    w = TINY.replace(tau=1.5, gen_len=16)
+    tr = Case(w).decode()
+    assert tr.steps_per_block == [w.block] * (w.gen_len // w.block)
+    for s, r in tr.steps:
+        assert r.commit.sum() == 1
+        m = ~np.isnan(r.conf[0])
+        best = np.where(m)[0][np.argmax(r.conf[0][m])]
+        assert r.commit[0, best]
+
+
+def test_tau_below_one_over_v_takes_one_step_per_block():
+    w = TINY.replace(tau=0.5 / TINY.vocab)
+    tr = Case(w).decode()
+    assert tr.steps_per_block == [1] * (w.gen_len // w.block)
+
+
+def test_strong_plant_decodes_planted_token():
+    # a = 50 and no noise: the target logit dominates, token = t
+    w = TINY.replace(plant_a_max=50.0)
+    case = Case(w, a_override=50.0, noise=False)
+    r = case.decode(max_steps=1).steps[0][1]
+    assert np.array_equal(r.tok[0], case.plants.t.numpy()[0, :w.block])
+
+
+def test_gqa_equals_mha_with_repeated_kv_heads():
+    # GQA with g = Hq/Hkv must equal MHA whose k/v weights repeat each kv head g times
+    w = TINY.replace(n_q_heads=4, n_kv_heads=2, gen_len=8, rope_theta=1e4)
+    case = Case(w)
+    D, Hq, Hkv = w.head_dim, w.n_q_heads, w.n_kv_heads
+    g = Hq // Hkv
+    wq = case.weights.wqkv[:, :Hq * D]
+    wk = case.weights.wqkv[:, Hq * D:(Hq + Hkv) * D].reshape(w.n_layers, Hkv, D, w.hidden)
+    wv = case.weights.wqkv[:, (Hq + Hkv) * D:].reshape(w.n_layers, Hkv, D, w.hidden)
+    wk_r = wk.repeat_interleave(g, dim=1).reshape(w.n_layers, Hq * D, w.hidden)
+    wv_r = wv.repeat_interleave(g, dim=1).reshape(w.n_layers, Hq * D, w.hidden)
+    mha_w = w.replace(n_kv_heads=Hq)
+    mha = Case(mha_w)
+    mha.weights.wqkv = torch.cat([wq, wk_r, wv_r], dim=1)
+    mha.weights.wo = case.weights.wo
+    mha.weights.w_lm = case.weights.w_lm
+    from tests.oracle_inputs import oracle_weights
+    mha.W = oracle_weights(mha.weights)
+    mha.plants64 = case.plants64
+    a, b = case.decode(), mha.decode()
+    assert np.array_equal(a.tokens, b.tokens)
+    for (_, ra), (_, rb) in zip(a.steps, b.steps):
+        np.testing.assert_allclose(ra.conf, rb.conf, atol=1e-12, equal_nan=True)
+
+
+def test_batch_sequences_independent_with_left_padding():
+    # two sequences with different prompt lengths, left-padded to the longest:
+    # each must decode exactly as it does alone without padding (RoPE on)
+    w = TINY.replace(batch=3, prompt_len=64, prompt_len_min=40, rope_theta=1e4,
+                     mode=wl.MODE_DUAL, gen_len=16)
+    case = Case(w)
+    tr = case.decode()
+    starts = case.starts.numpy()
+    assert len(set(starts.tolist())) > 1
+    for bi in range(w.batch):
+        st = int(starts[bi])
+        wa = w.replace(batch=1, prompt_len=w.prompt_len - st, prompt_len_min=None)
+        alone = Case(wa)
+        alone.tokens = case.tokens[bi:bi + 1, st:].clone()
+        alone.masked = case.masked[bi:bi + 1, st:].clone()
+        alone.starts = torch.zeros(1, dtype=torch.int32)
+        alone.plants64 = alone.plants64 * 0 + case.plants64[bi:bi + 1]
+        ta = alone.decode()
+        np.testing.assert_array_equal(ta.tokens[0], tr.tokens[bi, st:])
+
+
+def test_pruned_large_window_decode_equals_dual():
+    w = TINY.replace(mode=wl.MODE_DUAL, gen_len=24)
+    a = Case(w).decode()
+    b = Case(w.replace(mode=wl.MODE_DUAL_PRUNED, window=w.gen_len)).decode()
+    assert np.array_equal(a.tokens, b.tokens)
+    for (_, ra), (_, rb) in zip(a.steps, b.steps):
+        np.testing.assert_allclose(ra.conf, rb.conf, atol=1e-12, equal_nan=True)
+
+
+def test_pruned_small_window_differs_from_dual():
+    # the pruned key set is really smaller: confidences change
+    w = TINY.replace(mode=wl.MODE_DUAL, gen_len=32)
+    a = Case(w).decode(max_steps=1)
+    b = Case(w.replace(mode=wl.MODE_DUAL_PRUNED, window=4)).decode(max_steps=1)
+    assert np.abs(np.nan_to_num(a.steps[0][1].conf) - np.nan_to_num(b.steps[0][1].conf)).max() > 1e-9
+
+
+def test_refresh_writes_committed_block_kv():
+    # after a block is done, its cache rows are the keys/values of its
+    # committed tokens (one layer: k = Wk E[token], rounded to bf16)
+    w = TINY.replace(mode=wl.MODE_PREFIX, gen_len=8)
+    case = Case(w)
+    cfg, W = case.cfg, case.W
+    st = O.new_state(cfg, case.tokens.numpy(), case.masked.numpy().astype(bool),
+                     case.starts.numpy())
+    O.prefill(cfg, W, st)
+    s = w.prompt_len
+    while st.masked[:, s:s + w.block].any():
+        O.decode_step(cfg, W, st, case.plants64, s)
+    O.refresh_block(cfg, W, st, s)
+    D, Hq, Hkv = w.head_dim, w.n_q_heads, w.n_kv_heads
+    x = O.round_bf16(W.embed(st.tokens[0, s:s + w.block]))
+    k = x @ W.wqkv(0)[Hq * D:(Hq + Hkv) * D].T
+    want = O.round_bf16(k.reshape(w.block, Hkv, D).transpose(1, 0, 2))
+    np.testing.assert_array_equal(st.kcache[0, 0][:, s:s + w.block], want)
