@@ -1,0 +1,385 @@
+"""Benchmark of the block-decode hot path on B200.
+
+One "step" is one whole generation of the workload after the inputs are in
+HBM: reset tokens and mask, prefill the cache, then decode every block to
+completion (threshold-commit steps plus the cache refresh of each block).
+value = committed tokens per second over the timed steps (all ranks).
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                       [--impl ours|reference]
+For N > 1 launch one process per GPU with torch.distributed.run; each rank
+decodes its own copy of the workload (independent sequences, no exchange).
+``--impl reference`` times the fp64 CPU oracle on this host instead.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes as C
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = ("committed tokens/s & decode-step µs at 1 B200; "
+          "HBM GB/s / tensor-pipe % of peak")
+DEFAULT_WORKLOAD = "llada8b_dual"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+def workload_config(w, data_note):
+    return {"workload": w.name, "batch": w.batch, "layers": w.n_layers, "hidden": w.hidden,
+            "heads": f"{w.n_q_heads}/{w.n_kv_heads}x{w.head_dim}", "vocab": w.vocab,
+            "prompt_len": w.prompt_len, "gen_len": w.gen_len, "block": w.block, "tau": w.tau,
+            "cache": ["none", "prefix", "dual", "dual_pruned"][w.mode],
+            "l2": data_note}
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    def __init__(self, index: int):
+        self.path = tempfile.mktemp(prefix="clocks_", suffix=".csv")
+        q = ("clocks.sm,clocks.max.sm,utilization.gpu,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+        try:
+            self.f = open(self.path, "w")
+            self.p = subprocess.Popen(["nvidia-smi", "-i", str(index), f"--query-gpu={q}",
+                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except Exception:
+            self.p.kill()
+        self.f.close()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 7:
+                try:
+                    rows.append((float(parts[0]), float(parts[1]), float(parts[2]), parts[3:7]))
+                except ValueError:
+                    pass
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        loaded = [r for r in rows if r[2] > 0] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[3])
+                          if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(loaded)}
+
+
+# ---------------------------------------------------------------- oracle timing
+def oracle_sample(w, weights, tokens, masked, starts, plants, budget_s=20.0):
+    """Time the fp64 oracle on this host: denoising steps of the first block,
+    from the prefilled state where the workload is small enough, else from
+    zero caches (the step's arithmetic does not depend on the cache values).
+    Returns (seconds per step, steps, rows committed, threads)."""
+    import numpy as np
+    import torch
+    from oracle import dllm_oracle as O
+
+    cfg = O.Config(batch=w.batch, n_layers=w.n_layers, hidden=w.hidden, n_q_heads=w.n_q_heads,
+                   n_kv_heads=w.n_kv_heads, head_dim=w.head_dim, vocab=w.vocab,
+                   prompt_len=w.prompt_len, gen_len=w.gen_len, block=w.block, tau=w.tau,
+                   mode=w.mode, window=w.window, rope_theta=w.rope_theta, mask_id=w.mask_id)
+    W = O.Weights(lambda l: weights.wqkv[l].cpu().double().numpy(),
+                  lambda l: weights.wo[l].cpu().double().numpy(),
+                  weights.w_lm.cpu().double().numpy())
+    st = O.new_state(cfg, tokens.numpy(), masked.numpy().astype(bool), starts.numpy())
+    small = w.n_layers * w.hidden * w.hidden <= 64 * 1024 * 1024
+    if small:
+        O.prefill(cfg, W, st)
+    plants64 = plants.h.double().cpu().numpy()
+    s = w.prompt_len
+    t0 = time.perf_counter()
+    n, committed = 0, 0
+    while st.masked[:, s:s + w.block].any():
+        r = O.decode_step(cfg, W, st, plants64, s)
+        n += 1
+        committed += int(r.commit.sum())
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return dt / n, n, committed, torch.get_num_threads()
+
+
+def run_reference(args, rank, world):
+    """The oracle as it stands on this host's cores, for the same workload."""
+    if rank != 0:
+        return
+    import torch
+    from diffusion_decoding_step_b200 import workload as wl
+    w = wl.WORKLOADS[args.workload]
+    weights = wl.make_weights(w, device="cpu")
+    tokens, masked = wl.make_tokens(w)
+    starts = wl.seq_starts(w)
+    plants = wl.make_plants(w, weights.w_lm)
+    step_s = []
+    commits = 0
+    steps = 0
+    for _ in range(args.warmup):
+        oracle_sample(w, weights, tokens, masked, starts, plants, budget_s=5.0)
+    for _ in range(args.steps):
+        sp, n, c, thr = oracle_sample(w, weights, tokens, masked, starts, plants, budget_s=20.0)
+        step_s.append(sp * n)
+        commits += c
+        steps += n
+    total = sum(step_s)
+    value = commits / total
+    sample = (f"first block of {w.name}: {steps} oracle denoising steps over {args.steps} "
+              f"timed samples (each <= 20 s), {commits} rows committed")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000.0 * total / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(w, "cpu"),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": thr, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- our path
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from diffusion_decoding_step_b200 import abi, build
+    from diffusion_decoding_step_b200 import workload as wl
+    from diffusion_decoding_step_b200.runtime import Decoder, _ptr
+
+    build.build()
+    abi.lib()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = wl.WORKLOADS[args.workload]
+    weights = wl.make_weights(w, device=dev)
+    tokens, masked = wl.make_tokens(w)
+    starts = wl.seq_starts(w)
+    plants = wl.make_plants(w, weights.w_lm)
+    dec = Decoder(w, weights, tokens, masked, starts, plants, device=str(dev))
+    stream = dec.stream
+
+    def generation():
+        dec.reset()
+        dec.prefill()
+        n = 0
+        for s in range(w.prompt_len, w.seq_len, w.block):
+            n += dec.decode_block(s)
+        return n
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        generation()
+    barrier()
+    clocks = ClockSampler(local_rank) if rank == 0 else None
+    launches0 = abi.dllm_launch_count()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    denoise_steps = 0
+    for _ in range(args.steps):
+        denoise_steps += generation()
+    e1.record(stream)
+    barrier()
+    launches = abi.dllm_launch_count() - launches0
+    clk = clocks.stop() if clocks else None
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t)
+    tokens_total = world * w.batch * w.gen_len * args.steps
+    value = tokens_total / (ms / 1000.0)
+    assert dec.device_status() == 0
+    assert not bool(dec.masked.any())
+
+    # prefill share and per-step latency (separate untimed measurement)
+    p0 = torch.cuda.Event(enable_timing=True)
+    p1 = torch.cuda.Event(enable_timing=True)
+    dec.reset()
+    p0.record(stream)
+    dec.prefill()
+    p1.record(stream)
+    torch.cuda.synchronize(dev)
+    prefill_ms = p0.elapsed_time(p1)
+    step_us = []
+    s = w.prompt_len
+    for _ in range(min(6, w.block)):
+        a = torch.cuda.Event(enable_timing=True)
+        b_ = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        dec.step(s)
+        b_.record(stream)
+        torch.cuda.synchronize(dev)
+        step_us.append(1000.0 * a.elapsed_time(b_))
+
+    # dominant kernel: the Q/K/V projection of one layer, same launch shape as a step
+    hbm, tflops, peak_kind = peaks()
+    rows = w.batch * w.block
+    cfg_p = C.byref(dec.cfg)
+    q = torch.empty(rows * w.n_q_heads * w.head_dim, dtype=torch.bfloat16, device=dev)
+    xb = torch.randn(rows, w.hidden, device=dev).to(torch.bfloat16)
+    sh = C.c_void_p(stream.cuda_stream)
+    iters = 3 * w.n_layers
+    for _ in range(2):
+        for l in range(w.n_layers):
+            abi.check(abi.dllm_qkv_proj(cfg_p, C.byref(dec.weights_c), l, _ptr(xb), s, w.block,
+                                        _ptr(dec.seq_start), _ptr(q), _ptr(dec.k_cache),
+                                        _ptr(dec.v_cache), _ptr(dec.ws), dec.ws_bytes, sh), "qkv")
+    k0 = torch.cuda.Event(enable_timing=True)
+    k1 = torch.cuda.Event(enable_timing=True)
+    k0.record(stream)
+    for i in range(iters):
+        abi.check(abi.dllm_qkv_proj(cfg_p, C.byref(dec.weights_c), i % w.n_layers, _ptr(xb), s,
+                                    w.block, _ptr(dec.seq_start), _ptr(q), _ptr(dec.k_cache),
+                                    _ptr(dec.v_cache), _ptr(dec.ws), dec.ws_bytes, sh), "qkv")
+    k1.record(stream)
+    torch.cuda.synchronize(dev)
+    qkv_ms = k0.elapsed_time(k1) / iters
+    kv_bytes = 2 * rows * w.n_kv_heads * w.head_dim * 2
+    qkv_bytes = (w.qkv_rows * w.hidden * 2 + rows * w.hidden * 2
+                 + rows * w.n_q_heads * w.head_dim * 2 + kv_bytes)
+    achieved = qkv_bytes / (qkv_ms / 1000.0) / 1e9
+    traffic = None
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            traffic = json.load(f).get(f"{w.name}:qkv_proj")
+    except Exception:
+        pass
+
+    # end to end through the C ABI with host buffers: inputs copied in from
+    # pinned memory, result copied out, every step
+    h_tokens = tokens.to(torch.int32).pin_memory()
+    h_masked = masked.to(torch.uint8).pin_memory()
+    h_plants = plants.h.to("cpu").pin_memory()
+    h_out = torch.empty_like(h_tokens).pin_memory()
+    h2d = h_tokens.numel() * 4 + h_masked.numel() + h_plants.numel() * 2
+    d2h = h_out.numel() * 4
+
+    def e2e_generation():
+        dec.tokens.copy_(h_tokens, non_blocking=True)
+        dec.masked.copy_(h_masked, non_blocking=True)
+        dec.plants.copy_(h_plants, non_blocking=True)
+        dec.prefill()
+        for s_ in range(w.prompt_len, w.seq_len, w.block):
+            dec.decode_block(s_)
+        h_out.copy_(dec.tokens, non_blocking=True)
+
+    e2e_generation()
+    barrier()
+    x0 = torch.cuda.Event(enable_timing=True)
+    x1 = torch.cuda.Event(enable_timing=True)
+    x0.record(stream)
+    for _ in range(args.steps):
+        e2e_generation()
+    x1.record(stream)
+    barrier()
+    e2e_ms = x0.elapsed_time(x1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t)
+    e2e_value = tokens_total / (e2e_ms / 1000.0)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        wc = weights
+        sp, n, c, thr = oracle_sample(w, wc, tokens, masked, starts, plants, budget_s=20.0)
+        per_step_commit = w.batch * w.gen_len * args.steps / max(1, denoise_steps)
+        cpu = {"value": per_step_commit / sp, "unit": "tokens/s", "cores": thr,
+               "kind": "oracle",
+               "sample": (f"{n} oracle denoising steps of the first block of {w.name} "
+                          f"({sp:.2f} s each, fp64); tokens/s = the GPU run's mean commits per "
+                          f"step ({per_step_commit:.2f}) / oracle step time")}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": workload_config(w, "inputs larger than L2 (weights stream from HBM)"),
+            "decode_step_us": {"mean": (ms * 1000.0) / denoise_steps,
+                               "isolated_p50": statistics.median(step_us),
+                               "isolated_max": max(step_us)},
+            "denoising_steps_per_generation": denoise_steps / args.steps,
+            "prefill_ms": prefill_ms,
+            "roofline": {"bound": "hbm", "kernel": "qkv_proj (tcgen05 GEMM, fused RoPE + "
+                         "cache write)", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                         "frac": achieved / hbm, "traffic": traffic,
+                         "peak_kind": peak_kind, "launch_us": qkv_ms * 1000.0,
+                         "algorithmic_bytes": qkv_bytes},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": int(launches),
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

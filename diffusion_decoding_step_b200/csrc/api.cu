@@ -1,0 +1,804 @@
+// C-ABI entry points: argument checks, workspace layout, TMA descriptors,
+// work partitioning and the launch sequence of a decode step.
+#include <cudaTypedefs.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <vector>
+
+#include "../../include/dllm.h"
+#include "kernels.cuh"
+
+namespace dllm {
+unsigned long long launch_count();
+}
+
+using namespace dllm;
+
+namespace {
+
+// ------------------------------------------------------------------ helpers
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 3-D bf16 tensor map: dims {d0 (innermost), d1, d2}, box {b0, b1, 1}.
+bool make_map(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0,
+              uint32_t b1, CUtensorMapSwizzle sw) {
+  auto fn = encode_fn();
+  if (!fn || !ptr) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  cuuint32_t box[3] = {b0, b1, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
+                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ shapes
+struct Shape {
+  int b, L, d, Hq, Hkv, D, V, P, G, B, S, W, mode, wfmt;
+  int qkv_rows, Kw, Ko;
+  float tau, theta;
+  int mask_id;
+};
+
+dllm_status check_cfg(const dllm_config* c, Shape* s) {
+  if (!c) return DLLM_ERR_INVALID;
+  if (c->batch < 1 || c->n_layers < 1 || c->hidden < 1 || c->n_q_heads < 1 ||
+      c->n_kv_heads < 1 || c->head_dim < 1 || c->vocab < 2 || c->prompt_len < 0 ||
+      c->gen_len < 1 || c->block < 1)
+    return DLLM_ERR_INVALID;
+  if (c->mode < DLLM_CACHE_NONE || c->mode > DLLM_CACHE_DUAL_PRUNED) return DLLM_ERR_INVALID;
+  if (c->weight_format != DLLM_W_BF16 && c->weight_format != DLLM_W_F32_SPLIT)
+    return DLLM_ERR_INVALID;
+  if (c->n_q_heads % c->n_kv_heads) return DLLM_ERR_INVALID;
+  if (c->gen_len % c->block) return DLLM_ERR_INVALID;
+  if (c->mode == DLLM_CACHE_DUAL_PRUNED && c->window < 0) return DLLM_ERR_INVALID;
+  if (c->mask_id < 0 || c->mask_id >= c->vocab) return DLLM_ERR_INVALID;
+  if (!(c->tau == c->tau) || c->rope_theta < 0.f) return DLLM_ERR_INVALID;
+  if (c->head_dim != 32 && c->head_dim != 128) return DLLM_ERR_UNSUPPORTED;
+  const int qkv = (c->n_q_heads + 2 * c->n_kv_heads) * c->head_dim;
+  if (c->hidden % 128 || (c->n_q_heads * c->head_dim) % 128 || qkv % 128 || c->vocab % 128)
+    return DLLM_ERR_UNSUPPORTED;
+  if (c->block > 64 || c->batch > 1024) return DLLM_ERR_UNSUPPORTED;
+  s->b = c->batch;
+  s->L = c->n_layers;
+  s->d = c->hidden;
+  s->Hq = c->n_q_heads;
+  s->Hkv = c->n_kv_heads;
+  s->D = c->head_dim;
+  s->V = c->vocab;
+  s->P = c->prompt_len;
+  s->G = c->gen_len;
+  s->B = c->block;
+  s->S = c->prompt_len + c->gen_len;
+  s->W = c->window;
+  s->mode = c->mode;
+  s->wfmt = c->weight_format;
+  s->qkv_rows = qkv;
+  const int f = c->weight_format == DLLM_W_F32_SPLIT ? 2 : 1;
+  s->Kw = f * c->hidden;
+  s->Ko = f * c->n_q_heads * c->head_dim;
+  s->tau = c->tau;
+  s->theta = c->rope_theta;
+  s->mask_id = c->mask_id;
+  return DLLM_OK;
+}
+
+// ------------------------------------------------------------------ partitioning
+struct GemmPlan {
+  int nt, m_tiles, n_tiles, splits, kbps, units, grid;
+};
+
+GemmPlan plan_gemm(int M, int R, int K, bool allow_split) {
+  GemmPlan g;
+  g.nt = R <= 32 ? 32 : R <= 64 ? 64 : R <= 128 ? 128 : 256;
+  g.n_tiles = cdiv(R, g.nt);
+  g.m_tiles = M / 128;
+  const int tiles = g.m_tiles * g.n_tiles;
+  const int kbt = K / 64;
+  int best_s = 1, best_kbps = kbt;
+  double best_cost = 1e30;
+  const int max_s = allow_split ? std::min(32, kbt) : 1;
+  for (int s = 1; s <= max_s; ++s) {
+    const int kbps = cdiv(kbt, s);
+    const int se = cdiv(kbt, kbps);
+    if (se != s) continue;
+    const int units = tiles * se;
+    const int per_cta = cdiv(units, kNumSMs);
+    const double cost = (double)per_cta * kbps + 1.0 * per_cta + (se > 1 ? 1.0 : 0.0);
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best_s = se;
+      best_kbps = kbps;
+    }
+  }
+  g.splits = best_s;
+  g.kbps = best_kbps;
+  g.units = tiles * best_s;
+  g.grid = std::min(g.units, kNumSMs);
+  return g;
+}
+
+GemmPlan plan_lmhead(int V, int R, int K) {
+  GemmPlan g = plan_gemm(V, R, K, false);
+  int grid = std::min(g.units, kNumSMs);
+  grid = std::max(g.n_tiles, grid / g.n_tiles * g.n_tiles);
+  g.grid = grid;
+  return g;
+}
+
+struct AttnPlan {
+  int row_tiles, chunks, tpc;
+};
+
+AttnPlan plan_attn(const Shape& s, int n_rows, int ntile_bound) {
+  AttnPlan a;
+  const int g = s.Hq / s.Hkv;
+  a.row_tiles = cdiv(g * n_rows, 128);
+  const int base = s.b * s.Hkv * a.row_tiles;
+  int chunks = std::max(1, std::min(ntile_bound, cdiv(kNumSMs, base)));
+  if (base >= kNumSMs) chunks = 1;
+  a.tpc = cdiv(ntile_bound, chunks);
+  a.chunks = cdiv(ntile_bound, a.tpc);
+  return a;
+}
+
+// Upper bound of key tiles of a sequence for a block at blk (first valid
+// position 0), or for a plain range [0, seg_end) when seg_end > 0.
+int key_tiles_bound(const Shape& s, int blk, int seg_end) {
+  if (seg_end > 0) return cdiv(seg_end, 128);
+  const int end = blk + s.B;
+  switch (s.mode) {
+    case DLLM_CACHE_DUAL: return cdiv(s.S, 128);
+    case DLLM_CACHE_DUAL_PRUNED: {
+      const int wend = std::min(end + s.W, s.S);
+      return cdiv(wend, 128) + ((end < s.S && s.S - 1 >= wend) ? 1 : 0);
+    }
+    default: return cdiv(end, 128);
+  }
+}
+
+// ------------------------------------------------------------------ workspace
+struct Layout {
+  size_t status, gcnt, acnt, x, xb, q, attn, h, slots, stats, part_o, part_ml, conf, tok, gap,
+      commit, remaining, segs, rope, total;
+  int rmax, lm_slots, gcnt_n, acnt_n;
+};
+
+// Row counts (per sequence) a configuration uses: decode steps and prefill.
+std::vector<int> row_counts(const Shape& s) {
+  std::vector<int> r;
+  if (s.mode == DLLM_CACHE_NONE) {
+    for (int blk = s.P; blk < s.S; blk += s.B) r.push_back(blk + s.B);
+  } else {
+    r.push_back(s.B);
+    r.push_back(s.mode == DLLM_CACHE_PREFIX ? std::max(s.P, 1) : s.S);
+  }
+  return r;
+}
+
+Layout layout(const Shape& s) {
+  Layout l{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  const std::vector<int> rows = row_counts(s);
+  int max_rows = 0;
+  size_t slot_bytes = 0;
+  int gtiles = 1;
+  size_t part_rows = 0;
+  int acnt = 1;
+  for (int n : rows) {
+    max_rows = std::max(max_rows, n);
+    const int R = s.b * n;
+    const GemmPlan gq = plan_gemm(s.qkv_rows, R, s.Kw, true);
+    const GemmPlan go = plan_gemm(s.d, R, s.Ko, true);
+    for (const GemmPlan& g : {gq, go}) {
+      if (g.splits > 1) slot_bytes = std::max(slot_bytes, (size_t)g.units * g.nt * 128 * 4);
+      gtiles = std::max(gtiles, g.m_tiles * g.n_tiles);
+    }
+  }
+  // attention partials: every decode step, plus the unit-level entry point
+  // (block rows against up to ceil(S/128)+1 key tiles)
+  auto need_attn = [&](int n_rows, int ntb) {
+    const AttnPlan a = plan_attn(s, n_rows, ntb);
+    if (a.chunks > 1)
+      part_rows = std::max(part_rows, (size_t)s.b * s.Hkv * a.row_tiles * a.chunks * 128);
+    acnt = std::max(acnt, s.b * s.Hkv * a.row_tiles);
+  };
+  for (int blk = s.P; blk < s.S; blk += s.B) {
+    if (s.mode == DLLM_CACHE_NONE)
+      need_attn(blk + s.B, key_tiles_bound(s, blk, blk + s.B));
+    else
+      need_attn(s.B, key_tiles_bound(s, blk, 0));
+  }
+  need_attn(s.B, cdiv(s.S, 128) + 1);
+  l.rmax = s.b * max_rows;
+  const GemmPlan gl = plan_lmhead(s.V, s.b * s.B, s.Kw);
+  l.lm_slots = gl.grid / gl.n_tiles;
+  l.gcnt_n = gtiles;
+  l.acnt_n = acnt;
+  l.status = take(256);
+  l.gcnt = take((size_t)gtiles * 4);
+  l.acnt = take((size_t)acnt * 4);
+  l.x = take((size_t)l.rmax * s.d * 4);
+  l.xb = take((size_t)l.rmax * s.d * 2);
+  l.q = take((size_t)l.rmax * s.Hq * s.D * 2);
+  l.attn = take((size_t)l.rmax * s.Hq * s.D * 2);
+  l.h = take((size_t)s.b * s.B * s.d * 2);
+  l.slots = take(std::max<size_t>(slot_bytes, 256));
+  l.stats = take((size_t)s.b * s.B * l.lm_slots * sizeof(LmStat));
+  l.part_o = take(std::max<size_t>(part_rows * s.D * 4, 256));
+  l.part_ml = take(std::max<size_t>(part_rows * 8, 256));
+  l.conf = take((size_t)s.b * s.B * 4);
+  l.tok = take((size_t)s.b * s.B * 4);
+  l.gap = take((size_t)s.b * s.B * 4);
+  l.commit = take((size_t)s.b * s.B);
+  l.remaining = take((size_t)s.b * 4);
+  l.segs = take((size_t)s.b * 16);
+  l.rope = take(s.theta > 0.f ? (size_t)s.S * (s.D / 2) * 8 : 256);
+  l.total = off;
+  return l;
+}
+
+// ------------------------------------------------------------------ context
+struct Ctx {
+  Shape s;
+  Layout l;
+  uint8_t* ws;
+  cudaStream_t st;
+  template <class T>
+  T* at(size_t off) const {
+    return reinterpret_cast<T*>(ws + off);
+  }
+};
+
+dllm_status make_ctx(const dllm_config* cfg, void* ws, size_t ws_bytes, dllm_stream stream,
+                     Ctx* c) {
+  dllm_status e = check_cfg(cfg, &c->s);
+  if (e != DLLM_OK) return e;
+  if (!ws) return DLLM_ERR_INVALID;
+  c->l = layout(c->s);
+  if (ws_bytes < c->l.total) return DLLM_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(ws) % 256) return DLLM_ERR_INVALID;
+  c->ws = static_cast<uint8_t*>(ws);
+  c->st = reinterpret_cast<cudaStream_t>(stream);
+  return DLLM_OK;
+}
+
+dllm_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DLLM_OK : DLLM_ERR_CUDA; }
+
+#define DLLM_TRY(x)                       \
+  do {                                    \
+    dllm_status _e = (x);                 \
+    if (_e != DLLM_OK) return _e;         \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ------------------------------------------------------------------ launches
+dllm_status run_qkv(const Ctx& c, const void* wqkv, int layer, const void* xb, int row0,
+                    int n_rows, const int* seq_start, void* q_out, void* kc, void* vc, bool pdl) {
+  const Shape& s = c.s;
+  const int R = s.b * n_rows;
+  const GemmPlan g = plan_gemm(s.qkv_rows, R, s.Kw, true);
+  CUtensorMap wm, xm;
+  if (!make_map(&wm, wqkv, s.Kw, s.qkv_rows, s.L, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&xm, xb, s.d, R, 1, 64, g.nt, CU_TENSOR_MAP_SWIZZLE_128B))
+    return DLLM_ERR_CUDA;
+  GemmParams p{};
+  p.M = s.qkv_rows;
+  p.R = R;
+  p.K = s.Kw;
+  p.kx_blocks = s.d / 64;
+  p.m_tiles = g.m_tiles;
+  p.n_tiles = g.n_tiles;
+  p.splits = g.splits;
+  p.kb_per_split = g.kbps;
+  p.units = g.units;
+  p.layer = layer;
+  p.status = c.at<int>(c.l.status);
+  p.slots = c.at<float>(c.l.slots);
+  p.counters = c.at<int>(c.l.gcnt);
+  p.n_rows = n_rows;
+  p.row0 = row0;
+  p.seq_start = seq_start;
+  p.Hq = s.Hq;
+  p.Hkv = s.Hkv;
+  p.D = s.D;
+  p.S = s.S;
+  p.batch = s.b;
+  p.rope_tab = s.theta > 0.f ? c.at<float2>(c.l.rope) : nullptr;
+  p.q_out = static_cast<__nv_bfloat16*>(q_out);
+  p.k_cache = static_cast<__nv_bfloat16*>(kc);
+  p.v_cache = static_cast<__nv_bfloat16*>(vc);
+  return cuda_status(launch_gemm(EPI_QKV, g.nt, wm, xm, p, g.grid, pdl, c.st));
+}
+
+dllm_status run_oproj(const Ctx& c, const void* wo, int layer, const void* attn, int row0,
+                      int n_rows, float* x, void* xb, void* h_out, int blk_start, bool pdl) {
+  const Shape& s = c.s;
+  const int R = s.b * n_rows;
+  const GemmPlan g = plan_gemm(s.d, R, s.Ko, true);
+  CUtensorMap wm, xm;
+  if (!make_map(&wm, wo, s.Ko, s.d, s.L, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&xm, attn, s.Hq * s.D, R, 1, 64, g.nt, CU_TENSOR_MAP_SWIZZLE_128B))
+    return DLLM_ERR_CUDA;
+  GemmParams p{};
+  p.M = s.d;
+  p.R = R;
+  p.K = s.Ko;
+  p.kx_blocks = s.Hq * s.D / 64;
+  p.m_tiles = g.m_tiles;
+  p.n_tiles = g.n_tiles;
+  p.splits = g.splits;
+  p.kb_per_split = g.kbps;
+  p.units = g.units;
+  p.layer = layer;
+  p.status = c.at<int>(c.l.status);
+  p.slots = c.at<float>(c.l.slots);
+  p.counters = c.at<int>(c.l.gcnt);
+  p.n_rows = n_rows;
+  p.row0 = row0;
+  p.x = x;
+  p.xb = static_cast<__nv_bfloat16*>(xb);
+  p.d_model = s.d;
+  p.h_out = static_cast<__nv_bfloat16*>(h_out);
+  p.blk_start = blk_start;
+  p.blk_len = s.B;
+  return cuda_status(launch_gemm(EPI_OPROJ, g.nt, wm, xm, p, g.grid, pdl, c.st));
+}
+
+dllm_status run_attn(const Ctx& c, int layer, int n_rows, const void* q, const void* kc,
+                     const void* vc, const int* segs, void* out, int ntile_bound, bool pdl) {
+  const Shape& s = c.s;
+  const int g = s.Hq / s.Hkv;
+  AttnPlan a = plan_attn(s, n_rows, ntile_bound);
+  if (a.chunks > 1) {
+    // The partial buffers are sized for the decode row counts; larger row
+    // counts have enough (row tile) CTAs without splitting the keys.
+    const size_t need = (size_t)s.b * s.Hkv * a.row_tiles * a.chunks * 128;
+    const size_t have = (c.l.part_ml - c.l.part_o) / (4 * (size_t)s.D);
+    if (need > have || (size_t)s.b * s.Hkv * a.row_tiles > (size_t)c.l.acnt_n) {
+      a.chunks = 1;
+      a.tpc = ntile_bound;
+    }
+  }
+  const int box_d = s.D >= 64 ? 64 : s.D;
+  const CUtensorMapSwizzle sw = s.D >= 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  CUtensorMap qm, km, vm;
+  if (!make_map(&qm, q, s.D, (uint64_t)g * n_rows, (uint64_t)s.b * s.Hkv, box_d, 128, sw) ||
+      !make_map(&km, kc, s.D, s.S, (uint64_t)s.L * s.b * s.Hkv, box_d, 128, sw) ||
+      !make_map(&vm, vc, s.D, s.S, (uint64_t)s.L * s.b * s.Hkv, box_d, 128, sw))
+    return DLLM_ERR_CUDA;
+  AttnParams p{};
+  p.batch = s.b;
+  p.Hq = s.Hq;
+  p.Hkv = s.Hkv;
+  p.D = s.D;
+  p.S = s.S;
+  p.layer = layer;
+  p.n_rows = n_rows;
+  p.group_rows = g * n_rows;
+  p.row_tiles = a.row_tiles;
+  p.chunks = a.chunks;
+  p.tiles_per_chunk = a.tpc;
+  p.segs = segs;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.part_o = c.at<float>(c.l.part_o);
+  p.part_ml = c.at<float2>(c.l.part_ml);
+  p.counters = c.at<int>(c.l.acnt);
+  p.status = c.at<int>(c.l.status);
+  p.scale_log2 = 1.4426950408889634f / sqrtf((float)s.D);
+  return cuda_status(launch_attn(s.D, qm, km, vm, p, pdl, c.st));
+}
+
+dllm_status run_embed(const Ctx& c, const dllm_weights* w, const dllm_state* stt, int row0,
+                      int n_rows, int use_plants, int blk_start, int seg_end, bool pdl) {
+  const Shape& s = c.s;
+  EmbedParams e{};
+  e.batch = s.b;
+  e.S = s.S;
+  e.G = s.G;
+  e.P = s.P;
+  e.d = s.d;
+  e.n_rows = n_rows;
+  e.row0 = row0;
+  e.use_plants = use_plants;
+  e.blk_start = blk_start;
+  e.blk_len = s.B;
+  e.embed_f32 = s.wfmt == DLLM_W_F32_SPLIT;
+  e.tokens = stt->tokens;
+  e.masked = stt->masked;
+  e.embed = w->embed;
+  e.plants = static_cast<const __nv_bfloat16*>(stt->plants);
+  e.x = c.at<float>(c.l.x);
+  e.xb = c.at<__nv_bfloat16>(c.l.xb);
+  e.segs = c.at<int>(c.l.segs);
+  e.seq_start = stt->seq_start;
+  e.mode = s.mode;
+  e.window = s.W;
+  e.seg_end = seg_end;
+  return cuda_status(launch_embed(e, pdl, c.st));
+}
+
+// Embed + L layers for n_rows rows per sequence at row0.  When h_out is set,
+// the last layer copies the block rows to it.
+dllm_status run_forward(const Ctx& c, const dllm_weights* w, const dllm_state* stt, int row0,
+                        int n_rows, int use_plants, int blk_start, int seg_end, void* h_out) {
+  const Shape& s = c.s;
+  DLLM_TRY(run_embed(c, w, stt, row0, n_rows, use_plants, blk_start, seg_end, true));
+  const int ntb = key_tiles_bound(s, blk_start, seg_end);
+  for (int l = 0; l < s.L; ++l) {
+    DLLM_TRY(run_qkv(c, w->wqkv, l, c.at<void>(c.l.xb), row0, n_rows, stt->seq_start,
+                     c.at<void>(c.l.q), stt->k_cache, stt->v_cache, true));
+    DLLM_TRY(run_attn(c, l, n_rows, c.at<void>(c.l.q), stt->k_cache, stt->v_cache,
+                      c.at<int>(c.l.segs), c.at<void>(c.l.attn), ntb, true));
+    DLLM_TRY(run_oproj(c, w->wo, l, c.at<void>(c.l.attn), row0, n_rows, c.at<float>(c.l.x),
+                       c.at<void>(c.l.xb), l == s.L - 1 ? h_out : nullptr, blk_start, true));
+  }
+  return DLLM_OK;
+}
+
+dllm_status run_lmhead(const Ctx& c, const void* w_lm, const void* h, int n_rows, bool pdl) {
+  const Shape& s = c.s;
+  const GemmPlan g = plan_lmhead(s.V, n_rows, s.Kw);
+  if (g.grid / g.n_tiles > c.l.lm_slots) return DLLM_ERR_WORKSPACE;
+  CUtensorMap wm, xm;
+  if (!make_map(&wm, w_lm, s.Kw, s.V, 1, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&xm, h, s.d, n_rows, 1, 64, g.nt, CU_TENSOR_MAP_SWIZZLE_128B))
+    return DLLM_ERR_CUDA;
+  GemmParams p{};
+  p.M = s.V;
+  p.R = n_rows;
+  p.K = s.Kw;
+  p.kx_blocks = s.d / 64;
+  p.m_tiles = g.m_tiles;
+  p.n_tiles = g.n_tiles;
+  p.splits = 1;
+  p.kb_per_split = g.kbps;
+  p.units = g.units;
+  p.layer = 0;
+  p.status = c.at<int>(c.l.status);
+  p.stats = c.at<LmStat>(c.l.stats);
+  p.stat_slots = g.grid / g.n_tiles;
+  return cuda_status(launch_gemm(EPI_LMHEAD, g.nt, wm, xm, p, g.grid, pdl, c.st));
+}
+
+dllm_status run_commit(const Ctx& c, const dllm_state* stt, int blk_start, bool from_stats,
+                       const float* conf_in, const int* tok_in, bool pdl) {
+  const Shape& s = c.s;
+  const GemmPlan g = plan_lmhead(s.V, s.b * s.B, s.Kw);
+  CommitParams p{};
+  p.batch = s.b;
+  p.S = s.S;
+  p.B = s.B;
+  p.blk_start = blk_start;
+  p.stat_slots = g.grid / g.n_tiles;
+  p.vocab = s.V;
+  p.tau = s.tau;
+  p.stats = from_stats ? c.at<LmStat>(c.l.stats) : nullptr;
+  p.conf = from_stats ? c.at<float>(c.l.conf) : const_cast<float*>(conf_in);
+  p.tok = from_stats ? c.at<int>(c.l.tok) : const_cast<int*>(tok_in);
+  p.gap = from_stats ? c.at<float>(c.l.gap) : nullptr;
+  p.tokens = stt->tokens;
+  p.masked = stt->masked;
+  p.commit = c.at<uint8_t>(c.l.commit);
+  p.remaining = c.at<int>(c.l.remaining);
+  p.do_commit = 1;
+  return cuda_status(launch_commit(p, pdl, c.st));
+}
+
+dllm_status check_state(const Shape& s, const dllm_weights* w, const dllm_state* st) {
+  if (!w || !st || !w->wqkv || !w->wo || !w->w_lm || !w->embed || !st->tokens || !st->masked ||
+      !st->seq_start || !st->k_cache || !st->v_cache)
+    return DLLM_ERR_INVALID;
+  if (!aligned16(w->wqkv) || !aligned16(w->wo) || !aligned16(w->w_lm) || !aligned16(w->embed) ||
+      !aligned16(st->k_cache) || !aligned16(st->v_cache))
+    return DLLM_ERR_INVALID;
+  (void)s;
+  return DLLM_OK;
+}
+
+dllm_status check_block(const Shape& s, int blk) {
+  if (blk < s.P || blk + s.B > s.S || (blk - s.P) % s.B) return DLLM_ERR_INVALID;
+  return DLLM_OK;
+}
+
+dllm_status step(const Ctx& c, const dllm_weights* w, const dllm_state* st, int blk) {
+  const Shape& s = c.s;
+  if (!st->plants || !aligned16(st->plants)) return DLLM_ERR_INVALID;
+  if (s.mode == DLLM_CACHE_NONE) {
+    DLLM_TRY(run_forward(c, w, st, 0, blk + s.B, 1, blk, blk + s.B, c.at<void>(c.l.h)));
+  } else {
+    DLLM_TRY(run_forward(c, w, st, blk, s.B, 1, blk, 0, c.at<void>(c.l.h)));
+  }
+  DLLM_TRY(run_lmhead(c, w->w_lm, c.at<void>(c.l.h), s.b * s.B, true));
+  return run_commit(c, st, blk, true, nullptr, nullptr, true);
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+extern "C" {
+
+dllm_status dllm_workspace_size(const dllm_config* cfg, size_t* bytes) {
+  Shape s;
+  DLLM_TRY(check_cfg(cfg, &s));
+  if (!bytes) return DLLM_ERR_INVALID;
+  *bytes = layout(s).total;
+  return DLLM_OK;
+}
+
+dllm_status dllm_workspace_init(const dllm_config* cfg, void* ws, size_t ws_bytes,
+                                dllm_stream stream) {
+  Ctx c;
+  DLLM_TRY(make_ctx(cfg, ws, ws_bytes, stream, &c));
+  // status word, counters: zero
+  if (cudaMemsetAsync(c.ws, 0, c.l.x, c.st) != cudaSuccess) return DLLM_ERR_CUDA;
+  if (c.s.theta > 0.f)
+    return cuda_status(launch_rope_table(c.at<float2>(c.l.rope), c.s.S, c.s.D, c.s.theta, c.st));
+  return DLLM_OK;
+}
+
+dllm_status dllm_split_f32_weights(const float* src, void* dst, int64_t rows, int64_t cols,
+                                   dllm_stream stream) {
+  if (!src || !dst || rows < 1 || cols < 1) return DLLM_ERR_INVALID;
+  return cuda_status(launch_split_f32(src, static_cast<__nv_bfloat16*>(dst), rows, cols,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+dllm_status dllm_embed_rows(const dllm_config* cfg, const dllm_weights* w, const dllm_state* st,
+                            int32_t row0, int32_t n_rows, int32_t use_plants,
+                            int32_t block_start, float* x, void* xb, dllm_stream stream) {
+  Shape s;
+  DLLM_TRY(check_cfg(cfg, &s));
+  if (!w || !w->embed || !st || !st->tokens || !x || !xb) return DLLM_ERR_INVALID;
+  if (use_plants && (!st->masked || !st->plants)) return DLLM_ERR_INVALID;
+  if (row0 < 0 || n_rows < 1 || row0 + n_rows > s.S) return DLLM_ERR_INVALID;
+  EmbedParams e{};
+  e.batch = s.b;
+  e.S = s.S;
+  e.G = s.G;
+  e.P = s.P;
+  e.d = s.d;
+  e.n_rows = n_rows;
+  e.row0 = row0;
+  e.use_plants = use_plants;
+  e.blk_start = block_start;
+  e.blk_len = s.B;
+  e.embed_f32 = s.wfmt == DLLM_W_F32_SPLIT;
+  e.tokens = st->tokens;
+  e.masked = st->masked;
+  e.embed = w->embed;
+  e.plants = static_cast<const __nv_bfloat16*>(st->plants);
+  e.x = x;
+  e.xb = static_cast<__nv_bfloat16*>(xb);
+  e.segs = nullptr;
+  return cuda_status(launch_embed(e, false, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+dllm_status dllm_qkv_proj(const dllm_config* cfg, const dllm_weights* w, int32_t layer,
+                          const void* xb, int32_t row0, int32_t n_rows, const int32_t* seq_start,
+                          void* q_out, void* k_cache, void* v_cache, void* ws, size_t ws_bytes,
+                          dllm_stream stream) {
+  Ctx c;
+  DLLM_TRY(make_ctx(cfg, ws, ws_bytes, stream, &c));
+  if (!w || !w->wqkv || !xb || !seq_start || !q_out || !k_cache || !v_cache)
+    return DLLM_ERR_INVALID;
+  if (layer < 0 || layer >= c.s.L || row0 < 0 || n_rows < 1 || row0 + n_rows > c.s.S)
+    return DLLM_ERR_INVALID;
+  const GemmPlan g = plan_gemm(c.s.qkv_rows, c.s.b * n_rows, c.s.Kw, true);
+  if (g.splits > 1 && ((size_t)g.units * g.nt * 128 * 4 > c.l.stats - c.l.slots ||
+                       g.m_tiles * g.n_tiles > c.l.gcnt_n))
+    return DLLM_ERR_WORKSPACE;
+  return run_qkv(c, w->wqkv, layer, xb, row0, n_rows, seq_start, q_out, k_cache, v_cache, false);
+}
+
+dllm_status dllm_block_attn(const dllm_config* cfg, int32_t layer, int32_t n_rows, const void* q,
+                            const void* k_cache, const void* v_cache, const int32_t* segs,
+                            void* out, void* ws, size_t ws_bytes, dllm_stream stream) {
+  Ctx c;
+  DLLM_TRY(make_ctx(cfg, ws, ws_bytes, stream, &c));
+  if (!q || !k_cache || !v_cache || !segs || !out) return DLLM_ERR_INVALID;
+  if (layer < 0 || layer >= c.s.L || n_rows < 1 || n_rows > c.s.S) return DLLM_ERR_INVALID;
+  const int ntb = cdiv(c.s.S, 128) + 1;
+  return run_attn(c, layer, n_rows, q, k_cache, v_cache, segs, out, ntb, false);
+}
+
+dllm_status dllm_o_proj(const dllm_config* cfg, const dllm_weights* w, int32_t layer,
+                        const void* attn, int32_t row0, int32_t n_rows, float* x, void* xb,
+                        void* h_out, int32_t block_start, void* ws, size_t ws_bytes,
+                        dllm_stream stream) {
+  Ctx c;
+  DLLM_TRY(make_ctx(cfg, ws, ws_bytes, stream, &c));
+  if (!w || !w->wo || !attn || !x || !xb) return DLLM_ERR_INVALID;
+  if (layer < 0 || layer >= c.s.L || row0 < 0 || n_rows < 1 || row0 + n_rows > c.s.S)
+    return DLLM_ERR_INVALID;
+  const GemmPlan g = plan_gemm(c.s.d, c.s.b * n_rows, c.s.Ko, true);
+  if (g.splits > 1 && ((size_t)g.units * g.nt * 128 * 4 > c.l.stats - c.l.slots ||
+                       g.m_tiles * g.n_tiles > c.l.gcnt_n))
+    return DLLM_ERR_WORKSPACE;
+  return run_oproj(c, w->wo, layer, attn, row0, n_rows, x, xb, h_out, block_start, false);
+}
+
+dllm_status dllm_lmhead_confidence(const dllm_config* cfg, const dllm_weights* w, const void* h,
+                                   int32_t n_rows, float* conf, int32_t* tok, float* gap,
+                                   void* ws, size_t ws_bytes, dllm_stream stream) {
+  Ctx c;
+  DLLM_TRY(make_ctx(cfg, ws, ws_bytes, stream, &c));
+  if (!w || !w->w_lm || !h || !conf || !tok) return DLLM_ERR_INVALID;
+  if (n_rows < 1 || n_rows > c.s.b * c.s.B) return DLLM_ERR_INVALID;
+  DLLM_TRY(run_lmhead(c, w->w_lm, h, n_rows, false));
+  // reduce the per-CTA statistics (one "sequence" of n_rows rows, no commit)
+  const GemmPlan g = plan_lmhead(c.s.V, n_rows, c.s.Kw);
+  CommitParams p{};
+  p.batch = 1;
+  p.S = 0;
+  p.B = n_rows;
+  p.stat_slots = g.grid / g.n_tiles;
+  p.vocab = c.s.V;
+  p.tau = c.s.tau;
+  p.stats = c.at<LmStat>(c.l.stats);
+  p.conf = conf;
+  p.tok = tok;
+  p.gap = gap;
+  p.do_commit = 0;
+  if (n_rows > 64) {
+    // the reduce kernel handles up to 64 rows per CTA: run it per 64-row group
+    for (int r0 = 0; r0 < n_rows; r0 += 64) {
+      CommitParams q = p;
+      q.B = std::min(64, n_rows - r0);
+      q.stats = p.stats + (size_t)r0 * p.stat_slots;
+      q.conf = conf + r0;
+      q.tok = tok + r0;
+      q.gap = gap ? gap + r0 : nullptr;
+      DLLM_TRY(cuda_status(launch_commit(q, false, c.st)));
+    }
+    return DLLM_OK;
+  }
+  return cuda_status(launch_commit(p, false, c.st));
+}
+
+dllm_status dllm_threshold_commit(const dllm_config* cfg, int32_t block_start, const float* conf,
+                                  const int32_t* tok, int32_t* tokens, uint8_t* masked,
+                                  uint8_t* commit, int32_t* remaining, dllm_stream stream) {
+  Shape s;
+  DLLM_TRY(check_cfg(cfg, &s));
+  if (!conf || !tok || !tokens || !masked) return DLLM_ERR_INVALID;
+  DLLM_TRY(check_block(s, block_start));
+  CommitParams p{};
+  p.batch = s.b;
+  p.S = s.S;
+  p.B = s.B;
+  p.blk_start = block_start;
+  p.tau = s.tau;
+  p.vocab = s.V;
+  p.stats = nullptr;
+  p.conf = const_cast<float*>(conf);
+  p.tok = const_cast<int*>(tok);
+  p.tokens = tokens;
+  p.masked = masked;
+  p.commit = commit;
+  p.remaining = remaining;
+  p.do_commit = 1;
+  return cuda_status(launch_commit(p, false, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+dllm_status dllm_prefill(const dllm_config* cfg, const dllm_weights* w, const dllm_state* st,
+                         void* ws, size_t ws_bytes, dllm_stream stream) {
+  Ctx c;
+  DLLM_TRY(make_ctx(cfg, ws, ws_bytes, stream, &c));
+  DLLM_TRY(check_state(c.s, w, st));
+  if (c.s.mode == DLLM_CACHE_NONE) return DLLM_OK;
+  const int end = c.s.mode == DLLM_CACHE_PREFIX ? c.s.P : c.s.S;
+  if (end < 1) return DLLM_OK;
+  return run_forward(c, w, st, 0, end, 0, -1, end, nullptr);
+}
+
+dllm_status dllm_decode_step(const dllm_config* cfg, const dllm_weights* w, const dllm_state* st,
+                             int32_t block_start, void* ws, size_t ws_bytes,
+                             dllm_stream stream) {
+  Ctx c;
+  DLLM_TRY(make_ctx(cfg, ws, ws_bytes, stream, &c));
+  DLLM_TRY(check_state(c.s, w, st));
+  DLLM_TRY(check_block(c.s, block_start));
+  return step(c, w, st, block_start);
+}
+
+dllm_status dllm_kv_cache_refresh(const dllm_config* cfg, const dllm_weights* w,
+                                  const dllm_state* st, int32_t block_start, void* ws,
+                                  size_t ws_bytes, dllm_stream stream) {
+  Ctx c;
+  DLLM_TRY(make_ctx(cfg, ws, ws_bytes, stream, &c));
+  DLLM_TRY(check_state(c.s, w, st));
+  DLLM_TRY(check_block(c.s, block_start));
+  if (c.s.mode == DLLM_CACHE_NONE) return DLLM_OK;
+  return run_forward(c, w, st, block_start, c.s.B, 0, block_start, 0, nullptr);
+}
+
+dllm_status dllm_decode_block(const dllm_config* cfg, const dllm_weights* w, const dllm_state* st,
+                              int32_t block_start, int32_t max_steps, int32_t* steps_taken,
+                              void* ws, size_t ws_bytes, dllm_stream stream) {
+  Ctx c;
+  DLLM_TRY(make_ctx(cfg, ws, ws_bytes, stream, &c));
+  DLLM_TRY(check_state(c.s, w, st));
+  DLLM_TRY(check_block(c.s, block_start));
+  if (max_steps < 1) max_steps = c.s.B;
+  std::vector<int> rem(c.s.b + 1);
+  int n = 0;
+  for (; n < max_steps;) {
+    DLLM_TRY(step(c, w, st, block_start));
+    ++n;
+    if (cudaMemcpyAsync(rem.data(), c.at<int>(c.l.remaining), sizeof(int) * c.s.b,
+                        cudaMemcpyDeviceToHost, c.st) != cudaSuccess ||
+        cudaMemcpyAsync(rem.data() + c.s.b, c.at<int>(c.l.status), sizeof(int),
+                        cudaMemcpyDeviceToHost, c.st) != cudaSuccess ||
+        cudaStreamSynchronize(c.st) != cudaSuccess)
+      return DLLM_ERR_CUDA;
+    if (rem[c.s.b] != 0) return DLLM_ERR_TIMEOUT;
+    int left = 0;
+    for (int i = 0; i < c.s.b; ++i) left += rem[i];
+    if (left == 0) break;
+  }
+  if (steps_taken) *steps_taken = n;
+  if (c.s.mode != DLLM_CACHE_NONE)
+    DLLM_TRY(run_forward(c, w, st, block_start, c.s.B, 0, block_start, 0, nullptr));
+  return DLLM_OK;
+}
+
+dllm_status dllm_step_outputs(const dllm_config* cfg, void* ws, size_t ws_bytes, float** conf,
+                              int32_t** tok, float** gap, uint8_t** commit) {
+  Ctx c;
+  DLLM_TRY(make_ctx(cfg, ws, ws_bytes, nullptr, &c));
+  if (conf) *conf = c.at<float>(c.l.conf);
+  if (tok) *tok = c.at<int>(c.l.tok);
+  if (gap) *gap = c.at<float>(c.l.gap);
+  if (commit) *commit = c.at<uint8_t>(c.l.commit);
+  return DLLM_OK;
+}
+
+dllm_status dllm_device_status(void* ws, int32_t* code, dllm_stream stream) {
+  if (!ws || !code) return DLLM_ERR_INVALID;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(code, ws, sizeof(int32_t), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return DLLM_ERR_CUDA;
+  return DLLM_OK;
+}
+
+uint64_t dllm_launch_count(void) { return dllm::launch_count(); }
+
+const char* dllm_status_string(dllm_status s) {
+  switch (s) {
+    case DLLM_OK: return "ok";
+    case DLLM_ERR_INVALID: return "invalid argument";
+    case DLLM_ERR_UNSUPPORTED: return "unsupported shape";
+    case DLLM_ERR_CUDA: return "CUDA error";
+    case DLLM_ERR_TIMEOUT: return "device wait timed out";
+    case DLLM_ERR_WORKSPACE: return "workspace too small";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,441 @@
+// Weight-streaming GEMM on tcgen05 for the decode step's projections and LM head.
+//
+// Every projection of the step has few activation rows (b*B = 32..512) and a
+// large weight matrix, so the weights are the UMMA "A" operand (M = 128 weight
+// rows per tile) and the activations the "B" operand (N = NT rows):
+//     D^T[wrow][xrow] = sum_k W[wrow][k] * X[xrow][k]
+// with both operands K-major in shared memory (128-byte swizzle, staged by
+// TMA) and the fp32 accumulator in TMEM.  A persistent CTA (one per SM) runs
+// three warp roles: warp 0 issues TMA loads through a STAGES-deep ring,
+// warp 1 issues the UMMAs, warps 2-5 drain TMEM (double-buffered
+// accumulator) and run one of three fused epilogues:
+//   EPI_QKV    RoPE on q/k, bf16 store of q and of k/v into the cache slots
+//   EPI_OPROJ  residual add in fp32, bf16 copy for the next projection
+//   EPI_LMHEAD per-row running max / sum-exp / argmax / second max over the
+//              CTA's vocabulary tiles; logits never leave the SM
+// When (weight tiles x row tiles) would leave SMs idle, K is split; each split
+// writes an fp32 partial to a scratch slot and the last split to arrive (a
+// per-tile counter) sums the slots in split order and runs the epilogue, so
+// the result does not depend on arrival order.
+#include <float.h>
+#include <limits.h>
+
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace dllm {
+
+template <int NT>
+struct GemmCfg {
+  static constexpr int kStages = NT <= 32 ? 8 : NT <= 64 ? 6 : NT <= 128 ? 5 : 4;
+  static constexpr int kWBytes = 128 * 64 * 2;
+  static constexpr int kXBytes = NT * 64 * 2;
+  static constexpr int kTmemCols = 2 * NT;
+  static constexpr int kChunk = 16;
+  static constexpr size_t kSmem = 1024 + (size_t)kStages * (kWBytes + kXBytes) +
+                                  kChunk * 128 * 4 + NT * sizeof(LmStat) +
+                                  (2 * kStages + 4) * 8 + 64;
+};
+
+__device__ __forceinline__ void decode_unit(const GemmParams& p, int u, int& m, int& n, int& tile,
+                                            int& kb0, int& kb1) {
+  tile = u / p.splits;
+  const int sp = u - tile * p.splits;
+  m = tile / p.n_tiles;
+  n = tile - m * p.n_tiles;
+  kb0 = sp * p.kb_per_split;
+  kb1 = min(p.K / 64, kb0 + p.kb_per_split);
+}
+
+__device__ __forceinline__ LmStat lm_merge(const LmStat& a, const LmStat& b) {
+  const bool b_hi = (b.m > a.m) || (b.m == a.m && b.idx < a.idx);
+  const LmStat& hi = b_hi ? b : a;
+  const LmStat& lo = b_hi ? a : b;
+  LmStat r;
+  r.m = hi.m;
+  r.idx = hi.idx;
+  r.m2 = fmaxf(hi.m2, lo.m);
+  r.s = hi.s + (lo.s > 0.f ? lo.s * __expf(lo.m - hi.m) : 0.f);
+  return r;
+}
+
+__device__ __forceinline__ LmStat lm_shfl_xor(const LmStat& a, int mask) {
+  LmStat r;
+  r.m = __shfl_xor_sync(0xffffffffu, a.m, mask);
+  r.s = __shfl_xor_sync(0xffffffffu, a.s, mask);
+  r.m2 = __shfl_xor_sync(0xffffffffu, a.m2, mask);
+  r.idx = __shfl_xor_sync(0xffffffffu, a.idx, mask);
+  return r;
+}
+
+// Epilogue of one 16-column chunk; v[i] = D^T[m*128 + wl][n*NT + c0 + i].
+template <int NT, int EPI>
+__device__ __forceinline__ void epi_chunk(const GemmParams& p, int m, int n, int c0, int wl,
+                                          int et, const float (&v)[16], float* stage,
+                                          LmStat* run) {
+  if constexpr (EPI == EPI_OPROJ) {
+    const int wrow = m * 128 + wl;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int xrow = n * NT + c0 + i;
+      if (xrow < p.R) {
+        const size_t off = (size_t)xrow * p.d_model + wrow;
+        const float nx = p.x[off] + v[i];
+        p.x[off] = nx;
+        const __nv_bfloat16 nb = __float2bfloat16_rn(nx);
+        p.xb[off] = nb;
+        if (p.h_out != nullptr) {
+          const int b = xrow / p.n_rows;
+          const int pos = p.row0 + (xrow - b * p.n_rows);
+          if (pos >= p.blk_start && pos < p.blk_start + p.blk_len)
+            p.h_out[((size_t)b * p.blk_len + (pos - p.blk_start)) * p.d_model + wrow] = nb;
+        }
+      }
+    }
+  } else if constexpr (EPI == EPI_QKV) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) stage[i * 128 + wl] = v[i];
+    named_bar_sync(1, 128);
+    const int D = p.D, half = D >> 1;
+    const int wrow = m * 128 + wl;
+    const int head = wrow / D;
+    const int dd = wrow - head * D;
+    const bool is_q = head < p.Hq;
+    const bool is_k = !is_q && head < p.Hq + p.Hkv;
+    const bool rope = (p.rope_tab != nullptr) && (is_q || is_k);
+    const int partner = wl + (dd < half ? half : -half);
+    const int j = dd < half ? dd : dd - half;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int xrow = n * NT + c0 + i;
+      if (xrow >= p.R) continue;
+      const int b = xrow / p.n_rows;
+      const int ii = xrow - b * p.n_rows;
+      const int pos = p.row0 + ii;
+      float val = v[i];
+      if (rope) {
+        int rp = pos - p.seq_start[b];
+        rp = rp < 0 ? 0 : rp;
+        const float2 cs = p.rope_tab[(size_t)rp * half + j];
+        const float o = stage[i * 128 + partner];
+        val = dd < half ? (val * cs.x - o * cs.y) : (val * cs.x + o * cs.y);
+      }
+      const __nv_bfloat16 bv = __float2bfloat16_rn(val);
+      if (is_q) {
+        p.q_out[(((size_t)b * p.Hq + head) * p.n_rows + ii) * D + dd] = bv;
+      } else {
+        const int kvh = is_k ? head - p.Hq : head - p.Hq - p.Hkv;
+        const size_t off =
+            ((((size_t)p.layer * p.batch + b) * p.Hkv + kvh) * p.S + pos) * (size_t)D + dd;
+        (is_k ? p.k_cache : p.v_cache)[off] = bv;
+      }
+    }
+    named_bar_sync(1, 128);
+  } else {  // EPI_LMHEAD
+#pragma unroll
+    for (int i = 0; i < 16; ++i) stage[i * 128 + wl] = v[i];
+    named_bar_sync(1, 128);
+    const int col = et >> 3, sub = et & 7;
+    const float* cv = stage + col * 128 + sub * 16;
+    const int vbase = m * 128 + sub * 16;
+    LmStat st;
+    st.m = -FLT_MAX;
+    st.m2 = -FLT_MAX;
+    st.idx = INT_MAX;
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      const float x = cv[q];
+      if (x > st.m) {
+        st.m2 = st.m;
+        st.m = x;
+        st.idx = vbase + q;
+      } else if (x > st.m2) {
+        st.m2 = x;
+      }
+    }
+    float s = 0.f;
+#pragma unroll
+    for (int q = 0; q < 16; ++q) s += __expf(cv[q] - st.m);
+    st.s = s;
+#pragma unroll
+    for (int mask = 1; mask < 8; mask <<= 1) st = lm_merge(st, lm_shfl_xor(st, mask));
+    if (sub == 0) run[c0 + col] = lm_merge(run[c0 + col], st);
+    named_bar_sync(1, 128);
+  }
+}
+
+template <int NT, int EPI>
+__global__ void __launch_bounds__(192, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap xmap,
+                const GemmParams p) {
+  using C = GemmCfg<NT>;
+  constexpr int ST = C::kStages;
+  constexpr uint32_t kIdesc = idesc_bf16(128, NT, 0, 0);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* w_st = base;
+  uint8_t* x_st = w_st + ST * C::kWBytes;
+  float* stage = reinterpret_cast<float*>(x_st + ST * C::kXBytes);
+  LmStat* run = reinterpret_cast<LmStat*>(stage + C::kChunk * 128);
+  uint64_t* full = reinterpret_cast<uint64_t*>(run + NT);
+  uint64_t* empty = full + ST;
+  uint64_t* tfull = empty + ST;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  volatile int* flags = reinterpret_cast<volatile int*>(tmem_slot + 2);  // [0] abort, [1] last
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    flags[0] = 0;
+    flags[1] = 0;
+    fence_barrier_init();
+  }
+  for (int c = threadIdx.x; c < NT; c += blockDim.x) {
+    run[c].m = -FLT_MAX;
+    run[c].s = 0.f;
+    run[c].m2 = -FLT_MAX;
+    run[c].idx = INT_MAX;
+  }
+  if (threadIdx.x == 32) {
+    prefetch_tmap(&wmap);
+    prefetch_tmap(&xmap);
+  }
+  __syncthreads();
+  grid_dep_launch();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    grid_dep_wait();
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_first();
+      int it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+        int m, n, tile, kb0, kb1;
+        decode_unit(p, u, m, n, tile, kb0, kb1);
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int s = it % ST;
+          const uint32_t ph = (it / ST) & 1;
+          if (!mbar_wait(&empty[s], ph ^ 1, p.status) || flags[0]) {
+            flags[0] = 1;
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], C::kWBytes + C::kXBytes);
+          tma_load_3d_hint(w_st + s * C::kWBytes, &wmap, &full[s], kb * 64, m * 128, p.layer,
+                           pol_w);
+          tma_load_3d(x_st + s * C::kXBytes, &xmap, &full[s], (kb % p.kx_blocks) * 64, n * NT,
+                      0);
+        }
+      }
+      // Before leaving after an abort, let loads already in flight land.
+      if (!ok) {
+        for (int k = 0; k < ST && it - 1 - k >= 0; ++k) {
+          const int j = it - 1 - k;
+          mbar_wait(&full[j % ST], (j / ST) & 1, nullptr);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    grid_dep_wait();
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tc_fence_before();
+    named_bar_sync(2, 160);
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    if (lane == 0) {
+      int it = 0, j = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x, ++j) {
+        int m, n, tile, kb0, kb1;
+        decode_unit(p, u, m, n, tile, kb0, kb1);
+        const int acc = j & 1;
+        const uint32_t aph = (j >> 1) & 1;
+        if (!mbar_wait(&tempty[acc], aph ^ 1, p.status) || flags[0]) {
+          flags[0] = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + acc * NT;
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int s = it % ST;
+          const uint32_t ph = (it / ST) & 1;
+          if (!mbar_wait(&full[s], ph, p.status) || flags[0]) {
+            flags[0] = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t wa = smem_u32(w_st + s * C::kWBytes);
+          const uint32_t xa = smem_u32(x_st + s * C::kXBytes);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            umma_bf16(d_tmem, smem_desc(wa + k * 32, 16, 1024, 2),
+                      smem_desc(xa + k * 32, 16, 1024, 2), kIdesc,
+                      (kb > kb0 || k > 0) ? 1u : 0u);
+          }
+          umma_commit(&empty[s]);
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    grid_dep_wait();
+    named_bar_sync(2, 160);
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int et = threadIdx.x - 64;         // 0..127
+    const int lane_base = 32 * (warp & 3);   // TMEM lanes this warp may access
+    const int wl = lane_base + lane;         // weight row within the tile
+    int j = 0;
+    for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++j) {
+      int m, n, tile, kb0, kb1;
+      decode_unit(p, u, m, n, tile, kb0, kb1);
+      const int acc = j & 1;
+      const uint32_t aph = (j >> 1) & 1;
+      const bool bad = !mbar_wait(&tfull[acc], aph, p.status) || flags[0];
+      if (named_bar_or(1, 128, bad)) {
+        flags[0] = 1;
+        break;
+      }
+      tc_fence_after();
+      const bool split = p.splits > 1;
+      for (int c0 = 0; c0 < NT; c0 += 16) {
+        float v[16];
+        tmem_ld16(tmem + ((uint32_t)lane_base << 16) + acc * NT + c0, v);
+        tmem_ld_wait();
+        if (split) {
+          float* slot = p.slots + ((size_t)u * NT + c0) * 128;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) slot[i * 128 + wl] = v[i];
+        } else {
+          epi_chunk<NT, EPI>(p, m, n, c0, wl, et, v, stage, run);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+      if (split) {
+        __threadfence();
+        named_bar_sync(1, 128);
+        if (et == 0) {
+          const int old = atomicAdd(&p.counters[tile], 1);
+          const int last = (old == p.splits - 1);
+          if (last) p.counters[tile] = 0;
+          flags[1] = last;
+        }
+        named_bar_sync(1, 128);
+        const int last = flags[1];
+        named_bar_sync(1, 128);
+        if (last) {
+          __threadfence();
+          for (int c0 = 0; c0 < NT; c0 += 16) {
+            float v[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] = 0.f;
+            for (int sp = 0; sp < p.splits; ++sp) {
+              const float* slot = p.slots + ((size_t)(tile * p.splits + sp) * NT + c0) * 128;
+#pragma unroll
+              for (int i = 0; i < 16; ++i) v[i] += __ldcg(slot + i * 128 + wl);
+            }
+            epi_chunk<NT, EPI>(p, m, n, c0, wl, et, v, stage, run);
+          }
+        }
+      }
+    }
+    if constexpr (EPI == EPI_LMHEAD) {
+      named_bar_sync(1, 128);
+      const int n = blockIdx.x % p.n_tiles;
+      const int slot = blockIdx.x / p.n_tiles;
+      for (int c = et; c < NT; c += 128) {
+        const int xrow = n * NT + c;
+        if (xrow < p.R) p.stats[(size_t)xrow * p.stat_slots + slot] = run[c];
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(*tmem_slot, C::kTmemCols);
+  }
+}
+
+template <int NT, int EPI>
+static cudaError_t launch_t(const CUtensorMap& wmap, const CUtensorMap& xmap, const GemmParams& p,
+                            int grid, bool pdl, cudaStream_t s) {
+  auto kern = gemm_kernel<NT, EPI>;
+  const size_t smem = GemmCfg<NT>::kSmem;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  count_launch();
+  return cudaLaunchKernelEx(&cfg, kern, wmap, xmap, p);
+}
+
+int gemm_stages(int nt) {
+  switch (nt) {
+    case 32: return GemmCfg<32>::kStages;
+    case 64: return GemmCfg<64>::kStages;
+    case 128: return GemmCfg<128>::kStages;
+    default: return GemmCfg<256>::kStages;
+  }
+}
+
+size_t gemm_smem_bytes(int nt) {
+  switch (nt) {
+    case 32: return GemmCfg<32>::kSmem;
+    case 64: return GemmCfg<64>::kSmem;
+    case 128: return GemmCfg<128>::kSmem;
+    default: return GemmCfg<256>::kSmem;
+  }
+}
+
+template <int EPI>
+static cudaError_t launch_e(int nt, const CUtensorMap& wmap, const CUtensorMap& xmap,
+                            const GemmParams& p, int grid, bool pdl, cudaStream_t s) {
+  switch (nt) {
+    case 32: return launch_t<32, EPI>(wmap, xmap, p, grid, pdl, s);
+    case 64: return launch_t<64, EPI>(wmap, xmap, p, grid, pdl, s);
+    case 128: return launch_t<128, EPI>(wmap, xmap, p, grid, pdl, s);
+    case 256: return launch_t<256, EPI>(wmap, xmap, p, grid, pdl, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_gemm(int epi, int nt, const CUtensorMap& wmap, const CUtensorMap& xmap,
+                        const GemmParams& p, int grid, bool pdl, cudaStream_t s) {
+  switch (epi) {
+    case EPI_QKV: return launch_e<EPI_QKV>(nt, wmap, xmap, p, grid, pdl, s);
+    case EPI_OPROJ: return launch_e<EPI_OPROJ>(nt, wmap, xmap, p, grid, pdl, s);
+    case EPI_LMHEAD: return launch_e<EPI_LMHEAD>(nt, wmap, xmap, p, grid, pdl, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace dllm

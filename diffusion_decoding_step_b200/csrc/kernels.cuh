@@ -1,0 +1,118 @@
+// Internal parameter blocks and launchers shared by the kernel files and the
+// C-ABI layer.  Nothing here is part of the public interface.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace dllm {
+
+constexpr int kNumSMs = 148;
+
+enum EpiKind : int { EPI_QKV = 0, EPI_OPROJ = 1, EPI_LMHEAD = 2 };
+
+// Running softmax statistics of a set of logits: max, sum of exp(l - max),
+// second largest (a tied maximum counts), index of the first maximum.
+struct __align__(16) LmStat {
+  float m, s, m2;
+  int idx;
+};
+
+struct GemmParams {
+  // D^T[wrow][xrow] = sum_k W[layer][wrow][k] * X[xrow][k mod kx]
+  int M;          // weight rows (multiple of 128)
+  int R;          // activation rows
+  int K;          // weight K extent (multiple of 64)
+  int kx_blocks;  // X operand K extent / 64 (k-block kb reads X block kb % kx_blocks)
+  int m_tiles, n_tiles, splits, kb_per_split, units;
+  int layer;
+  int* status;
+  // split-K scratch: slots[unit][NT][128] fp32, counters[tile]
+  float* slots;
+  int* counters;
+  // rows are (sequence, i) with position row0 + i, n_rows per sequence
+  int n_rows, row0;
+  const int* seq_start;
+  // QKV epilogue
+  int Hq, Hkv, D, S, batch;
+  const float2* rope_tab;  // [S][D/2] (cos, sin) or null
+  __nv_bfloat16* q_out;
+  __nv_bfloat16* k_cache;
+  __nv_bfloat16* v_cache;
+  // O-proj epilogue
+  float* x;
+  __nv_bfloat16* xb;
+  int d_model;
+  __nv_bfloat16* h_out;
+  int blk_start, blk_len;
+  // LM-head epilogue: stats[xrow][slot]
+  LmStat* stats;
+  int stat_slots;
+};
+
+struct AttnParams {
+  int batch, Hq, Hkv, D, S, layer;
+  int n_rows;       // query rows per sequence and head
+  int group_rows;   // (Hq/Hkv) * n_rows
+  int row_tiles;    // ceil(group_rows / 128)
+  int chunks;       // key chunks per (sequence, kv head, row tile)
+  int tiles_per_chunk;
+  const int* segs;  // [b][2][2] (start, len)
+  __nv_bfloat16* out;  // [b*n_rows][Hq*D]
+  float* part_o;       // [b][Hkv][row_tiles][chunks][128][D]
+  float2* part_ml;     // [b][Hkv][row_tiles][chunks][128]
+  int* counters;       // [b][Hkv][row_tiles]
+  int* status;
+  float scale_log2;    // log2(e) / sqrt(D)
+};
+
+// Launch helpers (return cudaError_t of the launch).
+cudaError_t launch_gemm(int epi, int nt, const CUtensorMap& wmap, const CUtensorMap& xmap,
+                        const GemmParams& p, int grid, bool pdl, cudaStream_t s);
+int gemm_stages(int nt);
+size_t gemm_smem_bytes(int nt);
+
+cudaError_t launch_attn(int head_dim, const CUtensorMap& qmap, const CUtensorMap& kmap,
+                        const CUtensorMap& vmap, const AttnParams& p, bool pdl,
+                        cudaStream_t s);
+size_t attn_smem_bytes(int head_dim);
+
+struct EmbedParams {
+  int batch, S, G, P, d, n_rows, row0, use_plants, blk_start, blk_len, embed_f32;
+  const int* tokens;
+  const uint8_t* masked;
+  const void* embed;
+  const __nv_bfloat16* plants;
+  float* x;
+  __nv_bfloat16* xb;
+  // optional: key segments of the step, written by block 0 thread 0
+  int* segs;
+  const int* seq_start;
+  int mode, window, seg_end;  // seg_end: end of the key range for prefill/none
+};
+cudaError_t launch_embed(const EmbedParams& p, bool pdl, cudaStream_t s);
+
+struct CommitParams {
+  int batch, S, B, blk_start, stat_slots, vocab;
+  float tau;
+  const LmStat* stats;  // [b*B][stat_slots] or null when conf/tok are given
+  float* conf;          // [b][B]
+  int* tok;
+  float* gap;
+  int* tokens;
+  uint8_t* masked;
+  uint8_t* commit;
+  int* remaining;
+  int do_commit;
+};
+cudaError_t launch_commit(const CommitParams& p, bool pdl, cudaStream_t s);
+
+cudaError_t launch_rope_table(float2* tab, int S, int D, double theta, cudaStream_t s);
+cudaError_t launch_split_f32(const float* src, __nv_bfloat16* dst, int64_t rows, int64_t cols,
+                             cudaStream_t s);
+
+// Count of kernels launched by this library.
+void count_launch();
+
+}  // namespace dllm

@@ -1,0 +1,263 @@
+// Latency-bound kernels of the step: layer-0 input (plant or embedding),
+// cross-tile vocabulary reduce fused with the threshold commit, and the
+// one-time tables (RoPE cos/sin, fp32 weight split).
+#include <float.h>
+#include <limits.h>
+#include <math.h>
+
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace dllm {
+
+static unsigned long long g_launches = 0;
+void count_launch() { ++g_launches; }
+unsigned long long launch_count() { return g_launches; }
+
+template <class K, class... A>
+static cudaError_t launch_simple(K kern, dim3 grid, dim3 block, bool pdl, cudaStream_t s,
+                                 A... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  count_launch();
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+// ------------------------------------------------------------------ embed
+// One CTA per row.  x0 = plant (masked row of the block) or embed[token].
+// Block 0 also writes the step's key segments.
+__global__ void __launch_bounds__(256) embed_kernel(const EmbedParams p) {
+  grid_dep_wait();
+  grid_dep_launch();
+  const int row = blockIdx.x;
+  const int b = row / p.n_rows;
+  const int pos = p.row0 + (row - b * p.n_rows);
+  for (int bb = threadIdx.x; row == 0 && p.segs != nullptr && bb < p.batch; bb += blockDim.x) {
+    const int st = p.seq_start[bb];
+    int s0 = st, l0 = 0, s1 = 0, l1 = 0;
+    const int end = p.blk_start + p.blk_len;
+    if (p.seg_end > 0) {
+      l0 = p.seg_end - st;
+    } else if (p.mode == 2) {           // DUAL
+      l0 = p.S - st;
+    } else if (p.mode == 3) {           // DUAL_PRUNED
+      const int wend = min(end + p.window, p.S);
+      l0 = wend - st;
+      if (end < p.S && p.S - 1 >= wend) {
+        s1 = p.S - 1;
+        l1 = 1;
+      }
+    } else {                            // NONE, PREFIX
+      l0 = end - st;
+    }
+    int* o = p.segs + bb * 4;
+    o[0] = s0;
+    o[1] = l0 > 0 ? l0 : 0;
+    o[2] = s1;
+    o[3] = l1;
+  }
+  const bool plant = p.use_plants && p.masked[(size_t)b * p.S + pos] &&
+                     pos >= p.blk_start && pos < p.blk_start + p.blk_len;
+  float* xr = p.x + (size_t)row * p.d;
+  __nv_bfloat16* xbr = p.xb + (size_t)row * p.d;
+  if (plant) {
+    const __nv_bfloat16* src = p.plants + ((size_t)b * p.G + (pos - p.P)) * p.d;
+    for (int i = threadIdx.x * 8; i < p.d; i += blockDim.x * 8) {
+      const uint4 raw = *reinterpret_cast<const uint4*>(src + i);
+      *reinterpret_cast<uint4*>(xbr + i) = raw;
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 f = __bfloat1622float2(h2[k]);
+        xr[i + 2 * k] = f.x;
+        xr[i + 2 * k + 1] = f.y;
+      }
+    }
+  } else {
+    const int tok = p.tokens[(size_t)b * p.S + pos];
+    if (p.embed_f32) {
+      const float* src = reinterpret_cast<const float*>(p.embed) + (size_t)tok * p.d;
+      for (int i = threadIdx.x * 4; i < p.d; i += blockDim.x * 4) {
+        const float4 f = *reinterpret_cast<const float4*>(src + i);
+        *reinterpret_cast<float4*>(xr + i) = f;
+        xbr[i] = __float2bfloat16_rn(f.x);
+        xbr[i + 1] = __float2bfloat16_rn(f.y);
+        xbr[i + 2] = __float2bfloat16_rn(f.z);
+        xbr[i + 3] = __float2bfloat16_rn(f.w);
+      }
+    } else {
+      const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>(p.embed) + (size_t)tok * p.d;
+      for (int i = threadIdx.x * 8; i < p.d; i += blockDim.x * 8) {
+        const uint4 raw = *reinterpret_cast<const uint4*>(src + i);
+        *reinterpret_cast<uint4*>(xbr + i) = raw;
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 f = __bfloat1622float2(h2[k]);
+          xr[i + 2 * k] = f.x;
+          xr[i + 2 * k + 1] = f.y;
+        }
+      }
+    }
+  }
+}
+
+cudaError_t launch_embed(const EmbedParams& p, bool pdl, cudaStream_t s) {
+  return launch_simple(embed_kernel, dim3(p.batch * p.n_rows), dim3(256), pdl, s, p);
+}
+
+// ------------------------------------------------------------------ reduce + commit
+__device__ __forceinline__ LmStat merge_stat(const LmStat& a, const LmStat& b) {
+  const bool b_hi = (b.m > a.m) || (b.m == a.m && b.idx < a.idx);
+  const LmStat& hi = b_hi ? b : a;
+  const LmStat& lo = b_hi ? a : b;
+  LmStat r;
+  r.m = hi.m;
+  r.idx = hi.idx;
+  r.m2 = fmaxf(hi.m2, lo.m);
+  r.s = hi.s + (lo.s > 0.f ? lo.s * __expf(lo.m - hi.m) : 0.f);
+  return r;
+}
+
+// One CTA (256 threads) per sequence.  Phase 1: merge the per-CTA vocabulary
+// statistics of each block row into conf = 1 / sum exp(l - max), tok, gap.
+// Phase 2 (warp 0): commit masked rows with conf > tau, plus the most
+// confident masked row (lowest position on ties).
+__global__ void __launch_bounds__(256) commit_kernel(const CommitParams p) {
+  grid_dep_wait();
+  grid_dep_launch();
+  __shared__ float s_conf[64];
+  __shared__ int s_tok[64];
+  const int b = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (p.stats != nullptr) {
+    for (int i = warp; i < p.B; i += 8) {
+      const LmStat* src = p.stats + (size_t)(b * p.B + i) * p.stat_slots;
+      LmStat st;
+      st.m = -FLT_MAX;
+      st.s = 0.f;
+      st.m2 = -FLT_MAX;
+      st.idx = INT_MAX;
+      for (int k = lane; k < p.stat_slots; k += 32) st = merge_stat(st, src[k]);
+#pragma unroll
+      for (int mask = 16; mask > 0; mask >>= 1) {
+        LmStat o;
+        o.m = __shfl_xor_sync(0xffffffffu, st.m, mask);
+        o.s = __shfl_xor_sync(0xffffffffu, st.s, mask);
+        o.m2 = __shfl_xor_sync(0xffffffffu, st.m2, mask);
+        o.idx = __shfl_xor_sync(0xffffffffu, st.idx, mask);
+        st = merge_stat(st, o);
+      }
+      if (lane == 0) {
+        const float conf = 1.f / st.s;
+        s_conf[i] = conf;
+        s_tok[i] = st.idx;
+        p.conf[b * p.B + i] = conf;
+        p.tok[b * p.B + i] = st.idx;
+        if (p.gap) p.gap[b * p.B + i] = st.m - st.m2;
+      }
+    }
+  } else {
+    for (int i = threadIdx.x; i < p.B; i += blockDim.x) {
+      s_conf[i] = p.conf[b * p.B + i];
+      s_tok[i] = p.tok[b * p.B + i];
+    }
+  }
+  __syncthreads();
+  if (!p.do_commit || warp != 0) return;
+  // two rows per lane (B <= 64)
+  const int i0 = lane, i1 = lane + 32;
+  const size_t base = (size_t)b * p.S + p.blk_start;
+  const bool m0 = i0 < p.B && p.masked[base + i0];
+  const bool m1 = i1 < p.B && p.masked[base + i1];
+  const float c0 = m0 ? s_conf[i0] : -1.f;
+  const float c1 = m1 ? s_conf[i1] : -1.f;
+  // best masked row: largest conf, lowest position on ties
+  float bc = c0;
+  int bi = i0;
+  if (c1 > bc) {
+    bc = c1;
+    bi = i1;
+  }
+#pragma unroll
+  for (int mask = 16; mask > 0; mask >>= 1) {
+    const float oc = __shfl_xor_sync(0xffffffffu, bc, mask);
+    const int oi = __shfl_xor_sync(0xffffffffu, bi, mask);
+    if (oc > bc || (oc == bc && oi < bi)) {
+      bc = oc;
+      bi = oi;
+    }
+  }
+  const bool any_masked = bc >= 0.f;
+  const bool k0 = m0 && (c0 > p.tau || (any_masked && bi == i0));
+  const bool k1 = m1 && (c1 > p.tau || (any_masked && bi == i1));
+  if (k0) {
+    p.tokens[base + i0] = s_tok[i0];
+    p.masked[base + i0] = 0;
+  }
+  if (k1) {
+    p.tokens[base + i1] = s_tok[i1];
+    p.masked[base + i1] = 0;
+  }
+  if (p.commit) {
+    if (i0 < p.B) p.commit[b * p.B + i0] = k0;
+    if (i1 < p.B) p.commit[b * p.B + i1] = k1;
+  }
+  const unsigned left = __popc(__ballot_sync(0xffffffffu, m0 && !k0)) +
+                        __popc(__ballot_sync(0xffffffffu, m1 && !k1));
+  if (lane == 0 && p.remaining) p.remaining[b] = (int)left;
+}
+
+cudaError_t launch_commit(const CommitParams& p, bool pdl, cudaStream_t s) {
+  return launch_simple(commit_kernel, dim3(p.batch), dim3(256), pdl, s, p);
+}
+
+// ------------------------------------------------------------------ tables
+__global__ void rope_table_kernel(float2* tab, int S, int D, double theta) {
+  const int half = D / 2;
+  const int n = S * half;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    const int pos = i / half, j = i - pos * half;
+    const double inv = pow(theta, -2.0 * (double)j / (double)D);
+    double sn, cs;
+    sincos((double)pos * inv, &sn, &cs);
+    tab[i] = make_float2((float)cs, (float)sn);
+  }
+}
+
+cudaError_t launch_rope_table(float2* tab, int S, int D, double theta, cudaStream_t s) {
+  count_launch();
+  rope_table_kernel<<<148, 256, 0, s>>>(tab, S, D, theta);
+  return cudaGetLastError();
+}
+
+__global__ void split_f32_kernel(const float* src, __nv_bfloat16* dst, int64_t rows,
+                                 int64_t cols) {
+  const int64_t n = rows * cols;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = i / cols, c = i - r * cols;
+    const float w = src[i];
+    const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(w - __bfloat162float(hi));
+    dst[r * 2 * cols + c] = hi;
+    dst[r * 2 * cols + cols + c] = lo;
+  }
+}
+
+cudaError_t launch_split_f32(const float* src, __nv_bfloat16* dst, int64_t rows, int64_t cols,
+                             cudaStream_t s) {
+  count_launch();
+  split_f32_kernel<<<4 * 148, 256, 0, s>>>(src, dst, rows, cols);
+  return cudaGetLastError();
+}
+
+}  // namespace dllm

@@ -1,0 +1,203 @@
+/*
+ * dllm.h - C ABI of the B200 (sm_100a) block-decode step of a masked-diffusion LLM.
+ *
+ * The method (Fast-dLLM v1): a block of masked positions is denoised in
+ * parallel; each step every masked position gets the max-softmax confidence
+ * and argmax token of the LM head, and every position whose confidence
+ * clears the threshold tau is committed ("Fast-dLLM: Four Acceleration Tracks
+ * for Diffusion Language Models...", section "The v1 Mechanism: KV Cache Plus
+ * Confidence-Threshold Parallel Decoding").  A key/value cache holds the
+ * attention state of settled positions (same section; Fast-dLLM README,
+ * project table, "KV Cache + Parallel Decoding"); the suffix may be pruned to
+ * a window after the block plus the trailing position (Streaming-dLLM README,
+ * figure "Illustration of approximated suffix pruning").
+ *
+ * Conventions for every entry point
+ *  - All tensor pointers are DEVICE pointers owned by the caller unless a
+ *    parameter says "host".  The library allocates no device memory; scratch
+ *    comes from the caller's workspace (dllm_workspace_size bytes, prepared
+ *    once with dllm_workspace_init).
+ *  - Calls are asynchronous on `stream` unless documented otherwise; nothing
+ *    prints, nothing aborts.  Invalid arguments return DLLM_ERR_INVALID or
+ *    DLLM_ERR_UNSUPPORTED before anything is launched.
+ *  - Layouts are row-major, innermost index last.  bf16 = IEEE bfloat16.
+ *    b = batch, L = layers, d = hidden, Hq/Hkv = query/kv heads, D = head_dim,
+ *    V = vocab, P = prompt_len, G = gen_len, B = block, S = P + G.
+ *  - Supported: D in {32, 128}; d, Hq*D and (Hq+2Hkv)*D multiples of 128;
+ *    V a multiple of 128; Hq a multiple of Hkv; B <= 64; b <= 1024.
+ *  - Device-side waits are bounded (about 2 s); a wait that gives up sets a bit
+ *    in the workspace status word, read with dllm_device_status.
+ */
+#ifndef DLLM_H_
+#define DLLM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* dllm_stream; /* a cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+  DLLM_OK = 0,
+  DLLM_ERR_INVALID = -1,     /* bad pointer, size or configuration */
+  DLLM_ERR_UNSUPPORTED = -2, /* valid but not implemented shape */
+  DLLM_ERR_CUDA = -3,        /* a CUDA runtime/driver call failed */
+  DLLM_ERR_TIMEOUT = -4,     /* a device wait gave up (status word set) */
+  DLLM_ERR_WORKSPACE = -5    /* workspace too small */
+} dllm_status;
+
+/* Which keys a block row attends to (block at [s, s+B), sequence start st):
+ *   NONE        [st, s+B), every position recomputed each step (no cache)
+ *   PREFIX      [st, s+B), prefix keys/values from the cache
+ *   DUAL        [st, S),   prefix and suffix from the cache
+ *   DUAL_PRUNED [st, min(s+B+window, S)) plus S-1 when the suffix is not empty */
+typedef enum {
+  DLLM_CACHE_NONE = 0,
+  DLLM_CACHE_PREFIX = 1,
+  DLLM_CACHE_DUAL = 2,
+  DLLM_CACHE_DUAL_PRUNED = 3
+} dllm_cache_mode;
+
+/* Weight storage.  BF16: bf16 weights, K extent = the input width.
+ * F32_SPLIT: fp32 weights stored as two bf16 halves [hi | lo] along K
+ * (made by dllm_split_f32_weights); hi + lo equals the fp32 value to about
+ * 2^-17 relative, and the embedding stays fp32. */
+typedef enum { DLLM_W_BF16 = 0, DLLM_W_F32_SPLIT = 1 } dllm_weight_format;
+
+typedef struct {
+  int32_t batch, n_layers, hidden, n_q_heads, n_kv_heads, head_dim, vocab;
+  int32_t prompt_len; /* P: longest prompt; shorter prompts are left-padded */
+  int32_t gen_len, block, window, mask_id;
+  float tau;        /* commit threshold, strict conf > tau */
+  float rope_theta; /* rotate-half RoPE base; 0 disables RoPE */
+  int32_t mode;          /* dllm_cache_mode */
+  int32_t weight_format; /* dllm_weight_format */
+} dllm_config;
+
+/* Kw = hidden (BF16) or 2*hidden (F32_SPLIT); Ko = Hq*D or 2*Hq*D. */
+typedef struct {
+  const void* wqkv;  /* bf16 [L][(Hq+2Hkv)*D][Kw]; rows: q heads, k heads, v heads */
+  const void* wo;    /* bf16 [L][hidden][Ko] */
+  const void* w_lm;  /* bf16 [V][Kw] */
+  const void* embed; /* [V][hidden]; bf16 (BF16) or fp32 (F32_SPLIT); tied to w_lm */
+} dllm_weights;
+
+typedef struct {
+  int32_t* tokens;          /* [b][S] token ids */
+  uint8_t* masked;          /* [b][S] 1 = still masked; only ever goes 1 -> 0 */
+  const int32_t* seq_start; /* [b] first valid position (left padding before it) */
+  void* k_cache;            /* bf16 [L][b][Hkv][S][D]; must hold finite values */
+  void* v_cache;            /* bf16 [L][b][Hkv][S][D] */
+  const void* plants;       /* bf16 [b][G][hidden] layer-0 input of masked generated rows */
+} dllm_state;
+
+/* Bytes of workspace a configuration needs (host call, no GPU work). */
+dllm_status dllm_workspace_size(const dllm_config* cfg, size_t* bytes);
+
+/* Zero the workspace's counters and status word and build the RoPE table.
+ * Call once per workspace before any other call that takes it. */
+dllm_status dllm_workspace_init(const dllm_config* cfg, void* ws, size_t ws_bytes,
+                                dllm_stream stream);
+
+/* fp32 [rows][cols] -> bf16 [rows][2*cols] with hi = bf16(w), lo = bf16(w - hi). */
+dllm_status dllm_split_f32_weights(const float* src, void* dst, int64_t rows, int64_t cols,
+                                   dllm_stream stream);
+
+/* Layer-0 input of n_rows rows per sequence starting at position row0:
+ * x[b*n_rows+i] = plant of position p = row0+i if use_plants and masked[b][p]
+ * and block_start <= p < block_start+B, else embed[tokens[b][p]].
+ * x fp32 [b*n_rows][hidden]; xb bf16 copy of it. */
+dllm_status dllm_embed_rows(const dllm_config* cfg, const dllm_weights* w,
+                            const dllm_state* st, int32_t row0, int32_t n_rows,
+                            int32_t use_plants, int32_t block_start, float* x, void* xb,
+                            dllm_stream stream);
+
+/* Q/K/V projection of layer `layer` (GEMM on tcgen05, fp32 accumulate) for
+ * n_rows rows per sequence at positions row0.. : RoPE at position p-seq_start
+ * on q and k, q -> q_out bf16 [b][Hq][n_rows][D], k/v -> caches at p.
+ * xb bf16 [b*n_rows][hidden]. */
+dllm_status dllm_qkv_proj(const dllm_config* cfg, const dllm_weights* w, int32_t layer,
+                          const void* xb, int32_t row0, int32_t n_rows,
+                          const int32_t* seq_start, void* q_out, void* k_cache,
+                          void* v_cache, void* ws, size_t ws_bytes, dllm_stream stream);
+
+/* Non-causal GQA attention of n_rows query rows per sequence (q bf16
+ * [b][Hq][n_rows][D]) against layer `layer` of the caches.  Query head h reads
+ * kv head h/(Hq/Hkv).  Keys of sequence i: segs[i][j] = (start, len) for
+ * j = 0,1 (device int32 [b][2][2]; len 0 = unused).  Scale 1/sqrt(D).
+ * out bf16 [b*n_rows][Hq*D]. */
+dllm_status dllm_block_attn(const dllm_config* cfg, int32_t layer, int32_t n_rows,
+                            const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* segs, void* out, void* ws, size_t ws_bytes,
+                            dllm_stream stream);
+
+/* Output projection and residual: x += attn * Wo^T (fp32), xb = bf16(x).  If
+ * h_out is not NULL, rows at positions [block_start, block_start+B) are also
+ * copied as bf16 to h_out [b][B][hidden]. */
+dllm_status dllm_o_proj(const dllm_config* cfg, const dllm_weights* w, int32_t layer,
+                        const void* attn, int32_t row0, int32_t n_rows, float* x, void* xb,
+                        void* h_out, int32_t block_start, void* ws, size_t ws_bytes,
+                        dllm_stream stream);
+
+/* LM head + confidence over the full vocabulary for n_rows rows of h (bf16
+ * [n_rows][hidden]); no logits are written.  conf = max softmax probability,
+ * tok = argmax (lowest id on ties), gap = top-1 minus top-2 logit (may be NULL). */
+dllm_status dllm_lmhead_confidence(const dllm_config* cfg, const dllm_weights* w,
+                                   const void* h, int32_t n_rows, float* conf, int32_t* tok,
+                                   float* gap, void* ws, size_t ws_bytes, dllm_stream stream);
+
+/* Threshold commit of the block at block_start for every sequence: masked
+ * rows with conf > tau commit, and the most confident masked row always does
+ * (lowest position on ties).  conf/tok [b][B].  Updates tokens and masked;
+ * commit (opt, [b][B] u8) marks committed rows; remaining (opt, [b]) gets the
+ * number of rows still masked. */
+dllm_status dllm_threshold_commit(const dllm_config* cfg, int32_t block_start,
+                                  const float* conf, const int32_t* tok, int32_t* tokens,
+                                  uint8_t* masked, uint8_t* commit, int32_t* remaining,
+                                  dllm_stream stream);
+
+/* Fill the caches before decoding: PREFIX runs the prompt, DUAL and
+ * DUAL_PRUNED run prompt plus mask tokens (whole sequence); NONE does nothing. */
+dllm_status dllm_prefill(const dllm_config* cfg, const dllm_weights* w, const dllm_state* st,
+                         void* ws, size_t ws_bytes, dllm_stream stream);
+
+/* One denoising step of the block at block_start: embed, L layers, LM head,
+ * threshold commit.  The step's conf/tok/gap/commit stay in the workspace
+ * (dllm_step_outputs). */
+dllm_status dllm_decode_step(const dllm_config* cfg, const dllm_weights* w,
+                             const dllm_state* st, int32_t block_start, void* ws,
+                             size_t ws_bytes, dllm_stream stream);
+
+/* Recompute the keys/values of a finished block from its committed tokens:
+ * L layers with input embed[token], same key set as a step, no LM head. */
+dllm_status dllm_kv_cache_refresh(const dllm_config* cfg, const dllm_weights* w,
+                                  const dllm_state* st, int32_t block_start, void* ws,
+                                  size_t ws_bytes, dllm_stream stream);
+
+/* Decode one block to completion: steps until no row of the block is masked
+ * in any sequence (or max_steps), then the cache refresh.  Blocks the calling
+ * host thread until the block is done; *steps_taken (host) gets the count. */
+dllm_status dllm_decode_block(const dllm_config* cfg, const dllm_weights* w,
+                              const dllm_state* st, int32_t block_start, int32_t max_steps,
+                              int32_t* steps_taken, void* ws, size_t ws_bytes,
+                              dllm_stream stream);
+
+/* Device pointers (into ws) of the last step's outputs, each [b][B]. */
+dllm_status dllm_step_outputs(const dllm_config* cfg, void* ws, size_t ws_bytes, float** conf,
+                              int32_t** tok, float** gap, uint8_t** commit);
+
+/* Copy the workspace's device status word to *code (host); synchronises stream. */
+dllm_status dllm_device_status(void* ws, int32_t* code, dllm_stream stream);
+
+/* Number of kernels this library has launched in this process. */
+uint64_t dllm_launch_count(void);
+
+const char* dllm_status_string(dllm_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DLLM_H_ */

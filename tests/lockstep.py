@@ -1,0 +1,130 @@
+"""Lockstep comparison of the CUDA decode with the oracle (test helper).
+
+Every step the oracle starts from the GPU's current state (tokens, mask and
+bf16 caches) and recomputes the step; the GPU then runs the same step.
+Confidences must agree within 2e-3, argmax tokens and commit decisions
+exactly, except at rows the oracle flags as ambiguous, where the GPU's choice
+is kept (it is the state the next step starts from) and counted.
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import numpy as np
+import torch
+
+from oracle import dllm_oracle as O
+from tests.gpu_util import f64, rel_l2
+
+CONF_TOL = 2e-3
+
+
+@dataclasses.dataclass
+class Report:
+    steps: int = 0
+    rows: int = 0
+    flagged: int = 0
+    flagged_mismatch: int = 0
+    max_conf_err: float = 0.0
+    max_kv_rel: float = 0.0
+
+
+def state_from_gpu(dec, layers=None) -> O.State:
+    L = dec.w.n_layers if layers is None else layers
+    return O.State(tokens=dec.tokens.cpu().numpy().astype(np.int64),
+                   masked=dec.masked.cpu().numpy().astype(bool),
+                   kcache=f64(dec.k_cache[:L]), vcache=f64(dec.v_cache[:L]),
+                   starts=dec.seq_start.cpu().numpy().astype(np.int64))
+
+
+def compare_step(dec, case, s: int, rep: Report, check_kv: bool = True) -> None:
+    cfg, W = case.cfg, case.W
+    st = state_from_gpu(dec)
+    r = O.decode_step(cfg, W, st, case.plants64, s, apply=False)
+    dec.step(s)
+    torch.cuda.synchronize()
+    assert dec.device_status() == 0
+    conf, tok, gap, commit = (t.cpu().numpy() for t in dec.step_outputs())
+    B = cfg.block
+    for bi in range(cfg.batch):
+        m = ~np.isnan(r.conf[bi])
+        if not m.any():
+            assert not commit[bi].any()
+            continue
+        rep.rows += int(m.sum())
+        err = np.abs(conf[bi][m] - r.conf[bi][m])
+        rep.max_conf_err = max(rep.max_conf_err, float(err.max()))
+        assert err.max() <= CONF_TOL, f"conf error {err.max()} at block {s}"
+        flag = r.amb_tok[bi] | r.amb_commit[bi]
+        rep.flagged += int(flag.sum())
+        tok_bad = m & (tok[bi] != r.tok[bi])
+        com_bad = commit[bi].astype(bool) != r.commit[bi]
+        bad = tok_bad | com_bad
+        assert not (bad & ~flag).any(), (
+            f"block {s} seq {bi}: unflagged mismatch rows {np.where(bad & ~flag)[0]} "
+            f"gpu tok {tok[bi][bad]} oracle {r.tok[bi][bad]} gpu conf {conf[bi][bad]} "
+            f"oracle conf {r.conf[bi][bad]}")
+        rep.flagged_mismatch += int(bad.sum())
+        # the state update matches the step's own commit decisions
+        committed = commit[bi].astype(bool)
+        assert not (committed & ~m).any()
+        toks = dec.tokens[bi, s:s + B].cpu().numpy()
+        assert np.array_equal(toks[committed], tok[bi][committed])
+        assert not dec.masked[bi, s:s + B].cpu().numpy()[committed].any()
+    if check_kv and cfg.mode != O.MODE_NONE:
+        got = f64(dec.k_cache[:, :, :, s:s + B])
+        rep.max_kv_rel = max(rep.max_kv_rel, rel_l2(got, st.kcache[:, :, :, s:s + B]))
+        assert rel_l2(got, st.kcache[:, :, :, s:s + B]) <= 5e-3
+        got = f64(dec.v_cache[:, :, :, s:s + B])
+        assert rel_l2(got, st.vcache[:, :, :, s:s + B]) <= 5e-3
+    rep.steps += 1
+
+
+def compare_refresh(dec, case, s: int) -> None:
+    cfg, W = case.cfg, case.W
+    if cfg.mode == O.MODE_NONE:
+        return
+    st = state_from_gpu(dec)
+    O.refresh_block(cfg, W, st, s)
+    dec.refresh(s)
+    torch.cuda.synchronize()
+    B = cfg.block
+    for cache, ref in ((dec.k_cache, st.kcache), (dec.v_cache, st.vcache)):
+        assert rel_l2(f64(cache[:, :, :, s:s + B]), ref[:, :, :, s:s + B]) <= 5e-3
+
+
+def compare_prefill(dec, case) -> None:
+    cfg, W = case.cfg, case.W
+    dec.prefill()
+    torch.cuda.synchronize()
+    if cfg.mode == O.MODE_NONE:
+        return
+    st = state_from_gpu(dec)
+    st.kcache[:] = 0
+    st.vcache[:] = 0
+    O.prefill(cfg, W, st)
+    end = cfg.prompt_len if cfg.mode == O.MODE_PREFIX else cfg.seq_len
+    for bi in range(cfg.batch):
+        a = int(st.starts[bi])
+        for cache, ref in ((dec.k_cache, st.kcache), (dec.v_cache, st.vcache)):
+            got = f64(cache[:, bi, :, a:end])
+            assert rel_l2(got, ref[:, bi, :, a:end]) <= 5e-3
+
+
+def lockstep(dec, case, max_blocks: int | None = None, max_steps: int | None = None) -> Report:
+    rep = Report()
+    compare_prefill(dec, case)
+    cfg = case.cfg
+    blocks = list(range(cfg.prompt_len, cfg.seq_len, cfg.block))
+    if max_blocks is not None:
+        blocks = blocks[:max_blocks]
+    for s in blocks:
+        n = 0
+        while dec.masked[:, s:s + cfg.block].any():
+            if max_steps is not None and n >= max_steps:
+                break
+            compare_step(dec, case, s, rep)
+            n += 1
+            assert n <= cfg.block
+        compare_refresh(dec, case, s)
+    return rep

@@ -1,0 +1,89 @@
+"""The C-ABI library loads and exports what include/dllm.h declares (no GPU).
+
+Only host-side entry points that launch nothing are called here: the
+workspace-size query and argument validation.
+"""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from diffusion_decoding_step_b200 import abi, build
+from diffusion_decoding_step_b200 import workload as wl
+from diffusion_decoding_step_b200.runtime import make_config
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return abi.lib()
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "dllm.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dllm_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = header_functions()
+    for must in ("dllm_block_attn", "dllm_lmhead_confidence", "dllm_threshold_commit",
+                 "dllm_kv_cache_refresh", "dllm_decode_block"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in header_functions():
+        assert hasattr(lib, name), name
+        assert name in abi.SIGNATURES, f"binding lacks {name}"
+
+
+@pytest.mark.parametrize("name", list(wl.WORKLOADS))
+def test_workspace_size_for_every_workload(lib, name):
+    n = C.c_size_t(0)
+    assert abi.dllm_workspace_size(C.byref(make_config(wl.WORKLOADS[name])), C.byref(n)) == 0
+    assert n.value > 0 and n.value % 256 == 0
+
+
+def _status(w: wl.Workload):
+    n = C.c_size_t(0)
+    return abi.dllm_workspace_size(C.byref(make_config(w)), C.byref(n))
+
+
+def test_rejects_bad_configs(lib):
+    base = wl.WORKLOADS["tiny"]
+    assert _status(base) == abi.DLLM_OK
+    assert _status(base.replace(head_dim=64)) == abi.DLLM_ERR_UNSUPPORTED
+    assert _status(base.replace(n_kv_heads=3)) == abi.DLLM_ERR_INVALID
+    assert _status(base.replace(gen_len=30)) == abi.DLLM_ERR_INVALID
+    assert _status(base.replace(hidden=96)) == abi.DLLM_ERR_UNSUPPORTED
+    assert _status(base.replace(block=128, gen_len=128)) == abi.DLLM_ERR_UNSUPPORTED
+    assert _status(base.replace(vocab=1000, mask_id=5)) == abi.DLLM_ERR_UNSUPPORTED
+    assert _status(base.replace(mask_id=2000)) == abi.DLLM_ERR_INVALID
+    assert abi.dllm_workspace_size(None, None) == abi.DLLM_ERR_INVALID
+
+
+def test_null_pointers_rejected_before_launch(lib):
+    cfg = make_config(wl.WORKLOADS["tiny"])
+    n = C.c_size_t(0)
+    abi.dllm_workspace_size(C.byref(cfg), C.byref(n))
+    # null workspace / weights / state: rejected by validation, nothing launched
+    assert abi.dllm_decode_step(C.byref(cfg), None, None, 64, None, n.value, None) \
+        == abi.DLLM_ERR_INVALID
+    assert abi.dllm_workspace_init(C.byref(cfg), None, n.value, None) == abi.DLLM_ERR_INVALID
+    assert abi.dllm_threshold_commit(C.byref(cfg), 64, None, None, None, None, None, None,
+                                     None) == abi.DLLM_ERR_INVALID
+    # misaligned workspace pointer
+    assert abi.dllm_workspace_init(C.byref(cfg), C.c_void_p(0x1008), n.value, None) \
+        == abi.DLLM_ERR_INVALID
+    # too-small workspace
+    assert abi.dllm_workspace_init(C.byref(cfg), C.c_void_p(0x100000), 256, None) \
+        == abi.DLLM_ERR_WORKSPACE
+
+
+def test_status_strings(lib):
+    assert abi.dllm_status_string(0) == b"ok"
+    assert b"workspace" in abi.dllm_status_string(abi.DLLM_ERR_WORKSPACE)

@@ -1,0 +1,275 @@
+"""Per-kernel parity of the CUDA path against the fp64 oracle (B200 only).
+
+Each test feeds the same seeded bf16 inputs to one C-ABI entry point and to
+the oracle function that defines it, and compares element by element with the
+tolerances of the decode step: bf16 attention output rel-L2 <= 5e-3 and
+max-abs <= 1e-2; confidence abs <= 2e-3; argmax ids, commit masks and token
+updates bit-exact except rows the oracle flags as ambiguous.
+"""
+import ctypes as C
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import dllm_oracle as O
+from diffusion_decoding_step_b200 import workload as wl
+from diffusion_decoding_step_b200.runtime import make_config, workspace_bytes
+from tests.gpu_util import ensure_lib, ptr, stream, f64, bf16_ulp_close, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _ws(w):
+    abi = ensure_lib()
+    cfg = make_config(w)
+    n = workspace_bytes(w)
+    ws = torch.empty(n, dtype=torch.uint8, device=DEV)
+    abi.check(abi.dllm_workspace_init(C.byref(cfg), ptr(ws), n, stream()), "ws init")
+    return abi, cfg, ws, n
+
+
+def _gen(seed):
+    g = torch.Generator(device=DEV)
+    g.manual_seed(seed)
+    return g
+
+
+def _weights_c(abi, wqkv=None, wo=None, w_lm=None, embed=None):
+    return abi.dllm_weights(ptr(wqkv), ptr(wo), ptr(w_lm), ptr(embed if embed is not None else w_lm))
+
+
+# ---------------------------------------------------------------- LM head
+LM_CASES = [  # (rows, hidden, vocab, batch, block)
+    (8, 128, 1024, 1, 8),
+    (32, 512, 8192, 1, 32),
+    (50, 256, 4096, 1, 64),
+    (200, 256, 2048, 4, 64),
+    (512, 512, 4096, 16, 32),
+    (32, 4096, 126464, 1, 32),
+]
+
+
+@pytest.mark.parametrize("R,d,V,b,B", LM_CASES)
+def test_lmhead_confidence_matches_oracle(R, d, V, b, B):
+    w = wl.Workload("t", batch=b, n_layers=1, hidden=d, n_q_heads=1, n_kv_heads=1, head_dim=128,
+                    vocab=V, prompt_len=0, gen_len=B, block=B)
+    abi, cfg, ws, n = _ws(w)
+    g = _gen(R + d + V)
+    W = (torch.randn(V, d, generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    t = torch.randint(0, V, (R,), generator=g, device=DEV)
+    a = torch.rand(R, generator=g, device=DEV) * 20
+    rows = W[t].float()
+    h = a[:, None] * rows / (rows * rows).sum(1, keepdim=True)
+    h = h + torch.randn(R, d, generator=g, device=DEV) / (0.02 * d ** 0.5)
+    h[0] = 0.0  # uniform logits: conf = 1/V, token 0
+    h = h.to(torch.bfloat16)
+    conf = torch.empty(R, dtype=torch.float32, device=DEV)
+    tok = torch.empty(R, dtype=torch.int32, device=DEV)
+    gap = torch.empty(R, dtype=torch.float32, device=DEV)
+    wc = _weights_c(abi, w_lm=W)
+    abi.check(abi.dllm_lmhead_confidence(C.byref(cfg), C.byref(wc), ptr(h), R, ptr(conf),
+                                         ptr(tok), ptr(gap), ptr(ws), n, stream()), "lmhead")
+    torch.cuda.synchronize()
+    c_ref, t_ref, g_ref = O.lm_head_confidence(f64(h), f64(W))
+    c, tk, gp = f64(conf), tok.cpu().numpy(), f64(gap)
+    assert np.abs(c - c_ref).max() <= 2e-3
+    sure = g_ref >= O.AMBIG_GAP
+    assert np.array_equal(tk[sure], t_ref[sure])
+    assert np.abs(gp[sure] - g_ref[sure]).max() < 1e-3
+    assert tk[0] == 0 and abs(c[0] - 1.0 / V) < 1e-6
+    assert (c > 0).all() and (c <= 1.0 + 1e-6).all()
+
+
+# ---------------------------------------------------------------- QKV projection
+QKV_CASES = [  # (hidden, Hq, Hkv, D, batch, n_rows, row0, theta, S)
+    (128, 4, 4, 32, 1, 8, 64, 0.0, 96),
+    (512, 4, 4, 128, 1, 32, 256, 0.0, 512),
+    (896, 7, 1, 128, 2, 32, 512, 1e6, 1024),
+    (4096, 32, 32, 128, 1, 32, 256, 0.0, 512),
+    (3584, 28, 4, 128, 1, 32, 512, 1e6, 1024),
+    (512, 4, 2, 128, 2, 300, 0, 1e4, 300),
+]
+
+
+def _qkv_case(d, Hq, Hkv, D, b, nr, row0, theta, S, f32=False, seed=0):
+    w = wl.Workload("t", batch=b, n_layers=2, hidden=d, n_q_heads=Hq, n_kv_heads=Hkv,
+                    head_dim=D, vocab=1024, prompt_len=S - 32, gen_len=32, block=32,
+                    rope_theta=theta, weight_f32=f32)
+    abi, cfg, ws, n = _ws(w)
+    g = _gen(seed + d + nr)
+    rows = w.qkv_rows
+    Wf = torch.randn(2, rows, d, generator=g, device=DEV) * 0.02
+    x = torch.randn(b * nr, d, generator=g, device=DEV).to(torch.bfloat16)
+    starts = torch.randint(0, 5, (b,), generator=g, device=DEV).to(torch.int32)
+    if f32:
+        Wk = torch.empty(2, rows, 2 * d, dtype=torch.bfloat16, device=DEV)
+        abi.check(abi.dllm_split_f32_weights(ptr(Wf.contiguous()), ptr(Wk), 2 * rows, d,
+                                             stream()), "split")
+        Wref = f64(Wf)
+    else:
+        Wk = Wf.to(torch.bfloat16)
+        Wref = f64(Wk)
+    q = torch.zeros(b, Hq, nr, D, dtype=torch.bfloat16, device=DEV)
+    kc = torch.zeros(2, b, Hkv, S, D, dtype=torch.bfloat16, device=DEV)
+    vc = torch.zeros_like(kc)
+    wc = _weights_c(abi, wqkv=Wk, wo=Wk, w_lm=Wk)
+    layer = 1
+    abi.check(abi.dllm_qkv_proj(C.byref(cfg), C.byref(wc), layer, ptr(x), row0, nr, ptr(starts),
+                                ptr(q), ptr(kc), ptr(vc), ptr(ws), n, stream()), "qkv")
+    torch.cuda.synchronize()
+    X = f64(x).reshape(b, nr, d)
+    qkv = X @ Wref[layer].T
+    qr = qkv[..., :Hq * D].reshape(b, nr, Hq, D).transpose(0, 2, 1, 3)
+    kr = qkv[..., Hq * D:(Hq + Hkv) * D].reshape(b, nr, Hkv, D).transpose(0, 2, 1, 3)
+    vr = qkv[..., (Hq + Hkv) * D:].reshape(b, nr, Hkv, D).transpose(0, 2, 1, 3)
+    if theta > 0:
+        st = starts.cpu().numpy()
+        for bi in range(b):
+            pos = np.maximum(np.arange(row0, row0 + nr) - st[bi], 0)
+            qr[bi] = O.rope(qr[bi], pos, theta)
+            kr[bi] = O.rope(kr[bi], pos, theta)
+    return (f64(q), qr, f64(kc[layer, :, :, row0:row0 + nr]), kr,
+            f64(vc[layer, :, :, row0:row0 + nr]), vr, kc, vc, row0, nr)
+
+
+@pytest.mark.parametrize("case", QKV_CASES)
+def test_qkv_projection_rope_and_cache_write(case):
+    q, qr, k, kr, v, vr, kc, vc, row0, nr = _qkv_case(*case)
+    for gpu, ref in ((q, qr), (k, kr), (v, vr)):
+        bf16_ulp_close(gpu, O.round_bf16(ref), ulps=1.0, atol=1e-6)
+    # nothing outside the rows was written
+    assert float(kc[1, :, :, :row0].abs().sum()) == 0.0
+    assert float(vc[1, :, :, row0 + nr:].abs().sum()) == 0.0
+    assert float(kc[0].abs().sum()) == 0.0
+
+
+def test_qkv_projection_f32_split_weights():
+    q, qr, k, kr, v, vr, *_ = _qkv_case(128, 4, 4, 32, 1, 8, 64, 0.0, 96, f32=True)
+    for gpu, ref in ((q, qr), (k, kr), (v, vr)):
+        bf16_ulp_close(gpu, O.round_bf16(ref), ulps=1.0, atol=1e-6)
+
+
+# ---------------------------------------------------------------- O projection
+OPROJ_CASES = [  # (hidden, Hq, D, batch, n_rows, block_start)
+    (128, 4, 32, 1, 8, 64),
+    (4096, 32, 128, 1, 32, 256),
+    (3584, 28, 128, 1, 32, 512),
+    (512, 4, 128, 2, 96, 32),
+    (512, 8, 128, 16, 32, 0),
+]
+
+
+@pytest.mark.parametrize("d,Hq,D,b,nr,blk", OPROJ_CASES)
+def test_output_projection_residual(d, Hq, D, b, nr, blk):
+    w = wl.Workload("t", batch=b, n_layers=2, hidden=d, n_q_heads=Hq, n_kv_heads=Hq, head_dim=D,
+                    vocab=1024, prompt_len=max(blk, 32), gen_len=max(nr, 32), block=32)
+    abi, cfg, ws, n = _ws(w)
+    g = _gen(d + nr)
+    Wo = (torch.randn(2, d, Hq * D, generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+    attn = torch.randn(b * nr, Hq * D, generator=g, device=DEV).to(torch.bfloat16)
+    x = torch.randn(b * nr, d, generator=g, device=DEV)
+    x0 = x.clone()
+    xb = torch.zeros(b * nr, d, dtype=torch.bfloat16, device=DEV)
+    h = torch.zeros(b, 32, d, dtype=torch.bfloat16, device=DEV)
+    wc = _weights_c(abi, wqkv=Wo, wo=Wo, w_lm=Wo)
+    row0 = blk
+    abi.check(abi.dllm_o_proj(C.byref(cfg), C.byref(wc), 1, ptr(attn), row0, nr, ptr(x), ptr(xb),
+                              ptr(h), blk, ptr(ws), n, stream()), "oproj")
+    torch.cuda.synchronize()
+    ref = f64(x0) + f64(attn) @ f64(Wo[1]).T
+    got = f64(x)
+    assert np.abs(got - ref).max() <= 1e-4 * (1 + np.abs(ref).max())
+    bf16_ulp_close(f64(xb), O.round_bf16(got), ulps=0.0, atol=0.0)
+    # h_out holds the block rows [blk, blk+32) of each sequence
+    hb = f64(h)
+    for bi in range(b):
+        for i in range(min(32, nr)):
+            np.testing.assert_array_equal(hb[bi, i], f64(xb)[bi * nr + i])
+
+
+# ---------------------------------------------------------------- attention
+ATTN_CASES = [  # (Hq, Hkv, D, batch, n_rows, S, segs per sequence, layer)
+    (32, 32, 128, 1, 32, 512, [[(0, 512), (0, 0)]], 0),
+    (28, 4, 128, 1, 32, 1024, [[(0, 576), (0, 0)]], 1),
+    (2, 2, 128, 2, 5, 300, [[(3, 250), (299, 1)], [(0, 77), (0, 0)]], 0),
+    (4, 4, 32, 1, 8, 96, [[(0, 72), (0, 0)]], 0),
+    (4, 4, 32, 1, 1, 96, [[(40, 1), (0, 0)]], 0),
+    (28, 4, 128, 1, 64, 2300, [[(0, 2200), (2299, 1)]], 0),
+    (8, 8, 128, 3, 32, 1280, [[(300, 980), (0, 0)], [(0, 1280), (0, 0)], [(512, 768), (0, 0)]], 1),
+    (4, 2, 128, 1, 700, 700, [[(0, 700), (0, 0)]], 0),
+]
+
+
+@pytest.mark.parametrize("Hq,Hkv,D,b,nr,S,segs,layer", ATTN_CASES)
+def test_block_attention_matches_oracle(Hq, Hkv, D, b, nr, S, segs, layer):
+    w = wl.Workload("t", batch=b, n_layers=2, hidden=max(128, Hq * D), n_q_heads=Hq,
+                    n_kv_heads=Hkv, head_dim=D, vocab=1024, prompt_len=S - 32, gen_len=32,
+                    block=32)
+    abi, cfg, ws, n = _ws(w)
+    g = _gen(Hq * S + nr)
+    q = torch.randn(b, Hq, nr, D, generator=g, device=DEV).to(torch.bfloat16)
+    kc = torch.randn(2, b, Hkv, S, D, generator=g, device=DEV).to(torch.bfloat16)
+    vc = torch.randn(2, b, Hkv, S, D, generator=g, device=DEV).to(torch.bfloat16)
+    sg = torch.tensor([[v for seg in s for v in seg] for s in segs], dtype=torch.int32, device=DEV)
+    out = torch.zeros(b * nr, Hq * D, dtype=torch.bfloat16, device=DEV)
+    abi.check(abi.dllm_block_attn(C.byref(cfg), layer, nr, ptr(q), ptr(kc), ptr(vc), ptr(sg),
+                                  ptr(out), ptr(ws), n, stream()), "attn")
+    torch.cuda.synchronize()
+    Q, K, V = f64(q), f64(kc[layer]), f64(vc[layer])
+    ref = np.zeros((b, nr, Hq, D))
+    gsz = Hq // Hkv
+    for bi in range(b):
+        keys = np.concatenate([np.arange(s0, s0 + ln) for s0, ln in segs[bi]]).astype(int)
+        for h in range(Hq):
+            ref[bi, :, h] = O.attention(Q[bi, h], K[bi, h // gsz][keys], V[bi, h // gsz][keys])
+    got = f64(out).reshape(b, nr, Hq, D)
+    assert rel_l2(got, ref) <= 5e-3
+    assert np.abs(got - ref).max() <= 1e-2
+
+
+# ---------------------------------------------------------------- commit
+@pytest.mark.parametrize("b,B,tau", [(1, 8, 0.9), (1, 32, 0.9), (16, 32, 0.9), (4, 64, 0.5),
+                                     (3, 32, 1.5), (2, 32, 1e-6)])
+def test_threshold_commit_bit_exact(b, B, tau):
+    w = wl.Workload("t", batch=b, n_layers=1, hidden=128, n_q_heads=4, n_kv_heads=4,
+                    head_dim=32, vocab=1024, prompt_len=64, gen_len=2 * B, block=B, tau=tau)
+    abi = ensure_lib()
+    cfg = make_config(w)
+    rng = np.random.default_rng(b * 100 + B)
+    S = w.seq_len
+    s = w.prompt_len + B
+    conf = rng.uniform(0, 1, (b, B)).astype(np.float32)
+    conf[0, :3] = 0.95
+    conf[0, 3] = np.float32(tau) if tau < 1 else 0.5     # exactly tau: does not clear it
+    if B > 8:
+        conf[-1, 5] = conf[-1, 6] = 0.99999               # equal confidences
+    masked = np.zeros((b, S), dtype=np.uint8)
+    masked[:, s:s + B] = rng.uniform(size=(b, B)) < 0.7
+    masked[0, s:s + B] = 1
+    if b > 1:
+        masked[1, s:s + B] = 0                             # a finished sequence
+    tok = rng.integers(0, 1024, (b, B)).astype(np.int32)
+    tokens = rng.integers(0, 1024, (b, S)).astype(np.int32)
+    t_tokens = torch.tensor(tokens, device=DEV)
+    t_masked = torch.tensor(masked, device=DEV)
+    commit = torch.zeros(b, B, dtype=torch.uint8, device=DEV)
+    remaining = torch.zeros(b, dtype=torch.int32, device=DEV)
+    abi.check(abi.dllm_threshold_commit(C.byref(cfg), s, ptr(torch.tensor(conf, device=DEV)),
+                                        ptr(torch.tensor(tok, device=DEV)), ptr(t_tokens),
+                                        ptr(t_masked), ptr(commit), ptr(remaining), stream()),
+              "commit")
+    torch.cuda.synchronize()
+    for bi in range(b):
+        m = masked[bi, s:s + B].astype(bool)
+        c_ref = O.threshold_commit(conf[bi].astype(np.float64), m, tau)
+        assert np.array_equal(commit[bi].cpu().numpy().astype(bool), c_ref)
+        want_tok = tokens[bi].copy()
+        want_tok[s:s + B][c_ref] = tok[bi][c_ref]
+        want_mask = masked[bi].copy()
+        want_mask[s:s + B][c_ref] = 0
+        assert np.array_equal(t_tokens[bi].cpu().numpy(), want_tok)
+        assert np.array_equal(t_masked[bi].cpu().numpy(), want_mask)
+        assert int(remaining[bi]) == int(m.sum() - c_ref.sum())
