@@ -30,6 +30,16 @@ id; "clears the threshold" is strict ``conf > tau``; at least the single most
 confident masked row commits each step (lowest position on ties); the key set
 per cache mode is given by :func:`key_positions`.
 
+Layer stack.  The backbones the workloads are shaped like (LLaDA-8B,
+Dream-7B / Qwen2.5-7B) are pre-norm transformers; with the MLP replaced by identity each layer is
+    x <- x + Wo . attention(q, k, v),   (q, k, v) = W_qkv . x / rms(x)
+with a weightless RMSNorm (eps 1e-6), and the LM head reads the final
+RMSNorm of the residual.  Without the norms, random N(0, 0.02^2) weights at
+d = 4096 have operator norm ~1.3 and the residual overflows within ~24
+layers.  A masked row's layer-0 input is the embedding of the mask token;
+its planted hidden state is added to the LM-head input (final normalised
+hidden state), which keeps the planted confidence spread at any depth.
+
 Precision.  Everything is float64.  With ``mirror=True`` values are rounded at
 the points where the CUDA path stores them: the projection input (bf16), q/k/v
 after RoPE (bf16), the attention output (bf16), the residual stream after each
@@ -66,6 +76,14 @@ def round_bf16(x) -> np.ndarray:
 
 def round_f32(x) -> np.ndarray:
     return np.asarray(x, dtype=np.float64).astype(np.float32).astype(np.float64)
+
+
+RMS_EPS = 1e-6
+
+
+def inv_rms(x: np.ndarray) -> np.ndarray:
+    """1 / sqrt(mean(x^2) + eps) over the last axis (weightless RMSNorm scale)."""
+    return 1.0 / np.sqrt(np.mean(x * x, axis=-1) + RMS_EPS)
 
 
 # --------------------------------------------------------------------------
@@ -231,11 +249,13 @@ def forward_rows(cfg: Config, W: Weights, x0: np.ndarray, rows: np.ndarray,
                  starts: np.ndarray, mirror: bool) -> np.ndarray:
     """Run the layer stack for query rows at positions ``rows`` of every sequence.
 
-    x0 [b, n, d] is the layer-0 input.  Per layer: project to q/k/v (rotary
-    embedding at position p - start on q and k when rope_theta > 0), write this
-    layer's k/v of the rows into the caches ([L, b, Hkv, S, D]), attend every
-    row to the key positions keys[b], add the output projection to the
-    residual.  Returns the final residual [b, n, d].
+    x0 [b, n, d] is the layer-0 input.  Per layer: project the RMS-normalised
+    residual to q/k/v (rotary embedding at position p - start on q and k when
+    rope_theta > 0), write this layer's k/v of the rows into the caches
+    ([L, b, Hkv, S, D]), attend every row to the key positions keys[b], add
+    the output projection to the residual.  Returns the final residual
+    [b, n, d].  (The projection input is bf16(x) scaled by 1/rms(x) after the
+    product, the order in which the CUDA path rounds.)
     """
     b, n, d = x0.shape
     Hq, Hkv, D = cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim
@@ -243,7 +263,7 @@ def forward_rows(cfg: Config, W: Weights, x0: np.ndarray, rows: np.ndarray,
     x = round_f32(x0) if mirror else x0.copy()
     for layer in range(cfg.n_layers):
         xin = round_bf16(x) if mirror else x
-        qkv = xin @ W.wqkv(layer).T                         # [b, n, (Hq+2Hkv)D]
+        qkv = (xin @ W.wqkv(layer).T) * inv_rms(x)[..., None]   # [b, n, (Hq+2Hkv)D]
         q = qkv[..., :Hq * D].reshape(b, n, Hq, D).transpose(0, 2, 1, 3)
         k = qkv[..., Hq * D:(Hq + Hkv) * D].reshape(b, n, Hkv, D).transpose(0, 2, 1, 3)
         v = qkv[..., (Hq + Hkv) * D:].reshape(b, n, Hkv, D).transpose(0, 2, 1, 3)
@@ -301,19 +321,23 @@ def prefill(cfg: Config, W: Weights, st: State, mirror: bool = True) -> None:
     S = cfg.seq_len
     end = cfg.prompt_len if cfg.mode == MODE_PREFIX else S
     rows = np.arange(0, end)
-    x0 = W.embed(st.tokens[:, :end])
+    x0 = W.embed(input_ids(cfg, st, 0, end))
     keys = [np.arange(st.starts[bi], end) for bi in range(cfg.batch)]
     forward_rows(cfg, W, x0, rows, keys, st.kcache, st.vcache, st.starts, mirror)
 
 
-def block_inputs(cfg: Config, W: Weights, st: State, plants: np.ndarray, s: int) -> np.ndarray:
-    """Layer-0 input of the block rows: the plant where masked, else E[token]."""
-    B = cfg.block
-    x0 = W.embed(st.tokens[:, s:s + B])
+def input_ids(cfg: Config, st: State, lo: int, hi: int) -> np.ndarray:
+    """Token ids fed to the embedding for positions [lo, hi): mask_id where masked."""
+    return np.where(st.masked[:, lo:hi], cfg.mask_id, st.tokens[:, lo:hi])
+
+
+def lm_input(cfg: Config, x: np.ndarray, plants: np.ndarray, masked: np.ndarray, s: int,
+             mirror: bool) -> np.ndarray:
+    """LM-head input of the block rows: RMSNorm(x) plus the plant where masked."""
     gi = s - cfg.prompt_len
-    pl = plants[:, gi:gi + B, :]
-    m = st.masked[:, s:s + B]
-    return np.where(m[..., None], pl, x0)
+    pl = plants[:, gi:gi + cfg.block, :]
+    h = x * inv_rms(x)[..., None] + np.where(masked[..., None], pl, 0.0)
+    return round_bf16(h) if mirror else h
 
 
 @dataclasses.dataclass
@@ -337,21 +361,20 @@ def decode_step(cfg: Config, W: Weights, st: State, plants: np.ndarray, s: int,
     Without a cache (MODE_NONE) all positions [start, s+B) are recomputed.
     """
     B, b = cfg.block, cfg.batch
-    x0_blk = block_inputs(cfg, W, st, plants, s)
     if cfg.mode == MODE_NONE:
         rows = np.arange(0, s + B)
-        x0 = W.embed(st.tokens[:, :s + B])
-        x0[:, s:s + B] = x0_blk
+        x0 = W.embed(input_ids(cfg, st, 0, s + B))
         keys = [np.arange(st.starts[bi], s + B) for bi in range(b)]
         shape = (cfg.n_layers, b, cfg.n_kv_heads, cfg.seq_len, cfg.head_dim)
         kc, vc = np.zeros(shape), np.zeros(shape)
         x = forward_rows(cfg, W, x0, rows, keys, kc, vc, st.starts, mirror)[:, s:s + B]
     else:
         rows = np.arange(s, s + B)
+        x0 = W.embed(input_ids(cfg, st, s, s + B))
         keys = [key_positions(cfg.mode, s, B, cfg.seq_len, cfg.window, st.starts[bi])
                 for bi in range(b)]
-        x = forward_rows(cfg, W, x0_blk, rows, keys, st.kcache, st.vcache, st.starts, mirror)
-    h = round_bf16(x) if mirror else x
+        x = forward_rows(cfg, W, x0, rows, keys, st.kcache, st.vcache, st.starts, mirror)
+    h = lm_input(cfg, x, plants, st.masked[:, s:s + B], s, mirror)
     conf = np.full((b, B), np.nan)
     tok = np.full((b, B), -1, dtype=np.int64)
     gap = np.full((b, B), np.inf)

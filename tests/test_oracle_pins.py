@@ -31,6 +31,32 @@ def test_round_bf16_ties_to_even():
     assert O.round_bf16(1.0 + 3 * 2.0 ** -8) == 1.0 + 2.0 ** -6
 
 
+# ---------------------------------------------------------------- rms norm
+def test_inv_rms_closed_form_and_scale_invariance():
+    x = np.array([[3.0, 4.0], [0.0, 0.0]])
+    r = O.inv_rms(x)
+    assert abs(r[0] - 1.0 / np.sqrt(12.5 + 1e-6)) < 1e-15
+    assert abs(r[1] - 1.0 / np.sqrt(1e-6)) < 1e-6
+    y = RNG.standard_normal((4, 64)) * 5
+    for c in (0.25, 3.0, 1e3):
+        np.testing.assert_allclose((c * y) * O.inv_rms(c * y)[:, None], y * O.inv_rms(y)[:, None],
+                                   rtol=1e-6)
+    z = y * O.inv_rms(y)[:, None]
+    np.testing.assert_allclose((z * z).mean(axis=1), 1.0, rtol=1e-6)
+
+
+def test_deep_stack_stays_finite():
+    # 24 layers of d = 512 with N(0, 0.02^2) weights: without the
+    # normalisation the residual would grow by ~1.3x per layer
+    w = TINY.replace(n_layers=24, hidden=512, n_q_heads=4, n_kv_heads=4, head_dim=128,
+                     gen_len=8, weight_f32=False, mode=wl.MODE_DUAL)
+    tr = Case(w).decode(max_steps=1)
+    r = tr.steps[0][1]
+    assert np.isfinite(r.hidden).all()
+    assert np.abs(r.hidden).max() < 1e3
+    assert (r.conf[0] > 0.5).any() and (r.conf[0] < 0.1).any()
+
+
 # ---------------------------------------------------------------- rope
 def test_rope_position_zero_is_identity():
     x = RNG.standard_normal((5, 3, 16))
@@ -276,8 +302,7 @@ def test_dual_step_equals_fresh_full_forward_at_one_layer():
     s = w.prompt_len
     r = O.decode_step(cfg, W, st, case.plants64, s, apply=False)
     S = w.seq_len
-    x0 = W.embed(case.tokens.numpy()[:, :S])
-    x0[:, s:s + w.block] = case.plants64[:, :w.block]
+    x0 = W.embed(case.tokens.numpy()[:, :S])       # masked positions hold mask_id
     shape = (cfg.n_layers, 1, cfg.n_kv_heads, S, cfg.head_dim)
     kc, vc = np.zeros(shape), np.zeros(shape)
     x = O.forward_rows(cfg, W, x0, np.arange(S), [np.arange(S)], kc, vc, np.zeros(1, int), True)
@@ -386,7 +411,8 @@ def test_refresh_writes_committed_block_kv():
         O.decode_step(cfg, W, st, case.plants64, s)
     O.refresh_block(cfg, W, st, s)
     D, Hq, Hkv = w.head_dim, w.n_q_heads, w.n_kv_heads
-    x = O.round_bf16(W.embed(st.tokens[0, s:s + w.block]))
-    k = x @ W.wqkv(0)[Hq * D:(Hq + Hkv) * D].T
+    e = W.embed(st.tokens[0, s:s + w.block])
+    scale = 1.0 / np.sqrt((e * e).mean(axis=1) + 1e-6)
+    k = (O.round_bf16(e) @ W.wqkv(0)[Hq * D:(Hq + Hkv) * D].T) * scale[:, None]
     want = O.round_bf16(k.reshape(w.block, Hkv, D).transpose(1, 0, 2))
     np.testing.assert_array_equal(st.kcache[0, 0][:, s:s + w.block], want)
