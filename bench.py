@@ -40,7 +40,43 @@ def parse():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", action="store_true",
+                    help="profiling run: prefill, then --warmup + --steps single denoising "
+                         "steps of the first block; prints launch counts, no JSON line")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="profiling only: override the layer count (smaller device footprint)")
     return ap.parse_args()
+
+
+def run_profile(args):
+    """Small, fixed launch sequence for ncu: prefill, then single steps."""
+    import torch
+    from diffusion_decoding_step_b200 import abi, build
+    from diffusion_decoding_step_b200 import workload as wl
+    from diffusion_decoding_step_b200.runtime import Decoder
+
+    build.build()
+    w = wl.WORKLOADS[args.workload]
+    if args.layers:
+        w = w.replace(n_layers=args.layers)
+    weights = wl.make_weights(w, device="cuda")
+    tokens, masked = wl.make_tokens(w)
+    plants = wl.make_plants(w, weights.w_lm)
+    dec = Decoder(w, weights, tokens, masked, wl.seq_starts(w), plants)
+    dec.prefill()
+    torch.cuda.synchronize()
+    n0 = abi.dllm_launch_count()
+    for _ in range(args.warmup):
+        dec.step(w.prompt_len)
+    torch.cuda.synchronize()
+    n1 = abi.dllm_launch_count()
+    for _ in range(args.steps):
+        dec.step(w.prompt_len)
+    torch.cuda.synchronize()
+    n2 = abi.dllm_launch_count()
+    assert dec.device_status() == 0
+    print(f"profile {w.name} layers={w.n_layers}: launches before warm-up {n0}, "
+          f"warm-up {n1 - n0}, timed {n2 - n1} ({(n2 - n1) // max(1, args.steps)} per step)")
 
 
 def peaks():
@@ -260,19 +296,22 @@ def run_ours(args, rank, world, local_rank):
     cfg_p = C.byref(dec.cfg)
     q = torch.empty(rows * w.n_q_heads * w.head_dim, dtype=torch.bfloat16, device=dev)
     xb = torch.randn(rows, w.hidden, device=dev).to(torch.bfloat16)
+    sumsq = torch.ones(rows, w.hidden // 128, device=dev)
     sh = C.c_void_p(stream.cuda_stream)
     iters = 3 * w.n_layers
     for _ in range(2):
         for l in range(w.n_layers):
-            abi.check(abi.dllm_qkv_proj(cfg_p, C.byref(dec.weights_c), l, _ptr(xb), s, w.block,
+            abi.check(abi.dllm_qkv_proj(cfg_p, C.byref(dec.weights_c), l, _ptr(xb),
+                                        _ptr(sumsq), s, w.block,
                                         _ptr(dec.seq_start), _ptr(q), _ptr(dec.k_cache),
                                         _ptr(dec.v_cache), _ptr(dec.ws), dec.ws_bytes, sh), "qkv")
     k0 = torch.cuda.Event(enable_timing=True)
     k1 = torch.cuda.Event(enable_timing=True)
     k0.record(stream)
     for i in range(iters):
-        abi.check(abi.dllm_qkv_proj(cfg_p, C.byref(dec.weights_c), i % w.n_layers, _ptr(xb), s,
-                                    w.block, _ptr(dec.seq_start), _ptr(q), _ptr(dec.k_cache),
+        abi.check(abi.dllm_qkv_proj(cfg_p, C.byref(dec.weights_c), i % w.n_layers, _ptr(xb),
+                                    _ptr(sumsq), s, w.block, _ptr(dec.seq_start), _ptr(q),
+                                    _ptr(dec.k_cache),
                                     _ptr(dec.v_cache), _ptr(dec.ws), dec.ws_bytes, sh), "qkv")
     k1.record(stream)
     torch.cuda.synchronize(dev)
@@ -366,6 +405,9 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.profile:
+        run_profile(args)
         return
     if world > 1:
         import datetime

@@ -52,10 +52,12 @@ SIGNATURES = {
     "dllm_workspace_size": (C.c_int, [_CFG, C.POINTER(C.c_size_t)]),
     "dllm_workspace_init": (C.c_int, [_CFG, _P, C.c_size_t, _P]),
     "dllm_split_f32_weights": (C.c_int, [_P, _P, C.c_int64, C.c_int64, _P]),
-    "dllm_embed_rows": (C.c_int, [_CFG, _W, _ST, _I, _I, _I, _I, _P, _P, _P]),
-    "dllm_qkv_proj": (C.c_int, [_CFG, _W, _I, _P, _I, _I, _P, _P, _P, _P, _P, C.c_size_t, _P]),
+    "dllm_embed_rows": (C.c_int, [_CFG, _W, _ST, _I, _I, _P, _P, _P, _P]),
+    "dllm_qkv_proj": (C.c_int, [_CFG, _W, _I, _P, _P, _I, _I, _P, _P, _P, _P, _P, C.c_size_t,
+                                _P]),
     "dllm_block_attn": (C.c_int, [_CFG, _I, _I, _P, _P, _P, _P, _P, _P, C.c_size_t, _P]),
-    "dllm_o_proj": (C.c_int, [_CFG, _W, _I, _P, _I, _I, _P, _P, _P, _I, _P, C.c_size_t, _P]),
+    "dllm_o_proj": (C.c_int, [_CFG, _W, _I, _P, _I, _I, _P, _P, _P, _P, C.c_size_t, _P]),
+    "dllm_final_norm": (C.c_int, [_CFG, _P, _I, _I, _I, _P, _P, _P, _P]),
     "dllm_lmhead_confidence": (C.c_int, [_CFG, _W, _P, _I, _P, _P, _P, _P, C.c_size_t, _P]),
     "dllm_threshold_commit": (C.c_int, [_CFG, _I, _P, _P, _P, _P, _P, _P, _P]),
     "dllm_prefill": (C.c_int, [_CFG, _W, _ST, _P, C.c_size_t, _P]),

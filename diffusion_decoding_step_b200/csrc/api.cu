@@ -177,8 +177,8 @@ int key_tiles_bound(const Shape& s, int blk, int seg_end) {
 
 // ------------------------------------------------------------------ workspace
 struct Layout {
-  size_t status, gcnt, acnt, x, xb, q, attn, h, slots, stats, part_o, part_ml, conf, tok, gap,
-      commit, remaining, segs, rope, total;
+  size_t status, gcnt, acnt, x, xb, sumsq, q, attn, h, slots, stats, part_o, part_ml, conf, tok,
+      gap, commit, remaining, segs, rope, total;
   int rmax, lm_slots, gcnt_n, acnt_n;
 };
 
@@ -243,6 +243,7 @@ Layout layout(const Shape& s) {
   l.acnt = take((size_t)acnt * 4);
   l.x = take((size_t)l.rmax * s.d * 4);
   l.xb = take((size_t)l.rmax * s.d * 2);
+  l.sumsq = take((size_t)l.rmax * (s.d / 128) * 4);
   l.q = take((size_t)l.rmax * s.Hq * s.D * 2);
   l.attn = take((size_t)l.rmax * s.Hq * s.D * 2);
   l.h = take((size_t)s.b * s.B * s.d * 2);
@@ -297,8 +298,9 @@ dllm_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DLLM_OK : DLL
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // ------------------------------------------------------------------ launches
-dllm_status run_qkv(const Ctx& c, const void* wqkv, int layer, const void* xb, int row0,
-                    int n_rows, const int* seq_start, void* q_out, void* kc, void* vc, bool pdl) {
+dllm_status run_qkv(const Ctx& c, const void* wqkv, int layer, const void* xb,
+                    const float* sumsq, int row0, int n_rows, const int* seq_start, void* q_out,
+                    void* kc, void* vc, bool pdl) {
   const Shape& s = c.s;
   const int R = s.b * n_rows;
   const GemmPlan g = plan_gemm(s.qkv_rows, R, s.Kw, true);
@@ -329,6 +331,10 @@ dllm_status run_qkv(const Ctx& c, const void* wqkv, int layer, const void* xb, i
   p.S = s.S;
   p.batch = s.b;
   p.rope_tab = s.theta > 0.f ? c.at<float2>(c.l.rope) : nullptr;
+  p.sumsq_in = sumsq;
+  p.npart = s.d / 128;
+  p.d_norm = s.d;
+  p.rms_eps = kRmsEps;
   p.q_out = static_cast<__nv_bfloat16*>(q_out);
   p.k_cache = static_cast<__nv_bfloat16*>(kc);
   p.v_cache = static_cast<__nv_bfloat16*>(vc);
@@ -336,7 +342,7 @@ dllm_status run_qkv(const Ctx& c, const void* wqkv, int layer, const void* xb, i
 }
 
 dllm_status run_oproj(const Ctx& c, const void* wo, int layer, const void* attn, int row0,
-                      int n_rows, float* x, void* xb, void* h_out, int blk_start, bool pdl) {
+                      int n_rows, float* x, void* xb, float* sumsq, bool pdl) {
   const Shape& s = c.s;
   const int R = s.b * n_rows;
   const GemmPlan g = plan_gemm(s.d, R, s.Ko, true);
@@ -363,9 +369,9 @@ dllm_status run_oproj(const Ctx& c, const void* wo, int layer, const void* attn,
   p.x = x;
   p.xb = static_cast<__nv_bfloat16*>(xb);
   p.d_model = s.d;
-  p.h_out = static_cast<__nv_bfloat16*>(h_out);
-  p.blk_start = blk_start;
-  p.blk_len = s.B;
+  p.sumsq_out = sumsq;
+  p.npart = s.d / 128;
+  p.d_norm = s.d;
   return cuda_status(launch_gemm(EPI_OPROJ, g.nt, wm, xm, p, g.grid, pdl, c.st));
 }
 
@@ -414,26 +420,27 @@ dllm_status run_attn(const Ctx& c, int layer, int n_rows, const void* q, const v
 }
 
 dllm_status run_embed(const Ctx& c, const dllm_weights* w, const dllm_state* stt, int row0,
-                      int n_rows, int use_plants, int blk_start, int seg_end, bool pdl) {
+                      int n_rows, int blk_start, int seg_end, bool pdl) {
   const Shape& s = c.s;
   EmbedParams e{};
   e.batch = s.b;
   e.S = s.S;
-  e.G = s.G;
-  e.P = s.P;
   e.d = s.d;
   e.n_rows = n_rows;
   e.row0 = row0;
-  e.use_plants = use_plants;
   e.blk_start = blk_start;
   e.blk_len = s.B;
   e.embed_f32 = s.wfmt == DLLM_W_F32_SPLIT;
+  e.vocab = s.V;
+  e.mask_id = s.mask_id;
+  e.npart = s.d / 128;
+  e.status = c.at<int>(c.l.status);
   e.tokens = stt->tokens;
   e.masked = stt->masked;
   e.embed = w->embed;
-  e.plants = static_cast<const __nv_bfloat16*>(stt->plants);
   e.x = c.at<float>(c.l.x);
   e.xb = c.at<__nv_bfloat16>(c.l.xb);
+  e.sumsq = c.at<float>(c.l.sumsq);
   e.segs = c.at<int>(c.l.segs);
   e.seq_start = stt->seq_start;
   e.mode = s.mode;
@@ -442,22 +449,42 @@ dllm_status run_embed(const Ctx& c, const dllm_weights* w, const dllm_state* stt
   return cuda_status(launch_embed(e, pdl, c.st));
 }
 
-// Embed + L layers for n_rows rows per sequence at row0.  When h_out is set,
-// the last layer copies the block rows to it.
+// Embed + L pre-norm layers for n_rows rows per sequence at row0.
 dllm_status run_forward(const Ctx& c, const dllm_weights* w, const dllm_state* stt, int row0,
-                        int n_rows, int use_plants, int blk_start, int seg_end, void* h_out) {
+                        int n_rows, int blk_start, int seg_end) {
   const Shape& s = c.s;
-  DLLM_TRY(run_embed(c, w, stt, row0, n_rows, use_plants, blk_start, seg_end, true));
+  DLLM_TRY(run_embed(c, w, stt, row0, n_rows, blk_start, seg_end, true));
   const int ntb = key_tiles_bound(s, blk_start, seg_end);
   for (int l = 0; l < s.L; ++l) {
-    DLLM_TRY(run_qkv(c, w->wqkv, l, c.at<void>(c.l.xb), row0, n_rows, stt->seq_start,
-                     c.at<void>(c.l.q), stt->k_cache, stt->v_cache, true));
+    DLLM_TRY(run_qkv(c, w->wqkv, l, c.at<void>(c.l.xb), c.at<float>(c.l.sumsq), row0, n_rows,
+                     stt->seq_start, c.at<void>(c.l.q), stt->k_cache, stt->v_cache, true));
     DLLM_TRY(run_attn(c, l, n_rows, c.at<void>(c.l.q), stt->k_cache, stt->v_cache,
                       c.at<int>(c.l.segs), c.at<void>(c.l.attn), ntb, true));
     DLLM_TRY(run_oproj(c, w->wo, l, c.at<void>(c.l.attn), row0, n_rows, c.at<float>(c.l.x),
-                       c.at<void>(c.l.xb), l == s.L - 1 ? h_out : nullptr, blk_start, true));
+                       c.at<void>(c.l.xb), c.at<float>(c.l.sumsq), true));
   }
   return DLLM_OK;
+}
+
+dllm_status run_final_norm(const Ctx& c, const float* x, int row0, int n_rows, int blk_start,
+                           const uint8_t* masked, const void* plants, void* h, bool pdl) {
+  const Shape& s = c.s;
+  FinalNormParams f{};
+  f.batch = s.b;
+  f.B = s.B;
+  f.d = s.d;
+  f.n_rows = n_rows;
+  f.row0 = row0;
+  f.blk_start = blk_start;
+  f.S = s.S;
+  f.P = s.P;
+  f.G = s.G;
+  f.eps = kRmsEps;
+  f.x = x;
+  f.masked = masked;
+  f.plants = static_cast<const __nv_bfloat16*>(plants);
+  f.h = static_cast<__nv_bfloat16*>(h);
+  return cuda_status(launch_final_norm(f, pdl, c.st));
 }
 
 dllm_status run_lmhead(const Ctx& c, const void* w_lm, const void* h, int n_rows, bool pdl) {
@@ -528,11 +555,11 @@ dllm_status check_block(const Shape& s, int blk) {
 dllm_status step(const Ctx& c, const dllm_weights* w, const dllm_state* st, int blk) {
   const Shape& s = c.s;
   if (!st->plants || !aligned16(st->plants)) return DLLM_ERR_INVALID;
-  if (s.mode == DLLM_CACHE_NONE) {
-    DLLM_TRY(run_forward(c, w, st, 0, blk + s.B, 1, blk, blk + s.B, c.at<void>(c.l.h)));
-  } else {
-    DLLM_TRY(run_forward(c, w, st, blk, s.B, 1, blk, 0, c.at<void>(c.l.h)));
-  }
+  const int row0 = s.mode == DLLM_CACHE_NONE ? 0 : blk;
+  const int n_rows = s.mode == DLLM_CACHE_NONE ? blk + s.B : s.B;
+  DLLM_TRY(run_forward(c, w, st, row0, n_rows, blk, s.mode == DLLM_CACHE_NONE ? blk + s.B : 0));
+  DLLM_TRY(run_final_norm(c, c.at<float>(c.l.x), row0, n_rows, blk, st->masked, st->plants,
+                          c.at<void>(c.l.h), true));
   DLLM_TRY(run_lmhead(c, w->w_lm, c.at<void>(c.l.h), s.b * s.B, true));
   return run_commit(c, st, blk, true, nullptr, nullptr, true);
 }
@@ -569,39 +596,52 @@ dllm_status dllm_split_f32_weights(const float* src, void* dst, int64_t rows, in
 }
 
 dllm_status dllm_embed_rows(const dllm_config* cfg, const dllm_weights* w, const dllm_state* st,
-                            int32_t row0, int32_t n_rows, int32_t use_plants,
-                            int32_t block_start, float* x, void* xb, dllm_stream stream) {
+                            int32_t row0, int32_t n_rows, float* x, void* xb, float* row_sumsq,
+                            dllm_stream stream) {
   Shape s;
   DLLM_TRY(check_cfg(cfg, &s));
-  if (!w || !w->embed || !st || !st->tokens || !x || !xb) return DLLM_ERR_INVALID;
-  if (use_plants && (!st->masked || !st->plants)) return DLLM_ERR_INVALID;
+  if (!w || !w->embed || !st || !st->tokens || !st->masked || !x || !xb) return DLLM_ERR_INVALID;
   if (row0 < 0 || n_rows < 1 || row0 + n_rows > s.S) return DLLM_ERR_INVALID;
   EmbedParams e{};
   e.batch = s.b;
   e.S = s.S;
-  e.G = s.G;
-  e.P = s.P;
   e.d = s.d;
   e.n_rows = n_rows;
   e.row0 = row0;
-  e.use_plants = use_plants;
-  e.blk_start = block_start;
-  e.blk_len = s.B;
   e.embed_f32 = s.wfmt == DLLM_W_F32_SPLIT;
+  e.vocab = s.V;
+  e.mask_id = s.mask_id;
+  e.npart = s.d / 128;
+  e.status = nullptr;
   e.tokens = st->tokens;
   e.masked = st->masked;
   e.embed = w->embed;
-  e.plants = static_cast<const __nv_bfloat16*>(st->plants);
   e.x = x;
   e.xb = static_cast<__nv_bfloat16*>(xb);
+  e.sumsq = row_sumsq;
   e.segs = nullptr;
   return cuda_status(launch_embed(e, false, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+dllm_status dllm_final_norm(const dllm_config* cfg, const float* x, int32_t row0, int32_t n_rows,
+                            int32_t block_start, const uint8_t* masked, const void* plants,
+                            void* h, dllm_stream stream) {
+  Shape s;
+  DLLM_TRY(check_cfg(cfg, &s));
+  if (!x || !masked || !plants || !h) return DLLM_ERR_INVALID;
+  DLLM_TRY(check_block(s, block_start));
+  if (row0 < 0 || n_rows < 1 || block_start < row0 || block_start + s.B > row0 + n_rows)
+    return DLLM_ERR_INVALID;
+  Ctx c;
+  c.s = s;
+  c.st = reinterpret_cast<cudaStream_t>(stream);
+  return run_final_norm(c, x, row0, n_rows, block_start, masked, plants, h, false);
+}
+
 dllm_status dllm_qkv_proj(const dllm_config* cfg, const dllm_weights* w, int32_t layer,
-                          const void* xb, int32_t row0, int32_t n_rows, const int32_t* seq_start,
-                          void* q_out, void* k_cache, void* v_cache, void* ws, size_t ws_bytes,
-                          dllm_stream stream) {
+                          const void* xb, const float* row_sumsq, int32_t row0, int32_t n_rows,
+                          const int32_t* seq_start, void* q_out, void* k_cache, void* v_cache,
+                          void* ws, size_t ws_bytes, dllm_stream stream) {
   Ctx c;
   DLLM_TRY(make_ctx(cfg, ws, ws_bytes, stream, &c));
   if (!w || !w->wqkv || !xb || !seq_start || !q_out || !k_cache || !v_cache)
@@ -612,7 +652,8 @@ dllm_status dllm_qkv_proj(const dllm_config* cfg, const dllm_weights* w, int32_t
   if (g.splits > 1 && ((size_t)g.units * g.nt * 128 * 4 > c.l.stats - c.l.slots ||
                        g.m_tiles * g.n_tiles > c.l.gcnt_n))
     return DLLM_ERR_WORKSPACE;
-  return run_qkv(c, w->wqkv, layer, xb, row0, n_rows, seq_start, q_out, k_cache, v_cache, false);
+  return run_qkv(c, w->wqkv, layer, xb, row_sumsq, row0, n_rows, seq_start, q_out, k_cache,
+                 v_cache, false);
 }
 
 dllm_status dllm_block_attn(const dllm_config* cfg, int32_t layer, int32_t n_rows, const void* q,
@@ -628,8 +669,7 @@ dllm_status dllm_block_attn(const dllm_config* cfg, int32_t layer, int32_t n_row
 
 dllm_status dllm_o_proj(const dllm_config* cfg, const dllm_weights* w, int32_t layer,
                         const void* attn, int32_t row0, int32_t n_rows, float* x, void* xb,
-                        void* h_out, int32_t block_start, void* ws, size_t ws_bytes,
-                        dllm_stream stream) {
+                        float* row_sumsq, void* ws, size_t ws_bytes, dllm_stream stream) {
   Ctx c;
   DLLM_TRY(make_ctx(cfg, ws, ws_bytes, stream, &c));
   if (!w || !w->wo || !attn || !x || !xb) return DLLM_ERR_INVALID;
@@ -639,7 +679,7 @@ dllm_status dllm_o_proj(const dllm_config* cfg, const dllm_weights* w, int32_t l
   if (g.splits > 1 && ((size_t)g.units * g.nt * 128 * 4 > c.l.stats - c.l.slots ||
                        g.m_tiles * g.n_tiles > c.l.gcnt_n))
     return DLLM_ERR_WORKSPACE;
-  return run_oproj(c, w->wo, layer, attn, row0, n_rows, x, xb, h_out, block_start, false);
+  return run_oproj(c, w->wo, layer, attn, row0, n_rows, x, xb, row_sumsq, false);
 }
 
 dllm_status dllm_lmhead_confidence(const dllm_config* cfg, const dllm_weights* w, const void* h,
@@ -713,7 +753,7 @@ dllm_status dllm_prefill(const dllm_config* cfg, const dllm_weights* w, const dl
   if (c.s.mode == DLLM_CACHE_NONE) return DLLM_OK;
   const int end = c.s.mode == DLLM_CACHE_PREFIX ? c.s.P : c.s.S;
   if (end < 1) return DLLM_OK;
-  return run_forward(c, w, st, 0, end, 0, -1, end, nullptr);
+  return run_forward(c, w, st, 0, end, -1, end);
 }
 
 dllm_status dllm_decode_step(const dllm_config* cfg, const dllm_weights* w, const dllm_state* st,
@@ -734,7 +774,7 @@ dllm_status dllm_kv_cache_refresh(const dllm_config* cfg, const dllm_weights* w,
   DLLM_TRY(check_state(c.s, w, st));
   DLLM_TRY(check_block(c.s, block_start));
   if (c.s.mode == DLLM_CACHE_NONE) return DLLM_OK;
-  return run_forward(c, w, st, block_start, c.s.B, 0, block_start, 0, nullptr);
+  return run_forward(c, w, st, block_start, c.s.B, block_start, 0);
 }
 
 dllm_status dllm_decode_block(const dllm_config* cfg, const dllm_weights* w, const dllm_state* st,
@@ -763,7 +803,7 @@ dllm_status dllm_decode_block(const dllm_config* cfg, const dllm_weights* w, con
   }
   if (steps_taken) *steps_taken = n;
   if (c.s.mode != DLLM_CACHE_NONE)
-    DLLM_TRY(run_forward(c, w, st, block_start, c.s.B, 0, block_start, 0, nullptr));
+    DLLM_TRY(run_forward(c, w, st, block_start, c.s.B, block_start, 0));
   return DLLM_OK;
 }
 

@@ -68,6 +68,40 @@ __device__ __forceinline__ LmStat lm_shfl_xor(const LmStat& a, int mask) {
   return r;
 }
 
+// Sum over the 128 lanes of each of the chunk's 16 columns staged as
+// stage[col][lane]: 8 threads per column, 16 lanes each, then a shuffle
+// tree.  Returns the column sum in the thread with (et & 7) == 0.
+__device__ __forceinline__ float column_sum16(const float* stage, int et) {
+  const int col = et >> 3, sub = et & 7;
+  const float* cv = stage + col * 128 + sub * 16;
+  float s = 0.f;
+#pragma unroll
+  for (int q = 0; q < 16; ++q) s += cv[q];
+#pragma unroll
+  for (int mask = 1; mask < 8; mask <<= 1) s += __shfl_xor_sync(0xffffffffu, s, mask);
+  return s;
+}
+
+// Per-unit preparation of the final epilogue (QKV: the RMS scale of each
+// activation row, from the partial sums of squares, into inv[NT]).
+template <int NT, int EPI>
+__device__ __forceinline__ void epi_prepare(const GemmParams& p, int n, int et, float* inv) {
+  if constexpr (EPI == EPI_QKV) {
+    for (int c = et; c < NT; c += 128) {
+      const int xrow = n * NT + c;
+      float r = 1.f;
+      if (p.sumsq_in != nullptr && xrow < p.R) {
+        const float* src = p.sumsq_in + (size_t)xrow * p.npart;
+        float s = 0.f;
+        for (int k = 0; k < p.npart; ++k) s += src[k];
+        r = rsqrtf(s / (float)p.d_norm + p.rms_eps);
+      }
+      inv[c] = r;
+    }
+    named_bar_sync(1, 128);
+  }
+}
+
 // Epilogue of one 16-column chunk; v[i] = D^T[m*128 + wl][n*NT + c0 + i].
 template <int NT, int EPI>
 __device__ __forceinline__ void epi_chunk(const GemmParams& p, int m, int n, int c0, int wl,
@@ -78,23 +112,27 @@ __device__ __forceinline__ void epi_chunk(const GemmParams& p, int m, int n, int
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const int xrow = n * NT + c0 + i;
+      float sq = 0.f;
       if (xrow < p.R) {
         const size_t off = (size_t)xrow * p.d_model + wrow;
         const float nx = p.x[off] + v[i];
         p.x[off] = nx;
-        const __nv_bfloat16 nb = __float2bfloat16_rn(nx);
-        p.xb[off] = nb;
-        if (p.h_out != nullptr) {
-          const int b = xrow / p.n_rows;
-          const int pos = p.row0 + (xrow - b * p.n_rows);
-          if (pos >= p.blk_start && pos < p.blk_start + p.blk_len)
-            p.h_out[((size_t)b * p.blk_len + (pos - p.blk_start)) * p.d_model + wrow] = nb;
-        }
+        p.xb[off] = __float2bfloat16_rn(nx);
+        sq = nx * nx;
       }
+      stage[i * 128 + wl] = sq;
+    }
+    if (p.sumsq_out != nullptr) {
+      named_bar_sync(1, 128);
+      const float s = column_sum16(stage, et);
+      const int xrow = n * NT + c0 + (et >> 3);
+      if ((et & 7) == 0 && xrow < p.R) p.sumsq_out[(size_t)xrow * p.npart + m] = s;
+      named_bar_sync(1, 128);
     }
   } else if constexpr (EPI == EPI_QKV) {
+    const float* inv = reinterpret_cast<const float*>(run);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) stage[i * 128 + wl] = v[i];
+    for (int i = 0; i < 16; ++i) stage[i * 128 + wl] = v[i] * inv[c0 + i];
     named_bar_sync(1, 128);
     const int D = p.D, half = D >> 1;
     const int wrow = m * 128 + wl;
@@ -112,7 +150,7 @@ __device__ __forceinline__ void epi_chunk(const GemmParams& p, int m, int n, int
       const int b = xrow / p.n_rows;
       const int ii = xrow - b * p.n_rows;
       const int pos = p.row0 + ii;
-      float val = v[i];
+      float val = stage[i * 128 + wl];
       if (rope) {
         int rp = pos - p.seq_start[b];
         rp = rp < 0 ? 0 : rp;
@@ -313,6 +351,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       tc_fence_after();
       const bool split = p.splits > 1;
+      if (!split) epi_prepare<NT, EPI>(p, n, et, reinterpret_cast<float*>(run));
       for (int c0 = 0; c0 < NT; c0 += 16) {
         float v[16];
         tmem_ld16(tmem + ((uint32_t)lane_base << 16) + acc * NT + c0, v);
@@ -341,6 +380,7 @@ __global__ void __launch_bounds__(192, 1)
         named_bar_sync(1, 128);
         if (last) {
           __threadfence();
+          epi_prepare<NT, EPI>(p, n, et, reinterpret_cast<float*>(run));
           for (int c0 = 0; c0 < NT; c0 += 16) {
             float v[16];
 #pragma unroll

@@ -40,12 +40,15 @@ struct GemmParams {
   __nv_bfloat16* q_out;
   __nv_bfloat16* k_cache;
   __nv_bfloat16* v_cache;
+  // row norms: sumsq[xrow][npart] partial sums of x^2 over 128-column slices
+  const float* sumsq_in;   // QKV: scale each row by 1/sqrt(sum/d_norm + eps)
+  float* sumsq_out;        // O-proj: this tile's slice sum of the new residual
+  int npart, d_norm;
+  float rms_eps;
   // O-proj epilogue
   float* x;
   __nv_bfloat16* xb;
   int d_model;
-  __nv_bfloat16* h_out;
-  int blk_start, blk_len;
   // LM-head epilogue: stats[xrow][slot]
   LmStat* stats;
   int stat_slots;
@@ -79,19 +82,33 @@ cudaError_t launch_attn(int head_dim, const CUtensorMap& qmap, const CUtensorMap
 size_t attn_smem_bytes(int head_dim);
 
 struct EmbedParams {
-  int batch, S, G, P, d, n_rows, row0, use_plants, blk_start, blk_len, embed_f32;
+  int batch, S, d, n_rows, row0, embed_f32, vocab, mask_id, npart, blk_start, blk_len;
+  int* status;
   const int* tokens;
   const uint8_t* masked;
   const void* embed;
-  const __nv_bfloat16* plants;
   float* x;
   __nv_bfloat16* xb;
+  float* sumsq;
   // optional: key segments of the step, written by block 0 thread 0
   int* segs;
   const int* seq_start;
   int mode, window, seg_end;  // seg_end: end of the key range for prefill/none
 };
 cudaError_t launch_embed(const EmbedParams& p, bool pdl, cudaStream_t s);
+
+// LM-head input of the block rows: h = bf16(x / rms(x) + plant where masked).
+struct FinalNormParams {
+  int batch, B, d, n_rows, row0, blk_start, S, P, G;
+  float eps;
+  const float* x;
+  const uint8_t* masked;
+  const __nv_bfloat16* plants;
+  __nv_bfloat16* h;
+};
+cudaError_t launch_final_norm(const FinalNormParams& p, bool pdl, cudaStream_t s);
+
+constexpr float kRmsEps = 1e-6f;
 
 struct CommitParams {
   int batch, S, B, blk_start, stat_slots, vocab;

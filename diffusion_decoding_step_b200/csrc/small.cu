@@ -32,9 +32,24 @@ static cudaError_t launch_simple(K kern, dim3 grid, dim3 block, bool pdl, cudaSt
 }
 
 // ------------------------------------------------------------------ embed
-// One CTA per row.  x0 = plant (masked row of the block) or embed[token].
-// Block 0 also writes the step's key segments.
+// Sum of a value over the CTA (blockDim.x a multiple of 32, <= 1024).
+__device__ __forceinline__ float block_sum(float v, float* red) {
+#pragma unroll
+  for (int mask = 16; mask > 0; mask >>= 1) v += __shfl_xor_sync(0xffffffffu, v, mask);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float t = 0.f;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += red[w];
+  return t;
+}
+
+// One CTA per row: x0 = embed[masked ? mask_id : token], its bf16 copy and
+// the row's sum of squares (partial slot 0; the other slots are zeroed).
+// Block 0 also writes the key segments of the launch sequence.
 __global__ void __launch_bounds__(256) embed_kernel(const EmbedParams p) {
+  __shared__ float red[32];
   grid_dep_wait();
   grid_dep_launch();
   const int row = blockIdx.x;
@@ -64,12 +79,27 @@ __global__ void __launch_bounds__(256) embed_kernel(const EmbedParams p) {
     o[2] = s1;
     o[3] = l1;
   }
-  const bool plant = p.use_plants && p.masked[(size_t)b * p.S + pos] &&
-                     pos >= p.blk_start && pos < p.blk_start + p.blk_len;
+  int tok = p.masked[(size_t)b * p.S + pos] ? p.mask_id : p.tokens[(size_t)b * p.S + pos];
+  if (tok < 0 || tok >= p.vocab) {  // never read outside the embedding table
+    if (threadIdx.x == 0 && p.status) atomicOr(p.status, kErrBadArg);
+    tok = 0;
+  }
   float* xr = p.x + (size_t)row * p.d;
   __nv_bfloat16* xbr = p.xb + (size_t)row * p.d;
-  if (plant) {
-    const __nv_bfloat16* src = p.plants + ((size_t)b * p.G + (pos - p.P)) * p.d;
+  float sq = 0.f;
+  if (p.embed_f32) {
+    const float* src = reinterpret_cast<const float*>(p.embed) + (size_t)tok * p.d;
+    for (int i = threadIdx.x * 4; i < p.d; i += blockDim.x * 4) {
+      const float4 f = *reinterpret_cast<const float4*>(src + i);
+      *reinterpret_cast<float4*>(xr + i) = f;
+      xbr[i] = __float2bfloat16_rn(f.x);
+      xbr[i + 1] = __float2bfloat16_rn(f.y);
+      xbr[i + 2] = __float2bfloat16_rn(f.z);
+      xbr[i + 3] = __float2bfloat16_rn(f.w);
+      sq += f.x * f.x + f.y * f.y + f.z * f.z + f.w * f.w;
+    }
+  } else {
+    const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>(p.embed) + (size_t)tok * p.d;
     for (int i = threadIdx.x * 8; i < p.d; i += blockDim.x * 8) {
       const uint4 raw = *reinterpret_cast<const uint4*>(src + i);
       *reinterpret_cast<uint4*>(xbr + i) = raw;
@@ -79,35 +109,55 @@ __global__ void __launch_bounds__(256) embed_kernel(const EmbedParams p) {
         const float2 f = __bfloat1622float2(h2[k]);
         xr[i + 2 * k] = f.x;
         xr[i + 2 * k + 1] = f.y;
-      }
-    }
-  } else {
-    const int tok = p.tokens[(size_t)b * p.S + pos];
-    if (p.embed_f32) {
-      const float* src = reinterpret_cast<const float*>(p.embed) + (size_t)tok * p.d;
-      for (int i = threadIdx.x * 4; i < p.d; i += blockDim.x * 4) {
-        const float4 f = *reinterpret_cast<const float4*>(src + i);
-        *reinterpret_cast<float4*>(xr + i) = f;
-        xbr[i] = __float2bfloat16_rn(f.x);
-        xbr[i + 1] = __float2bfloat16_rn(f.y);
-        xbr[i + 2] = __float2bfloat16_rn(f.z);
-        xbr[i + 3] = __float2bfloat16_rn(f.w);
-      }
-    } else {
-      const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>(p.embed) + (size_t)tok * p.d;
-      for (int i = threadIdx.x * 8; i < p.d; i += blockDim.x * 8) {
-        const uint4 raw = *reinterpret_cast<const uint4*>(src + i);
-        *reinterpret_cast<uint4*>(xbr + i) = raw;
-        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float2 f = __bfloat1622float2(h2[k]);
-          xr[i + 2 * k] = f.x;
-          xr[i + 2 * k + 1] = f.y;
-        }
+        sq += f.x * f.x + f.y * f.y;
       }
     }
   }
+  const float tot = block_sum(sq, red);
+  if (p.sumsq != nullptr)
+    for (int k = threadIdx.x; k < p.npart; k += blockDim.x)
+      p.sumsq[(size_t)row * p.npart + k] = k == 0 ? tot : 0.f;
+}
+
+// One CTA per block row: h = bf16(x / rms(x) + plant where the row is masked).
+__global__ void __launch_bounds__(256) final_norm_kernel(const FinalNormParams p) {
+  __shared__ float red[32];
+  grid_dep_wait();
+  grid_dep_launch();
+  const int b = blockIdx.x / p.B, i = blockIdx.x - b * p.B;
+  const int pos = p.blk_start + i;
+  const float* xr = p.x + ((size_t)b * p.n_rows + (pos - p.row0)) * p.d;
+  float sq = 0.f;
+  for (int k = threadIdx.x * 4; k < p.d; k += blockDim.x * 4) {
+    const float4 f = *reinterpret_cast<const float4*>(xr + k);
+    sq += f.x * f.x + f.y * f.y + f.z * f.z + f.w * f.w;
+  }
+  const float inv = rsqrtf(block_sum(sq, red) / (float)p.d + p.eps);
+  const bool planted = p.masked[(size_t)b * p.S + pos] != 0;
+  const __nv_bfloat16* pl = p.plants + ((size_t)b * p.G + (pos - p.P)) * p.d;
+  __nv_bfloat16* hr = p.h + ((size_t)b * p.B + i) * p.d;
+  for (int k = threadIdx.x * 4; k < p.d; k += blockDim.x * 4) {
+    const float4 f = *reinterpret_cast<const float4*>(xr + k);
+    float a0 = f.x * inv, a1 = f.y * inv, a2 = f.z * inv, a3 = f.w * inv;
+    if (planted) {
+      const uint2 raw = *reinterpret_cast<const uint2*>(pl + k);
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+      const float2 u = __bfloat1622float2(h2[0]), w = __bfloat1622float2(h2[1]);
+      a0 += u.x;
+      a1 += u.y;
+      a2 += w.x;
+      a3 += w.y;
+    }
+    __nv_bfloat162 o0 = __floats2bfloat162_rn(a0, a1), o1 = __floats2bfloat162_rn(a2, a3);
+    uint2 out;
+    out.x = *reinterpret_cast<uint32_t*>(&o0);
+    out.y = *reinterpret_cast<uint32_t*>(&o1);
+    *reinterpret_cast<uint2*>(hr + k) = out;
+  }
+}
+
+cudaError_t launch_final_norm(const FinalNormParams& p, bool pdl, cudaStream_t s) {
+  return launch_simple(final_norm_kernel, dim3(p.batch * p.B), dim3(256), pdl, s, p);
 }
 
 cudaError_t launch_embed(const EmbedParams& p, bool pdl, cudaStream_t s) {

@@ -12,6 +12,12 @@
  * a window after the block plus the trailing position (Streaming-dLLM README,
  * figure "Illustration of approximated suffix pruning").
  *
+ * The model is a pre-norm transformer with the MLP dropped: per layer
+ * x <- x + Wo . attn(W_qkv . x / rms(x)) with a weightless RMSNorm
+ * (rms(x) = sqrt(mean(x^2) + 1e-6)); the LM head reads x_L / rms(x_L) plus,
+ * for a masked row, its planted hidden state.  A masked row enters layer 0 as
+ * the embedding of mask_id.
+ *
  * Conventions for every entry point
  *  - All tensor pointers are DEVICE pointers owned by the caller unless a
  *    parameter says "host".  The library allocates no device memory; scratch
@@ -106,23 +112,27 @@ dllm_status dllm_workspace_init(const dllm_config* cfg, void* ws, size_t ws_byte
 dllm_status dllm_split_f32_weights(const float* src, void* dst, int64_t rows, int64_t cols,
                                    dllm_stream stream);
 
+/* Per-row sums of squares of the residual are kept as row_sumsq
+ * [rows][hidden/128] fp32: entry j is the sum of x^2 over columns
+ * [128j, 128j+128) (a row's total is the sum of its entries). */
+
 /* Layer-0 input of n_rows rows per sequence starting at position row0:
- * x[b*n_rows+i] = plant of position p = row0+i if use_plants and masked[b][p]
- * and block_start <= p < block_start+B, else embed[tokens[b][p]].
- * x fp32 [b*n_rows][hidden]; xb bf16 copy of it. */
+ * x[b*n_rows+i] = embed[masked[b][p] ? mask_id : tokens[b][p]], p = row0+i.
+ * x fp32 [b*n_rows][hidden]; xb its bf16 copy; row_sumsq (may be NULL) gets
+ * each row's sum of squares in entry 0 and zeros elsewhere. */
 dllm_status dllm_embed_rows(const dllm_config* cfg, const dllm_weights* w,
-                            const dllm_state* st, int32_t row0, int32_t n_rows,
-                            int32_t use_plants, int32_t block_start, float* x, void* xb,
-                            dllm_stream stream);
+                            const dllm_state* st, int32_t row0, int32_t n_rows, float* x,
+                            void* xb, float* row_sumsq, dllm_stream stream);
 
 /* Q/K/V projection of layer `layer` (GEMM on tcgen05, fp32 accumulate) for
- * n_rows rows per sequence at positions row0.. : RoPE at position p-seq_start
- * on q and k, q -> q_out bf16 [b][Hq][n_rows][D], k/v -> caches at p.
+ * n_rows rows per sequence at positions row0..: (W_qkv . xb) / rms(x) with
+ * rms from row_sumsq (NULL = no scaling), RoPE at position p-seq_start on q
+ * and k, q -> q_out bf16 [b][Hq][n_rows][D], k/v -> the caches at p.
  * xb bf16 [b*n_rows][hidden]. */
 dllm_status dllm_qkv_proj(const dllm_config* cfg, const dllm_weights* w, int32_t layer,
-                          const void* xb, int32_t row0, int32_t n_rows,
-                          const int32_t* seq_start, void* q_out, void* k_cache,
-                          void* v_cache, void* ws, size_t ws_bytes, dllm_stream stream);
+                          const void* xb, const float* row_sumsq, int32_t row0, int32_t n_rows,
+                          const int32_t* seq_start, void* q_out, void* k_cache, void* v_cache,
+                          void* ws, size_t ws_bytes, dllm_stream stream);
 
 /* Non-causal GQA attention of n_rows query rows per sequence (q bf16
  * [b][Hq][n_rows][D]) against layer `layer` of the caches.  Query head h reads
@@ -134,13 +144,19 @@ dllm_status dllm_block_attn(const dllm_config* cfg, int32_t layer, int32_t n_row
                             const int32_t* segs, void* out, void* ws, size_t ws_bytes,
                             dllm_stream stream);
 
-/* Output projection and residual: x += attn * Wo^T (fp32), xb = bf16(x).  If
- * h_out is not NULL, rows at positions [block_start, block_start+B) are also
- * copied as bf16 to h_out [b][B][hidden]. */
+/* Output projection and residual: x += attn . Wo^T (fp32), xb = bf16(x),
+ * row_sumsq (may be NULL) = the new residual's per-slice sums of squares. */
 dllm_status dllm_o_proj(const dllm_config* cfg, const dllm_weights* w, int32_t layer,
                         const void* attn, int32_t row0, int32_t n_rows, float* x, void* xb,
-                        void* h_out, int32_t block_start, void* ws, size_t ws_bytes,
-                        dllm_stream stream);
+                        float* row_sumsq, void* ws, size_t ws_bytes, dllm_stream stream);
+
+/* LM-head input of the block at block_start: for every sequence b and block
+ * row i (position p = block_start+i, x row b*n_rows + p-row0):
+ * h[b][i] = bf16(x / rms(x) + (masked[b][p] ? plants[b][p-P] : 0)).
+ * x fp32 [b*n_rows][hidden]; h bf16 [b][B][hidden]. */
+dllm_status dllm_final_norm(const dllm_config* cfg, const float* x, int32_t row0, int32_t n_rows,
+                            int32_t block_start, const uint8_t* masked, const void* plants,
+                            void* h, dllm_stream stream);
 
 /* LM head + confidence over the full vocabulary for n_rows rows of h (bf16
  * [n_rows][hidden]); no logits are written.  conf = max softmax probability,

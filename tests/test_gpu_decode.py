@@ -122,13 +122,18 @@ def test_full_size_first_steps_lockstep(name):
     dec = make_decoder(case)
     dec.prefill()
     torch.cuda.synchronize()
+    assert dec.device_status() == 0
+    bad = [l for l in range(w.n_layers)
+           if not (bool(torch.isfinite(dec.k_cache[l]).all())
+                   and bool(torch.isfinite(dec.v_cache[l]).all()))]
+    assert not bad, f"non-finite cache after prefill in layers {bad[:8]}"
     # layer-0 keys of sampled prompt positions depend only on their embedding
     D, Hq, Hkv = w.head_dim, w.n_q_heads, w.n_kv_heads
     Wk = case.weights.wqkv[0, Hq * D:(Hq + Hkv) * D].double().cpu().numpy()
     for p in (0, 17, w.prompt_len - 1):
         tok = int(case.tokens[0, p])
-        x = O.round_bf16(case.weights.w_lm[tok].double().cpu().numpy())
-        k = (x @ Wk.T).reshape(Hkv, D)
+        e = case.weights.w_lm[tok].double().cpu().numpy()
+        k = ((O.round_bf16(e) @ Wk.T) * O.inv_rms(e)).reshape(Hkv, D)
         if w.rope_theta > 0:
             k = O.rope(k[:, None, :], np.array([p]), w.rope_theta)[:, 0, :]
         got = dec.k_cache[0, 0, :, p].double().cpu().numpy()

@@ -49,6 +49,8 @@ LM_CASES = [  # (rows, hidden, vocab, batch, block)
     (200, 256, 2048, 4, 64),
     (512, 512, 4096, 16, 32),
     (32, 4096, 126464, 1, 32),
+    (512, 512, 65536, 16, 32),      # several tiles per CTA at 256 rows
+    (128, 1024, 32768, 4, 32),      # several tiles per CTA at 128 rows
 ]
 
 
@@ -91,10 +93,13 @@ QKV_CASES = [  # (hidden, Hq, Hkv, D, batch, n_rows, row0, theta, S)
     (4096, 32, 32, 128, 1, 32, 256, 0.0, 512),
     (3584, 28, 4, 128, 1, 32, 512, 1e6, 1024),
     (512, 4, 2, 128, 2, 300, 0, 1e4, 300),
+    (4096, 32, 32, 128, 1, 512, 0, 0.0, 512),   # prefill shape: 256-row tiles, split K
+    (4096, 32, 32, 128, 1, 128, 0, 0.0, 512),   # 128-row tiles, several per CTA
+    (4096, 32, 32, 128, 1, 64, 0, 0.0, 512),
 ]
 
 
-def _qkv_case(d, Hq, Hkv, D, b, nr, row0, theta, S, f32=False, seed=0):
+def _qkv_case(d, Hq, Hkv, D, b, nr, row0, theta, S, f32=False, seed=0, norm=True):
     w = wl.Workload("t", batch=b, n_layers=2, hidden=d, n_q_heads=Hq, n_kv_heads=Hkv,
                     head_dim=D, vocab=1024, prompt_len=S - 32, gen_len=32, block=32,
                     rope_theta=theta, weight_f32=f32)
@@ -102,7 +107,9 @@ def _qkv_case(d, Hq, Hkv, D, b, nr, row0, theta, S, f32=False, seed=0):
     g = _gen(seed + d + nr)
     rows = w.qkv_rows
     Wf = torch.randn(2, rows, d, generator=g, device=DEV) * 0.02
-    x = torch.randn(b * nr, d, generator=g, device=DEV).to(torch.bfloat16)
+    xf = torch.randn(b * nr, d, generator=g, device=DEV) * 3
+    x = xf.to(torch.bfloat16)
+    sumsq = (xf * xf).reshape(b * nr, d // 128, 128).sum(-1).contiguous() if norm else None
     starts = torch.randint(0, 5, (b,), generator=g, device=DEV).to(torch.int32)
     if f32:
         Wk = torch.empty(2, rows, 2 * d, dtype=torch.bfloat16, device=DEV)
@@ -117,11 +124,14 @@ def _qkv_case(d, Hq, Hkv, D, b, nr, row0, theta, S, f32=False, seed=0):
     vc = torch.zeros_like(kc)
     wc = _weights_c(abi, wqkv=Wk, wo=Wk, w_lm=Wk)
     layer = 1
-    abi.check(abi.dllm_qkv_proj(C.byref(cfg), C.byref(wc), layer, ptr(x), row0, nr, ptr(starts),
-                                ptr(q), ptr(kc), ptr(vc), ptr(ws), n, stream()), "qkv")
+    abi.check(abi.dllm_qkv_proj(C.byref(cfg), C.byref(wc), layer, ptr(x), ptr(sumsq), row0, nr,
+                                ptr(starts), ptr(q), ptr(kc), ptr(vc), ptr(ws), n, stream()),
+              "qkv")
     torch.cuda.synchronize()
     X = f64(x).reshape(b, nr, d)
     qkv = X @ Wref[layer].T
+    if norm:
+        qkv = qkv * O.inv_rms(f64(xf).reshape(b, nr, d))[..., None]
     qr = qkv[..., :Hq * D].reshape(b, nr, Hq, D).transpose(0, 2, 1, 3)
     kr = qkv[..., Hq * D:(Hq + Hkv) * D].reshape(b, nr, Hkv, D).transpose(0, 2, 1, 3)
     vr = qkv[..., (Hq + Hkv) * D:].reshape(b, nr, Hkv, D).transpose(0, 2, 1, 3)
@@ -135,21 +145,34 @@ def _qkv_case(d, Hq, Hkv, D, b, nr, row0, theta, S, f32=False, seed=0):
             f64(vc[layer, :, :, row0:row0 + nr]), vr, kc, vc, row0, nr)
 
 
+def _acc_atol(ref):
+    # fp32 accumulation over K terms leaves an absolute error of a few 1e-6 of
+    # the output scale; values that cancel to near zero can round to another
+    # bf16 neighbour for that reason alone
+    return 1e-5 * max(1.0, float(np.sqrt(np.mean(ref * ref))))
+
+
 @pytest.mark.parametrize("case", QKV_CASES)
 def test_qkv_projection_rope_and_cache_write(case):
     q, qr, k, kr, v, vr, kc, vc, row0, nr = _qkv_case(*case)
     for gpu, ref in ((q, qr), (k, kr), (v, vr)):
-        bf16_ulp_close(gpu, O.round_bf16(ref), ulps=1.0, atol=1e-6)
+        bf16_ulp_close(gpu, O.round_bf16(ref), ulps=1.0, atol=_acc_atol(ref))
     # nothing outside the rows was written
     assert float(kc[1, :, :, :row0].abs().sum()) == 0.0
     assert float(vc[1, :, :, row0 + nr:].abs().sum()) == 0.0
     assert float(kc[0].abs().sum()) == 0.0
 
 
+def test_qkv_projection_without_row_scale():
+    q, qr, k, kr, v, vr, *_ = _qkv_case(512, 4, 4, 128, 1, 32, 256, 0.0, 512, norm=False)
+    for gpu, ref in ((q, qr), (k, kr), (v, vr)):
+        bf16_ulp_close(gpu, O.round_bf16(ref), ulps=1.0, atol=_acc_atol(ref))
+
+
 def test_qkv_projection_f32_split_weights():
     q, qr, k, kr, v, vr, *_ = _qkv_case(128, 4, 4, 32, 1, 8, 64, 0.0, 96, f32=True)
     for gpu, ref in ((q, qr), (k, kr), (v, vr)):
-        bf16_ulp_close(gpu, O.round_bf16(ref), ulps=1.0, atol=1e-6)
+        bf16_ulp_close(gpu, O.round_bf16(ref), ulps=1.0, atol=_acc_atol(ref))
 
 
 # ---------------------------------------------------------------- O projection
@@ -159,6 +182,8 @@ OPROJ_CASES = [  # (hidden, Hq, D, batch, n_rows, block_start)
     (3584, 28, 128, 1, 32, 512),
     (512, 4, 128, 2, 96, 32),
     (512, 8, 128, 16, 32, 0),
+    (4096, 32, 128, 1, 512, 0),
+    (4096, 32, 128, 1, 128, 0),
 ]
 
 
@@ -173,21 +198,73 @@ def test_output_projection_residual(d, Hq, D, b, nr, blk):
     x = torch.randn(b * nr, d, generator=g, device=DEV)
     x0 = x.clone()
     xb = torch.zeros(b * nr, d, dtype=torch.bfloat16, device=DEV)
-    h = torch.zeros(b, 32, d, dtype=torch.bfloat16, device=DEV)
+    sumsq = torch.full((b * nr, d // 128), -1.0, device=DEV)
     wc = _weights_c(abi, wqkv=Wo, wo=Wo, w_lm=Wo)
     row0 = blk
     abi.check(abi.dllm_o_proj(C.byref(cfg), C.byref(wc), 1, ptr(attn), row0, nr, ptr(x), ptr(xb),
-                              ptr(h), blk, ptr(ws), n, stream()), "oproj")
+                              ptr(sumsq), ptr(ws), n, stream()), "oproj")
     torch.cuda.synchronize()
     ref = f64(x0) + f64(attn) @ f64(Wo[1]).T
     got = f64(x)
     assert np.abs(got - ref).max() <= 1e-4 * (1 + np.abs(ref).max())
     bf16_ulp_close(f64(xb), O.round_bf16(got), ulps=0.0, atol=0.0)
-    # h_out holds the block rows [blk, blk+32) of each sequence
-    hb = f64(h)
-    for bi in range(b):
-        for i in range(min(32, nr)):
-            np.testing.assert_array_equal(hb[bi, i], f64(xb)[bi * nr + i])
+    want = (got * got).reshape(b * nr, d // 128, 128).sum(-1)
+    np.testing.assert_allclose(f64(sumsq), want, rtol=1e-5)
+
+
+# ---------------------------------------------------------------- embed / final norm
+@pytest.mark.parametrize("f32", [False, True])
+def test_embed_rows_mask_token_and_sumsq(f32):
+    w = wl.WORKLOADS["tiny"].replace(weight_f32=f32, batch=2, hidden=256, n_q_heads=8)
+    abi = ensure_lib()
+    cfg = make_config(w)
+    g = _gen(7)
+    E = torch.randn(w.vocab, w.hidden, generator=g, device=DEV) * 0.5
+    if not f32:
+        E = E.to(torch.bfloat16)
+    S = w.seq_len
+    tokens = torch.randint(0, w.vocab, (w.batch, S), generator=g, device=DEV).to(torch.int32)
+    masked = (torch.rand(w.batch, S, generator=g, device=DEV) < 0.3).to(torch.uint8)
+    row0, nr = 10, 70
+    x = torch.empty(w.batch * nr, w.hidden, device=DEV)
+    xb = torch.empty(w.batch * nr, w.hidden, dtype=torch.bfloat16, device=DEV)
+    sumsq = torch.full((w.batch * nr, w.hidden // 128), -1.0, device=DEV)
+    wc = _weights_c(abi, w_lm=E, embed=E)
+    st = abi.dllm_state(ptr(tokens), ptr(masked), None, None, None, None)
+    abi.check(abi.dllm_embed_rows(C.byref(cfg), C.byref(wc), C.byref(st), row0, nr, ptr(x),
+                                  ptr(xb), ptr(sumsq), stream()), "embed")
+    torch.cuda.synchronize()
+    ids = torch.where(masked[:, row0:row0 + nr].bool(), w.mask_id, tokens[:, row0:row0 + nr])
+    want = f64(E[ids.long()].float()).reshape(w.batch * nr, w.hidden)
+    np.testing.assert_array_equal(f64(x), want)
+    np.testing.assert_array_equal(f64(xb), O.round_bf16(want))
+    ss = f64(sumsq)
+    np.testing.assert_allclose(ss[:, 0], (want * want).sum(1), rtol=1e-5)
+    assert (ss[:, 1:] == 0).all()
+
+
+@pytest.mark.parametrize("mode,b,B", [(wl.MODE_DUAL, 1, 32), (wl.MODE_DUAL, 3, 64),
+                                      (wl.MODE_NONE, 2, 8)])
+def test_final_norm_adds_plants_of_masked_rows(mode, b, B):
+    w = wl.Workload("t", batch=b, n_layers=1, hidden=512, n_q_heads=4, n_kv_heads=4,
+                    head_dim=128, vocab=1024, prompt_len=64, gen_len=2 * B, block=B, mode=mode)
+    abi = ensure_lib()
+    cfg = make_config(w)
+    g = _gen(b * B)
+    blk = w.prompt_len + B
+    row0, nr = (0, blk + B) if mode == wl.MODE_NONE else (blk, B)
+    x = torch.randn(b * nr, w.hidden, generator=g, device=DEV) * 4
+    masked = (torch.rand(b, w.seq_len, generator=g, device=DEV) < 0.5).to(torch.uint8)
+    plants = torch.randn(b, w.gen_len, w.hidden, generator=g, device=DEV).to(torch.bfloat16)
+    h = torch.empty(b, B, w.hidden, dtype=torch.bfloat16, device=DEV)
+    abi.check(abi.dllm_final_norm(C.byref(cfg), ptr(x), row0, nr, blk, ptr(masked), ptr(plants),
+                                  ptr(h), stream()), "final_norm")
+    torch.cuda.synchronize()
+    X = f64(x).reshape(b, nr, w.hidden)[:, blk - row0:blk - row0 + B]
+    m = masked[:, blk:blk + B].cpu().numpy().astype(bool)
+    pl = f64(plants)[:, blk - w.prompt_len:blk - w.prompt_len + B]
+    want = X * O.inv_rms(X)[..., None] + np.where(m[..., None], pl, 0.0)
+    bf16_ulp_close(f64(h), O.round_bf16(want), ulps=1.0, atol=1e-6)
 
 
 # ---------------------------------------------------------------- attention
@@ -200,6 +277,7 @@ ATTN_CASES = [  # (Hq, Hkv, D, batch, n_rows, S, segs per sequence, layer)
     (28, 4, 128, 1, 64, 2300, [[(0, 2200), (2299, 1)]], 0),
     (8, 8, 128, 3, 32, 1280, [[(300, 980), (0, 0)], [(0, 1280), (0, 0)], [(512, 768), (0, 0)]], 1),
     (4, 2, 128, 1, 700, 700, [[(0, 700), (0, 0)]], 0),
+    (32, 32, 128, 1, 512, 512, [[(0, 512), (0, 0)]], 1),   # prefill shape
 ]
 
 
@@ -257,8 +335,9 @@ def test_threshold_commit_bit_exact(b, B, tau):
     t_masked = torch.tensor(masked, device=DEV)
     commit = torch.zeros(b, B, dtype=torch.uint8, device=DEV)
     remaining = torch.zeros(b, dtype=torch.int32, device=DEV)
-    abi.check(abi.dllm_threshold_commit(C.byref(cfg), s, ptr(torch.tensor(conf, device=DEV)),
-                                        ptr(torch.tensor(tok, device=DEV)), ptr(t_tokens),
+    t_conf = torch.tensor(conf, device=DEV)
+    t_tok = torch.tensor(tok, device=DEV)
+    abi.check(abi.dllm_threshold_commit(C.byref(cfg), s, ptr(t_conf), ptr(t_tok), ptr(t_tokens),
                                         ptr(t_masked), ptr(commit), ptr(remaining), stream()),
               "commit")
     torch.cuda.synchronize()
