@@ -70,6 +70,7 @@ SIGNATURES = {
                                     C.POINTER(C.c_void_p)]),
     "dllm_device_status": (C.c_int, [_P, C.POINTER(C.c_int32), _P]),
     "dllm_launch_count": (C.c_uint64, []),
+    "dllm_graph_cache_clear": (None, []),
     "dllm_status_string": (C.c_char_p, [C.c_int]),
 }
 

@@ -5,6 +5,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <mutex>
 #include <vector>
 
 #include "../../include/dllm.h"
@@ -12,6 +13,7 @@
 
 namespace dllm {
 unsigned long long launch_count();
+void add_launches(long long n);
 }
 
 using namespace dllm;
@@ -106,6 +108,9 @@ struct GemmPlan {
   int nt, m_tiles, n_tiles, splits, kbps, units, grid;
 };
 
+// Split K only for decode tiles (NT <= 64): the splits of a tile run as one
+// cluster whose partials meet in rank 0's stage buffers, which hold
+// (splits - 1) partials of 128 x NT fp32.
 GemmPlan plan_gemm(int M, int R, int K, bool allow_split) {
   GemmPlan g;
   g.nt = R <= 32 ? 32 : R <= 64 ? 64 : R <= 128 ? 128 : 256;
@@ -115,7 +120,9 @@ GemmPlan plan_gemm(int M, int R, int K, bool allow_split) {
   const int kbt = K / 64;
   int best_s = 1, best_kbps = kbt;
   double best_cost = 1e30;
-  const int max_s = allow_split ? std::min(32, kbt) : 1;
+  // rank 0's stage region: 3 x (16 KB + NT*128 B) -> 60 KB (NT 32), 72 KB (NT 64)
+  const int cluster_max = g.nt == 32 ? 4 : g.nt == 64 ? 3 : 1;
+  const int max_s = allow_split ? std::min(cluster_max, kbt) : 1;
   for (int s = 1; s <= max_s; ++s) {
     const int kbps = cdiv(kbt, s);
     const int se = cdiv(kbt, kbps);
@@ -132,7 +139,8 @@ GemmPlan plan_gemm(int M, int R, int K, bool allow_split) {
   g.splits = best_s;
   g.kbps = best_kbps;
   g.units = tiles * best_s;
-  g.grid = std::min(g.units, kNumSMs);
+  // split tiles: one unit per CTA (clusters); otherwise persistent CTAs
+  g.grid = best_s > 1 ? g.units : std::min(g.units, kNumSMs);
   return g;
 }
 
@@ -160,26 +168,28 @@ AttnPlan plan_attn(const Shape& s, int n_rows, int ntile_bound) {
   return a;
 }
 
+constexpr int kKeyTile = 128;  // keys per attention tile
+
 // Upper bound of key tiles of a sequence for a block at blk (first valid
 // position 0), or for a plain range [0, seg_end) when seg_end > 0.
 int key_tiles_bound(const Shape& s, int blk, int seg_end) {
-  if (seg_end > 0) return cdiv(seg_end, 128);
+  if (seg_end > 0) return cdiv(seg_end, kKeyTile);
   const int end = blk + s.B;
   switch (s.mode) {
-    case DLLM_CACHE_DUAL: return cdiv(s.S, 128);
+    case DLLM_CACHE_DUAL: return cdiv(s.S, kKeyTile);
     case DLLM_CACHE_DUAL_PRUNED: {
       const int wend = std::min(end + s.W, s.S);
-      return cdiv(wend, 128) + ((end < s.S && s.S - 1 >= wend) ? 1 : 0);
+      return cdiv(wend, kKeyTile) + ((end < s.S && s.S - 1 >= wend) ? 1 : 0);
     }
-    default: return cdiv(end, 128);
+    default: return cdiv(end, kKeyTile);
   }
 }
 
 // ------------------------------------------------------------------ workspace
 struct Layout {
-  size_t status, gcnt, acnt, x, xb, sumsq, q, attn, h, slots, stats, part_o, part_ml, conf, tok,
-      gap, commit, remaining, segs, rope, total;
-  int rmax, lm_slots, gcnt_n, acnt_n;
+  size_t status, acnt, x, xb, sumsq, q, attn, h, stats, part_o, part_ml, conf, tok, gap, commit,
+      remaining, segs, rope, total;
+  int rmax, lm_slots, acnt_n;
 };
 
 // Row counts (per sequence) a configuration uses: decode steps and prefill.
@@ -204,20 +214,9 @@ Layout layout(const Shape& s) {
   };
   const std::vector<int> rows = row_counts(s);
   int max_rows = 0;
-  size_t slot_bytes = 0;
-  int gtiles = 1;
   size_t part_rows = 0;
   int acnt = 1;
-  for (int n : rows) {
-    max_rows = std::max(max_rows, n);
-    const int R = s.b * n;
-    const GemmPlan gq = plan_gemm(s.qkv_rows, R, s.Kw, true);
-    const GemmPlan go = plan_gemm(s.d, R, s.Ko, true);
-    for (const GemmPlan& g : {gq, go}) {
-      if (g.splits > 1) slot_bytes = std::max(slot_bytes, (size_t)g.units * g.nt * 128 * 4);
-      gtiles = std::max(gtiles, g.m_tiles * g.n_tiles);
-    }
-  }
+  for (int n : rows) max_rows = std::max(max_rows, n);
   // attention partials: every decode step, plus the unit-level entry point
   // (block rows against up to ceil(S/128)+1 key tiles)
   auto need_attn = [&](int n_rows, int ntb) {
@@ -232,14 +231,12 @@ Layout layout(const Shape& s) {
     else
       need_attn(s.B, key_tiles_bound(s, blk, 0));
   }
-  need_attn(s.B, cdiv(s.S, 128) + 1);
+  need_attn(s.B, cdiv(s.S, kKeyTile) + 1);
   l.rmax = s.b * max_rows;
   const GemmPlan gl = plan_lmhead(s.V, s.b * s.B, s.Kw);
   l.lm_slots = gl.grid / gl.n_tiles;
-  l.gcnt_n = gtiles;
   l.acnt_n = acnt;
   l.status = take(256);
-  l.gcnt = take((size_t)gtiles * 4);
   l.acnt = take((size_t)acnt * 4);
   l.x = take((size_t)l.rmax * s.d * 4);
   l.xb = take((size_t)l.rmax * s.d * 2);
@@ -247,7 +244,6 @@ Layout layout(const Shape& s) {
   l.q = take((size_t)l.rmax * s.Hq * s.D * 2);
   l.attn = take((size_t)l.rmax * s.Hq * s.D * 2);
   l.h = take((size_t)s.b * s.B * s.d * 2);
-  l.slots = take(std::max<size_t>(slot_bytes, 256));
   l.stats = take((size_t)s.b * s.B * l.lm_slots * sizeof(LmStat));
   l.part_o = take(std::max<size_t>(part_rows * s.D * 4, 256));
   l.part_ml = take(std::max<size_t>(part_rows * 8, 256));
@@ -274,6 +270,21 @@ struct Ctx {
   }
 };
 
+// One-time per-device setup that must not run inside a graph capture:
+// kernel shared-memory attributes and the tensor-map encoder entry point.
+dllm_status prepare_device() {
+  static std::mutex mu;
+  static bool done[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DLLM_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (done[dev]) return DLLM_OK;
+  if (!encode_fn() || gemm_prepare() != cudaSuccess || attn_prepare() != cudaSuccess)
+    return DLLM_ERR_CUDA;
+  done[dev] = true;
+  return DLLM_OK;
+}
+
 dllm_status make_ctx(const dllm_config* cfg, void* ws, size_t ws_bytes, dllm_stream stream,
                      Ctx* c) {
   dllm_status e = check_cfg(cfg, &c->s);
@@ -284,7 +295,7 @@ dllm_status make_ctx(const dllm_config* cfg, void* ws, size_t ws_bytes, dllm_str
   if (reinterpret_cast<uintptr_t>(ws) % 256) return DLLM_ERR_INVALID;
   c->ws = static_cast<uint8_t*>(ws);
   c->st = reinterpret_cast<cudaStream_t>(stream);
-  return DLLM_OK;
+  return prepare_device();
 }
 
 dllm_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DLLM_OK : DLLM_ERR_CUDA; }
@@ -320,8 +331,6 @@ dllm_status run_qkv(const Ctx& c, const void* wqkv, int layer, const void* xb,
   p.units = g.units;
   p.layer = layer;
   p.status = c.at<int>(c.l.status);
-  p.slots = c.at<float>(c.l.slots);
-  p.counters = c.at<int>(c.l.gcnt);
   p.n_rows = n_rows;
   p.row0 = row0;
   p.seq_start = seq_start;
@@ -362,8 +371,6 @@ dllm_status run_oproj(const Ctx& c, const void* wo, int layer, const void* attn,
   p.units = g.units;
   p.layer = layer;
   p.status = c.at<int>(c.l.status);
-  p.slots = c.at<float>(c.l.slots);
-  p.counters = c.at<int>(c.l.gcnt);
   p.n_rows = n_rows;
   p.row0 = row0;
   p.x = x;
@@ -375,8 +382,15 @@ dllm_status run_oproj(const Ctx& c, const void* wo, int layer, const void* attn,
   return cuda_status(launch_gemm(EPI_OPROJ, g.nt, wm, xm, p, g.grid, pdl, c.st));
 }
 
+struct AttnKeys {
+  const int* segs;  // explicit segments, or null to derive them in the kernel
+  const int* seq_start;
+  int blk_start, seg_end, dep_lo, dep_hi;
+};
+
 dllm_status run_attn(const Ctx& c, int layer, int n_rows, const void* q, const void* kc,
-                     const void* vc, const int* segs, void* out, int ntile_bound, bool pdl) {
+                     const void* vc, const AttnKeys& keys, void* out, int ntile_bound,
+                     bool pdl) {
   const Shape& s = c.s;
   const int g = s.Hq / s.Hkv;
   AttnPlan a = plan_attn(s, n_rows, ntile_bound);
@@ -394,8 +408,8 @@ dllm_status run_attn(const Ctx& c, int layer, int n_rows, const void* q, const v
   const CUtensorMapSwizzle sw = s.D >= 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   CUtensorMap qm, km, vm;
   if (!make_map(&qm, q, s.D, (uint64_t)g * n_rows, (uint64_t)s.b * s.Hkv, box_d, 128, sw) ||
-      !make_map(&km, kc, s.D, s.S, (uint64_t)s.L * s.b * s.Hkv, box_d, 128, sw) ||
-      !make_map(&vm, vc, s.D, s.S, (uint64_t)s.L * s.b * s.Hkv, box_d, 128, sw))
+      !make_map(&km, kc, s.D, s.S, (uint64_t)s.L * s.b * s.Hkv, box_d, kKeyTile, sw) ||
+      !make_map(&vm, vc, s.D, s.S, (uint64_t)s.L * s.b * s.Hkv, box_d, kKeyTile, sw))
     return DLLM_ERR_CUDA;
   AttnParams p{};
   p.batch = s.b;
@@ -409,7 +423,15 @@ dllm_status run_attn(const Ctx& c, int layer, int n_rows, const void* q, const v
   p.row_tiles = a.row_tiles;
   p.chunks = a.chunks;
   p.tiles_per_chunk = a.tpc;
-  p.segs = segs;
+  p.segs = keys.segs;
+  p.mode = s.mode;
+  p.blk_start = keys.blk_start;
+  p.blk_len = s.B;
+  p.window = s.W;
+  p.seg_end = keys.seg_end;
+  p.seq_start = keys.seq_start;
+  p.dep_lo = keys.dep_lo;
+  p.dep_hi = keys.dep_hi;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.part_o = c.at<float>(c.l.part_o);
   p.part_ml = c.at<float2>(c.l.part_ml);
@@ -458,8 +480,9 @@ dllm_status run_forward(const Ctx& c, const dllm_weights* w, const dllm_state* s
   for (int l = 0; l < s.L; ++l) {
     DLLM_TRY(run_qkv(c, w->wqkv, l, c.at<void>(c.l.xb), c.at<float>(c.l.sumsq), row0, n_rows,
                      stt->seq_start, c.at<void>(c.l.q), stt->k_cache, stt->v_cache, true));
-    DLLM_TRY(run_attn(c, l, n_rows, c.at<void>(c.l.q), stt->k_cache, stt->v_cache,
-                      c.at<int>(c.l.segs), c.at<void>(c.l.attn), ntb, true));
+    const AttnKeys keys{nullptr, stt->seq_start, blk_start, seg_end, row0, row0 + n_rows};
+    DLLM_TRY(run_attn(c, l, n_rows, c.at<void>(c.l.q), stt->k_cache, stt->v_cache, keys,
+                      c.at<void>(c.l.attn), ntb, true));
     DLLM_TRY(run_oproj(c, w->wo, l, c.at<void>(c.l.attn), row0, n_rows, c.at<float>(c.l.x),
                        c.at<void>(c.l.xb), c.at<float>(c.l.sumsq), true));
   }
@@ -564,6 +587,107 @@ dllm_status step(const Ctx& c, const dllm_weights* w, const dllm_state* st, int 
   return run_commit(c, st, blk, true, nullptr, nullptr, true);
 }
 
+// ------------------------------------------------------------------ graphs
+// The launch sequence of a step, a refresh or a prefill is captured once per
+// (configuration, weight / state / workspace pointers, block) into a CUDA
+// graph and replayed with a single launch afterwards.  Capture runs on a
+// library-owned stream; the graph is launched on the caller's stream.
+struct GraphKey {
+  dllm_config cfg;
+  dllm_weights w;
+  dllm_state st;
+  const void* ws;
+  size_t ws_bytes;
+  int kind, blk, device;
+};
+
+struct GraphEntry {
+  GraphKey key;
+  cudaGraphExec_t exec;
+  long long kernels;
+};
+
+std::mutex g_graph_mu;
+std::vector<GraphEntry> g_graphs;
+constexpr size_t kMaxGraphs = 256;
+
+GraphKey make_key(const dllm_config* cfg, const dllm_weights* w, const dllm_state* st,
+                  const void* ws, size_t ws_bytes, int kind, int blk) {
+  GraphKey k;
+  memset(&k, 0, sizeof(k));
+  k.cfg = *cfg;
+  k.w = *w;
+  k.st = *st;
+  k.ws = ws;
+  k.ws_bytes = ws_bytes;
+  k.kind = kind;
+  k.blk = blk;
+  cudaGetDevice(&k.device);
+  return k;
+}
+
+cudaStream_t capture_stream(int device) {
+  static cudaStream_t streams[64] = {};
+  if (device < 0 || device >= 64) return nullptr;
+  if (!streams[device]) cudaStreamCreateWithFlags(&streams[device], cudaStreamNonBlocking);
+  return streams[device];
+}
+
+template <class F>
+dllm_status run_graph(const Ctx& c, const GraphKey& key, F&& body) {
+  std::lock_guard<std::mutex> lock(g_graph_mu);
+  for (const GraphEntry& e : g_graphs) {
+    if (memcmp(&e.key, &key, sizeof(GraphKey)) == 0) {
+      add_launches(e.kernels);
+      return cuda_status(cudaGraphLaunch(e.exec, c.st));
+    }
+  }
+  cudaStream_t cs = capture_stream(key.device);
+  if (!cs) return DLLM_ERR_CUDA;
+  Ctx cc = c;
+  cc.st = cs;
+  const unsigned long long n0 = launch_count();
+  if (cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal) != cudaSuccess)
+    return DLLM_ERR_CUDA;
+  const dllm_status e = body(cc);
+  cudaGraph_t g = nullptr;
+  const cudaError_t ce = cudaStreamEndCapture(cs, &g);
+  const long long kernels = (long long)(launch_count() - n0);
+  add_launches(-kernels);  // captured, not executed
+  if (e != DLLM_OK || ce != cudaSuccess || !g) {
+    if (g) cudaGraphDestroy(g);
+    return e != DLLM_OK ? e : DLLM_ERR_CUDA;
+  }
+  cudaGraphExec_t exec = nullptr;
+  const cudaError_t ie = cudaGraphInstantiate(&exec, g, 0);
+  cudaGraphDestroy(g);
+  if (ie != cudaSuccess) return DLLM_ERR_CUDA;
+  if (g_graphs.size() >= kMaxGraphs) {
+    cudaGraphExecDestroy(g_graphs.front().exec);
+    g_graphs.erase(g_graphs.begin());
+  }
+  g_graphs.push_back({key, exec, kernels});
+  add_launches(kernels);
+  return cuda_status(cudaGraphLaunch(exec, c.st));
+}
+
+enum GraphKind { kGraphStep = 1, kGraphRefresh = 2, kGraphPrefill = 3 };
+
+dllm_status step_graph(const Ctx& c, const dllm_config* cfg, const dllm_weights* w,
+                       const dllm_state* st, void* ws, size_t ws_bytes, int blk) {
+  const GraphKey key = make_key(cfg, w, st, ws, ws_bytes, kGraphStep, blk);
+  return run_graph(c, key, [&](const Ctx& cc) { return step(cc, w, st, blk); });
+}
+
+dllm_status refresh_graph(const Ctx& c, const dllm_config* cfg, const dllm_weights* w,
+                          const dllm_state* st, void* ws, size_t ws_bytes, int blk) {
+  if (c.s.mode == DLLM_CACHE_NONE) return DLLM_OK;
+  const GraphKey key = make_key(cfg, w, st, ws, ws_bytes, kGraphRefresh, blk);
+  return run_graph(c, key, [&](const Ctx& cc) {
+    return run_forward(cc, w, st, blk, cc.s.B, blk, 0);
+  });
+}
+
 }  // namespace
 
 // ====================================================================== C ABI
@@ -648,10 +772,6 @@ dllm_status dllm_qkv_proj(const dllm_config* cfg, const dllm_weights* w, int32_t
     return DLLM_ERR_INVALID;
   if (layer < 0 || layer >= c.s.L || row0 < 0 || n_rows < 1 || row0 + n_rows > c.s.S)
     return DLLM_ERR_INVALID;
-  const GemmPlan g = plan_gemm(c.s.qkv_rows, c.s.b * n_rows, c.s.Kw, true);
-  if (g.splits > 1 && ((size_t)g.units * g.nt * 128 * 4 > c.l.stats - c.l.slots ||
-                       g.m_tiles * g.n_tiles > c.l.gcnt_n))
-    return DLLM_ERR_WORKSPACE;
   return run_qkv(c, w->wqkv, layer, xb, row_sumsq, row0, n_rows, seq_start, q_out, k_cache,
                  v_cache, false);
 }
@@ -663,8 +783,9 @@ dllm_status dllm_block_attn(const dllm_config* cfg, int32_t layer, int32_t n_row
   DLLM_TRY(make_ctx(cfg, ws, ws_bytes, stream, &c));
   if (!q || !k_cache || !v_cache || !segs || !out) return DLLM_ERR_INVALID;
   if (layer < 0 || layer >= c.s.L || n_rows < 1 || n_rows > c.s.S) return DLLM_ERR_INVALID;
-  const int ntb = cdiv(c.s.S, 128) + 1;
-  return run_attn(c, layer, n_rows, q, k_cache, v_cache, segs, out, ntb, false);
+  const int ntb = cdiv(c.s.S, kKeyTile) + 1;
+  const AttnKeys keys{segs, nullptr, 0, 0, 0, c.s.S};
+  return run_attn(c, layer, n_rows, q, k_cache, v_cache, keys, out, ntb, false);
 }
 
 dllm_status dllm_o_proj(const dllm_config* cfg, const dllm_weights* w, int32_t layer,
@@ -675,10 +796,6 @@ dllm_status dllm_o_proj(const dllm_config* cfg, const dllm_weights* w, int32_t l
   if (!w || !w->wo || !attn || !x || !xb) return DLLM_ERR_INVALID;
   if (layer < 0 || layer >= c.s.L || row0 < 0 || n_rows < 1 || row0 + n_rows > c.s.S)
     return DLLM_ERR_INVALID;
-  const GemmPlan g = plan_gemm(c.s.d, c.s.b * n_rows, c.s.Ko, true);
-  if (g.splits > 1 && ((size_t)g.units * g.nt * 128 * 4 > c.l.stats - c.l.slots ||
-                       g.m_tiles * g.n_tiles > c.l.gcnt_n))
-    return DLLM_ERR_WORKSPACE;
   return run_oproj(c, w->wo, layer, attn, row0, n_rows, x, xb, row_sumsq, false);
 }
 
@@ -753,7 +870,8 @@ dllm_status dllm_prefill(const dllm_config* cfg, const dllm_weights* w, const dl
   if (c.s.mode == DLLM_CACHE_NONE) return DLLM_OK;
   const int end = c.s.mode == DLLM_CACHE_PREFIX ? c.s.P : c.s.S;
   if (end < 1) return DLLM_OK;
-  return run_forward(c, w, st, 0, end, -1, end);
+  const GraphKey key = make_key(cfg, w, st, ws, ws_bytes, kGraphPrefill, 0);
+  return run_graph(c, key, [&](const Ctx& cc) { return run_forward(cc, w, st, 0, end, -1, end); });
 }
 
 dllm_status dllm_decode_step(const dllm_config* cfg, const dllm_weights* w, const dllm_state* st,
@@ -763,7 +881,8 @@ dllm_status dllm_decode_step(const dllm_config* cfg, const dllm_weights* w, cons
   DLLM_TRY(make_ctx(cfg, ws, ws_bytes, stream, &c));
   DLLM_TRY(check_state(c.s, w, st));
   DLLM_TRY(check_block(c.s, block_start));
-  return step(c, w, st, block_start);
+  if (!st->plants || !aligned16(st->plants)) return DLLM_ERR_INVALID;
+  return step_graph(c, cfg, w, st, ws, ws_bytes, block_start);
 }
 
 dllm_status dllm_kv_cache_refresh(const dllm_config* cfg, const dllm_weights* w,
@@ -773,8 +892,7 @@ dllm_status dllm_kv_cache_refresh(const dllm_config* cfg, const dllm_weights* w,
   DLLM_TRY(make_ctx(cfg, ws, ws_bytes, stream, &c));
   DLLM_TRY(check_state(c.s, w, st));
   DLLM_TRY(check_block(c.s, block_start));
-  if (c.s.mode == DLLM_CACHE_NONE) return DLLM_OK;
-  return run_forward(c, w, st, block_start, c.s.B, block_start, 0);
+  return refresh_graph(c, cfg, w, st, ws, ws_bytes, block_start);
 }
 
 dllm_status dllm_decode_block(const dllm_config* cfg, const dllm_weights* w, const dllm_state* st,
@@ -785,10 +903,11 @@ dllm_status dllm_decode_block(const dllm_config* cfg, const dllm_weights* w, con
   DLLM_TRY(check_state(c.s, w, st));
   DLLM_TRY(check_block(c.s, block_start));
   if (max_steps < 1) max_steps = c.s.B;
+  if (!st->plants || !aligned16(st->plants)) return DLLM_ERR_INVALID;
   std::vector<int> rem(c.s.b + 1);
   int n = 0;
   for (; n < max_steps;) {
-    DLLM_TRY(step(c, w, st, block_start));
+    DLLM_TRY(step_graph(c, cfg, w, st, ws, ws_bytes, block_start));
     ++n;
     if (cudaMemcpyAsync(rem.data(), c.at<int>(c.l.remaining), sizeof(int) * c.s.b,
                         cudaMemcpyDeviceToHost, c.st) != cudaSuccess ||
@@ -802,9 +921,13 @@ dllm_status dllm_decode_block(const dllm_config* cfg, const dllm_weights* w, con
     if (left == 0) break;
   }
   if (steps_taken) *steps_taken = n;
-  if (c.s.mode != DLLM_CACHE_NONE)
-    DLLM_TRY(run_forward(c, w, st, block_start, c.s.B, block_start, 0));
-  return DLLM_OK;
+  return refresh_graph(c, cfg, w, st, ws, ws_bytes, block_start);
+}
+
+void dllm_graph_cache_clear(void) {
+  std::lock_guard<std::mutex> lock(g_graph_mu);
+  for (GraphEntry& e : g_graphs) cudaGraphExecDestroy(e.exec);
+  g_graphs.clear();
 }
 
 dllm_status dllm_step_outputs(const dllm_config* cfg, void* ws, size_t ws_bytes, float** conf,

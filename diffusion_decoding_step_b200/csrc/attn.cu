@@ -5,17 +5,22 @@
 // g = Hq/Hkv heads x n_rows block rows, contiguous in the q buffer
 // [b][Hq][n_rows][D], so a row tile is one TMA box (rows past the group are
 // zero-filled).  Key/value tiles of 128 positions stream from the bf16 cache
-// [L][b][Hkv][S][D] through a 2-stage TMA ring.  Per key tile:
-//   S = Q K^T           UMMA M=128 (rows) N=128 (keys) into TMEM columns [0,128)
-//   softmax             thread t owns query row t (TMEM lane t): running max
-//                       and sum in registers, exp2 in the log2 domain, P in bf16
-//                       written to shared memory in the UMMA K-major layout
-//   O_tile = P V        UMMA M=128 N=D, V read MN-major straight from the TMA
-//                       tile; O accumulates in registers with the usual
-//                       rescaling by exp2(m_old - m_new)
-// Keys outside the sequence's segments are masked inside the tile.  When a
-// (row tile) is split over several key chunks, each chunk writes an
-// unnormalised partial (O, max, sum) and the last chunk to finish merges them.
+// [L][b][Hkv][S][D] through a TMA ring of ST stages.  Per key tile:
+//   S = Q K^T      UMMA M=128 (rows) x N=128 (keys) into TMEM columns [0,128)
+//   softmax        thread t owns query row t (TMEM lane t): the row is read
+//                  from TMEM once, max and sum run in registers in the log2
+//                  domain, P goes to shared memory in bf16 in the UMMA
+//                  K-major layout
+//   O += P V       UMMA M=128 x N=D into TMEM columns [128,128+D); V is read
+//                  MN-major straight from its TMA tile.  O stays in TMEM; a
+//                  row is rescaled there only when its running max grows.
+// Key tiles that the preceding kernel does not write (everything outside
+// [dep_lo, dep_hi)) are requested before the programmatic-dependency wait,
+// so for a decode step the prefix/suffix cache is already in flight while the
+// Q/K/V projection finishes.  Keys outside the sequence's segments are
+// masked inside the tile.  When a row tile is split over several key
+// chunks, each chunk writes an unnormalised partial (O, max, sum) and the
+// last chunk to finish merges them in chunk order.
 #include <float.h>
 
 #include "kernels.cuh"
@@ -23,51 +28,114 @@
 
 namespace dllm {
 
-template <int D>
+constexpr int kKeys = 128;  // keys per tile
+
+template <int D, int ST>
 struct AttnCfg {
   static constexpr int kBoxD = D >= 64 ? 64 : D;      // elements per swizzled row
   static constexpr int kRowBytes = kBoxD * 2;         // 128 or 64
   static constexpr int kSwCode = kRowBytes == 128 ? 2 : 4;
   static constexpr int kNBox = D / kBoxD;
-  static constexpr int kBoxBytes = 128 * kRowBytes;   // one box of 128 rows
-  static constexpr int kTileBytes = 128 * D * 2;      // Q, K or V tile of 128 rows
-  static constexpr int kPBytes = 128 * 128 * 2;
-  static constexpr int kStages = 2;
-  static constexpr int kTmemCols = 256;
-  static constexpr size_t kSmem =
-      1024 + kTileBytes /*Q*/ + kStages * 2 * kTileBytes /*K,V*/ + kPBytes + 16 * 8 + 64;
+  static constexpr int kBoxBytes = 128 * kRowBytes;   // one box of 128 rows (Q or keys)
+  static constexpr int kQBytes = 128 * D * 2;
+  static constexpr int kKVBytes = kKeys * D * 2;      // K or V tile
+  static constexpr int kPBytes = 128 * kKeys * 2;     // two 128B-swizzle atom columns
+  static constexpr int kTmemCols = 256;               // S [0,128), O [128,128+D)
+  static constexpr size_t kSmem = 1024 + kQBytes + ST * 2 * kKVBytes + kPBytes + 128 + 64;
 };
 
+// Key segments (start, len) x 2 of sequence b: given explicitly, or derived
+// from the cache mode, the block and the sequence start.
+__device__ __forceinline__ void seq_segments(const AttnParams& p, int b, int* sg) {
+  if (p.segs != nullptr) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) sg[i] = p.segs[b * 4 + i];
+    return;
+  }
+  const int st = p.seq_start[b];
+  const int end = p.blk_start + p.blk_len;
+  int l0, s1 = 0, l1 = 0;
+  if (p.seg_end > 0) {
+    l0 = p.seg_end - st;
+  } else if (p.mode == 2) {  // DUAL
+    l0 = p.S - st;
+  } else if (p.mode == 3) {  // DUAL_PRUNED
+    const int wend = min(end + p.window, p.S);
+    l0 = wend - st;
+    if (end < p.S && p.S - 1 >= wend) {
+      s1 = p.S - 1;
+      l1 = 1;
+    }
+  } else {  // NONE, PREFIX
+    l0 = end - st;
+  }
+  sg[0] = st;
+  sg[1] = l0 > 0 ? l0 : 0;
+  sg[2] = s1;
+  sg[3] = l1;
+}
+
 __device__ __forceinline__ void tile_of(const int* sg, int t, int& start, int& nvalid) {
-  const int n0 = (sg[1] + 127) >> 7;
+  const int n0 = (sg[1] + kKeys - 1) / kKeys;
   if (t < n0) {
-    start = sg[0] + t * 128;
-    nvalid = min(128, sg[1] - t * 128);
+    start = sg[0] + t * kKeys;
+    nvalid = min(kKeys, sg[1] - t * kKeys);
   } else {
     const int tt = t - n0;
-    start = sg[2] + tt * 128;
-    nvalid = min(128, sg[3] - tt * 128);
+    start = sg[2] + tt * kKeys;
+    nvalid = min(kKeys, sg[3] - tt * kKeys);
   }
 }
 
-template <int D>
+DLLM_DEV void tmem_ld32(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32"
+      " {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+        "=r"(r[31])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+DLLM_DEV void tmem_st16(uint32_t taddr, const float (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0],"
+      " {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15]))
+      : "memory");
+}
+DLLM_DEV void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+template <int D, int ST>
 __global__ void __launch_bounds__(128, 1)
     attn_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                 const __grid_constant__ CUtensorMap vmap, const AttnParams p) {
-  using C = AttnCfg<D>;
+  using C = AttnCfg<D, ST>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* q_s = base;
-  uint8_t* k_s = q_s + C::kTileBytes;                    // [stage]
-  uint8_t* v_s = k_s + C::kStages * C::kTileBytes;       // [stage]
-  uint8_t* p_s = v_s + C::kStages * C::kTileBytes;
+  uint8_t* k_s = q_s + C::kQBytes;                 // [ST]
+  uint8_t* v_s = k_s + ST * C::kKVBytes;           // [ST]
+  uint8_t* p_s = v_s + ST * C::kKVBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(p_s + C::kPBytes);
   uint64_t* bar_q = bars;
-  uint64_t* bar_kv = bars + 1;  // [2]
-  uint64_t* bar_s = bars + 3;
-  uint64_t* bar_o = bars + 4;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 6);
+  uint64_t* bar_s = bars + 1;
+  uint64_t* bar_o = bars + 2;
+  uint64_t* bar_kv = bars + 3;  // [ST]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 + ST);
   volatile int* flags = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
   const int t = threadIdx.x;
@@ -79,13 +147,14 @@ __global__ void __launch_bounds__(128, 1)
   idx /= p.row_tiles;
   const int kvh = idx % p.Hkv;
   const int b = idx / p.Hkv;
+  const int zc = (p.layer * p.batch + b) * p.Hkv + kvh;  // cache plane
+  const int zq = b * p.Hkv + kvh;                         // q plane
 
   if (t == 0) {
     mbar_init(bar_q, 1);
-    mbar_init(&bar_kv[0], 1);
-    mbar_init(&bar_kv[1], 1);
     mbar_init(bar_s, 1);
     mbar_init(bar_o, 1);
+    for (int s = 0; s < ST; ++s) mbar_init(&bar_kv[s], 1);
     flags[0] = 0;
     flags[1] = 0;
     fence_barrier_init();
@@ -95,7 +164,48 @@ __global__ void __launch_bounds__(128, 1)
   }
   __syncthreads();
   grid_dep_launch();
+
+  // Segments come from the sequence start (an input of the step) unless an
+  // explicit list is given, which may be produced by earlier kernels.
+  int sg[4] = {0, 0, 0, 0};
+  if (p.segs == nullptr) seq_segments(p, b, sg);
+
+  auto issue_kv = [&](int j, int start) {  // key tile t0 + j into stage j % ST
+    const int st = j % ST;
+    mbar_arrive_expect_tx(&bar_kv[st], 2 * C::kKVBytes);
+#pragma unroll
+    for (int bx = 0; bx < C::kNBox; ++bx) {
+      tma_load_3d(k_s + st * C::kKVBytes + bx * C::kBoxBytes, &kmap, &bar_kv[st],
+                  bx * C::kBoxD, start, zc);
+      tma_load_3d(v_s + st * C::kKVBytes + bx * C::kBoxBytes, &vmap, &bar_kv[st],
+                  bx * C::kBoxD, start, zc);
+    }
+  };
+  auto chunk_range = [&](int& first, int& n) {
+    const int n_tiles = (sg[1] + kKeys - 1) / kKeys + (sg[3] + kKeys - 1) / kKeys;
+    first = chunk * p.tiles_per_chunk;
+    const int last = min(n_tiles, first + p.tiles_per_chunk);
+    n = last > first ? last - first : 0;
+  };
+
+  unsigned pre = 0;  // stages requested before the dependency wait
+  if (t == 0 && p.segs == nullptr) {
+    int first, n;
+    chunk_range(first, n);
+    for (int j = 0; j < min(n, ST); ++j) {
+      int start, nv;
+      tile_of(sg, first + j, start, nv);
+      if (start + kKeys <= p.dep_lo || start >= p.dep_hi) {
+        issue_kv(j, start);
+        pre |= 1u << j;
+      }
+    }
+  }
   grid_dep_wait();
+  if (p.segs != nullptr) seq_segments(p, b, sg);
+  int t0, my_tiles;
+  chunk_range(t0, my_tiles);
+
   if (warp == 0) tmem_alloc(tmem_slot, C::kTmemCols);
   tc_fence_before();
   __syncthreads();
@@ -103,59 +213,38 @@ __global__ void __launch_bounds__(128, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t s_tmem = tmem;
   const uint32_t o_tmem = tmem + 128;
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
 
-  const int* sg = p.segs + b * 4;
-  const int n_tiles = ((sg[1] + 127) >> 7) + ((sg[3] + 127) >> 7);
-  const int t0 = chunk * p.tiles_per_chunk;
-  const int t1 = min(n_tiles, t0 + p.tiles_per_chunk);
-  const int my_tiles = t1 > t0 ? t1 - t0 : 0;
-  const int zc = (p.layer * p.batch + b) * p.Hkv + kvh;   // cache plane
-  const int zq = b * p.Hkv + kvh;                          // q plane
-
-  constexpr uint32_t kIdescS = idesc_bf16(128, 128, 0, 0);
+  constexpr uint32_t kIdescS = idesc_bf16(128, kKeys, 0, 0);
   constexpr uint32_t kIdescO = idesc_bf16(128, D, 0, 1);
 
-  auto issue_kv = [&](int j) {  // load key tile t0 + j into stage j & 1
-    int start, nv;
-    tile_of(sg, t0 + j, start, nv);
-    const int st = j & 1;
-    mbar_arrive_expect_tx(&bar_kv[st], 2 * C::kTileBytes);
-#pragma unroll
-    for (int bx = 0; bx < C::kNBox; ++bx) {
-      tma_load_3d(k_s + st * C::kTileBytes + bx * C::kBoxBytes, &kmap, &bar_kv[st],
-                  bx * C::kBoxD, start, zc);
-      tma_load_3d(v_s + st * C::kTileBytes + bx * C::kBoxBytes, &vmap, &bar_kv[st],
-                  bx * C::kBoxD, start, zc);
-    }
-  };
-
   if (t == 0 && my_tiles > 0) {
-    mbar_arrive_expect_tx(bar_q, C::kTileBytes);
+    mbar_arrive_expect_tx(bar_q, C::kQBytes);
 #pragma unroll
     for (int bx = 0; bx < C::kNBox; ++bx)
       tma_load_3d(q_s + bx * C::kBoxBytes, &qmap, bar_q, bx * C::kBoxD, rt * 128, zq);
-    issue_kv(0);
-    if (my_tiles > 1) issue_kv(1);
+    for (int j = 0; j < min(my_tiles, ST); ++j) {
+      if (pre & (1u << j)) continue;
+      int start, nv;
+      tile_of(sg, t0 + j, start, nv);
+      issue_kv(j, start);
+    }
   }
 
-  float o[D];
-#pragma unroll
-  for (int i = 0; i < D; ++i) o[i] = 0.f;
   float m_run = -FLT_MAX, l_run = 0.f;
   bool ok = true;
-
-  for (int j = 0; j < my_tiles && ok; ++j) {
-    const int st = j & 1;
+  for (int j = 0; j < my_tiles; ++j) {
+    const int st = j % ST;
     int kstart, nvalid;
     tile_of(sg, t0 + j, kstart, nvalid);
     // ---- S = Q K^T
     if (t == 0) {
-      bool good = (j > 0 || mbar_wait(bar_q, 0, p.status)) &&
-                  mbar_wait(&bar_kv[st], (j >> 1) & 1, p.status);
+      const bool good = (j > 0 || mbar_wait(bar_q, 0, p.status)) &&
+                        mbar_wait(&bar_kv[st], (j / ST) & 1, p.status);
       if (good) {
         tc_fence_after();
         const uint32_t qa = smem_u32(q_s);
-        const uint32_t ka = smem_u32(k_s + st * C::kTileBytes);
+        const uint32_t ka = smem_u32(k_s + st * C::kKVBytes);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk * 16 / C::kBoxD) * C::kBoxBytes + ((kk * 16) % C::kBoxD) * 2;
@@ -174,83 +263,85 @@ __global__ void __launch_bounds__(128, 1)
       break;
     }
     tc_fence_after();
-    // ---- softmax over the tile (log2 domain)
-    const uint32_t lane_addr = s_tmem + ((uint32_t)(warp * 32) << 16);
+    // ---- softmax of row t over the tile (log2 domain), one TMEM read
+    float s[kKeys];
+#pragma unroll
+    for (int c = 0; c < kKeys / 32; ++c) tmem_ld32(s_tmem + lane_off + c * 32, s + c * 32);
+    tmem_ld_wait();
     float tmax = -FLT_MAX;
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      float v[16];
-      tmem_ld16(lane_addr + c * 16, v);
-      tmem_ld_wait();
-#pragma unroll
-      for (int i = 0; i < 16; ++i)
-        if (c * 16 + i < nvalid) tmax = fmaxf(tmax, v[i]);
-    }
+    for (int i = 0; i < kKeys; ++i)
+      if (i < nvalid) tmax = fmaxf(tmax, s[i]);
     const float m_new = fmaxf(m_run, tmax * p.scale_log2);
     const float alpha = exp2f(m_run - m_new);
     float lsum = 0.f;
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      float v[16];
-      tmem_ld16(lane_addr + c * 16, v);
-      tmem_ld_wait();
-      uint32_t pk[8];
+    for (int c = 0; c < kKeys / 8; ++c) {  // 8 keys = one 16-byte chunk of P
+      uint32_t pk[4];
 #pragma unroll
-      for (int i = 0; i < 16; i += 2) {
-        const float p0 = (c * 16 + i < nvalid) ? exp2f(v[i] * p.scale_log2 - m_new) : 0.f;
-        const float p1 = (c * 16 + i + 1 < nvalid) ? exp2f(v[i + 1] * p.scale_log2 - m_new) : 0.f;
+      for (int i = 0; i < 8; i += 2) {
+        const int k0 = c * 8 + i;
+        const float p0 = k0 < nvalid ? exp2f(s[k0] * p.scale_log2 - m_new) : 0.f;
+        const float p1 = k0 + 1 < nvalid ? exp2f(s[k0 + 1] * p.scale_log2 - m_new) : 0.f;
         const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
         lsum += __low2float(h2) + __high2float(h2);
         pk[i >> 1] = *reinterpret_cast<const uint32_t*>(&h2);
       }
-      // keys c*16 .. c*16+15: half (c / 4), 16-byte chunks 2*(c%4) and 2*(c%4)+1
-      uint8_t* prow = p_s + (c >> 2) * (128 * 128) + t * 128;
-      const int ch0 = 2 * (c & 3);
-      *reinterpret_cast<uint4*>(prow + (((ch0) ^ (t & 7)) << 4)) =
+      // keys 64h..64h+63 form atom column h; row t holds 8 chunks of 16 bytes
+      uint8_t* prow = p_s + (c >> 3) * (128 * 128) + t * 128;
+      *reinterpret_cast<uint4*>(prow + (((c & 7) ^ (t & 7)) << 4)) =
           make_uint4(pk[0], pk[1], pk[2], pk[3]);
-      *reinterpret_cast<uint4*>(prow + (((ch0 + 1) ^ (t & 7)) << 4)) =
-          make_uint4(pk[4], pk[5], pk[6], pk[7]);
+    }
+    // O (from earlier tiles) is rescaled in TMEM when the running max grew;
+    // the previous P V finished before this tile's S was committed.
+    if (j > 0 && __any_sync(0xffffffffu, alpha < 1.f)) {
+#pragma unroll
+      for (int c = 0; c < D / 16; ++c) {
+        float v[16];
+        tmem_ld16(o_tmem + lane_off + c * 16, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] *= alpha;
+        tmem_st16(o_tmem + lane_off + c * 16, v);
+      }
+      tmem_st_wait();
     }
     l_run = l_run * alpha + lsum;
     m_run = m_new;
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
-    // ---- O_tile = P V
+    // ---- O += P V
     if (t == 0) {
       tc_fence_after();
       const uint32_t pa = smem_u32(p_s);
-      const uint32_t va = smem_u32(v_s + st * C::kTileBytes);
+      const uint32_t va = smem_u32(v_s + st * C::kKVBytes);
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
+      for (int kk = 0; kk < kKeys / 16; ++kk) {
         const uint32_t aoff = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
         const uint32_t boff = kk * 16 * C::kRowBytes;
         umma_bf16(o_tmem, smem_desc(pa + aoff, 16, 1024, 2),
                   smem_desc(va + boff, C::kBoxBytes, 8 * C::kRowBytes, C::kSwCode), kIdescO,
-                  kk > 0 ? 1u : 0u);
+                  (j > 0 || kk > 0) ? 1u : 0u);
       }
       umma_commit(bar_o);
+      if (j + ST < my_tiles) {
+        // stage st is free once this P V has read V; the next S reads the other stage
+        if (mbar_wait(bar_o, j & 1, p.status)) {
+          int start, nv;
+          tile_of(sg, t0 + j + ST, start, nv);
+          issue_kv(j + ST, start);
+        } else {
+          flags[0] = 1;
+        }
+      }
     }
-    const bool bad_o = !mbar_wait(bar_o, j & 1, p.status);
-    if (__syncthreads_or(bad_o)) {
-      ok = false;
-      break;
-    }
-    tc_fence_after();
-    // stage st is free again: prefetch tile j + 2 into it
-    if (t == 0 && j + 2 < my_tiles) issue_kv(j + 2);
-    const uint32_t o_addr = o_tmem + ((uint32_t)(warp * 32) << 16);
-#pragma unroll
-    for (int c = 0; c < D / 16; ++c) {
-      float v[16];
-      tmem_ld16(o_addr + c * 16, v);
-      tmem_ld_wait();
-#pragma unroll
-      for (int i = 0; i < 16; ++i) o[c * 16 + i] = o[c * 16 + i] * alpha + v[i];
-    }
-    tc_fence_before();
-    __syncthreads();
   }
+  if (ok && my_tiles > 0) {
+    const bool bad = !mbar_wait(bar_o, (my_tiles - 1) & 1, p.status) || flags[0];
+    ok = !__syncthreads_or(bad);
+  }
+  tc_fence_after();
 
   // ---- output
   const int g = p.Hq / p.Hkv;
@@ -259,36 +350,53 @@ __global__ void __launch_bounds__(128, 1)
   const int hl = r / p.n_rows;
   const int ii = r - hl * p.n_rows;
   const int h = kvh * g + hl;
-  auto store_row = [&](const float* vals, float inv) {
-    __nv_bfloat16* dst = p.out + ((size_t)(b * p.n_rows + ii) * p.Hq + h) * D;
+  __nv_bfloat16* dst = p.out + ((size_t)(b * p.n_rows + ii) * p.Hq + h) * D;
+  auto store16 = [&](int d0, const float (&v)[16], float inv) {
 #pragma unroll
-    for (int d0 = 0; d0 < D; d0 += 8) {
-      __nv_bfloat162 q0 = __floats2bfloat162_rn(vals[d0] * inv, vals[d0 + 1] * inv);
-      __nv_bfloat162 q1 = __floats2bfloat162_rn(vals[d0 + 2] * inv, vals[d0 + 3] * inv);
-      __nv_bfloat162 q2 = __floats2bfloat162_rn(vals[d0 + 4] * inv, vals[d0 + 5] * inv);
-      __nv_bfloat162 q3 = __floats2bfloat162_rn(vals[d0 + 6] * inv, vals[d0 + 7] * inv);
+    for (int q = 0; q < 16; q += 8) {
+      __nv_bfloat162 a0 = __floats2bfloat162_rn(v[q] * inv, v[q + 1] * inv);
+      __nv_bfloat162 a1 = __floats2bfloat162_rn(v[q + 2] * inv, v[q + 3] * inv);
+      __nv_bfloat162 a2 = __floats2bfloat162_rn(v[q + 4] * inv, v[q + 5] * inv);
+      __nv_bfloat162 a3 = __floats2bfloat162_rn(v[q + 6] * inv, v[q + 7] * inv);
       uint4 w;
-      w.x = *reinterpret_cast<uint32_t*>(&q0);
-      w.y = *reinterpret_cast<uint32_t*>(&q1);
-      w.z = *reinterpret_cast<uint32_t*>(&q2);
-      w.w = *reinterpret_cast<uint32_t*>(&q3);
-      *reinterpret_cast<uint4*>(dst + d0) = w;
+      w.x = *reinterpret_cast<uint32_t*>(&a0);
+      w.y = *reinterpret_cast<uint32_t*>(&a1);
+      w.z = *reinterpret_cast<uint32_t*>(&a2);
+      w.w = *reinterpret_cast<uint32_t*>(&a3);
+      *reinterpret_cast<uint4*>(dst + d0 + q) = w;
     }
   };
 
   if (ok) {
     if (p.chunks == 1) {
-      if (row_ok && l_run > 0.f) store_row(o, 1.f / l_run);
+      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+#pragma unroll
+      for (int c = 0; c < D / 16; ++c) {
+        float v[16];
+        tmem_ld16(o_tmem + lane_off + c * 16, v);
+        tmem_ld_wait();
+        if (row_ok && my_tiles > 0) store16(c * 16, v, inv);
+      }
     } else {
       const size_t grp = ((size_t)(b * p.Hkv + kvh) * p.row_tiles + rt);
       const size_t prow = (grp * p.chunks + chunk) * 128 + t;
-      if (row_ok) {
-        float4* dst = reinterpret_cast<float4*>(p.part_o + prow * D);
 #pragma unroll
-        for (int d0 = 0; d0 < D; d0 += 4)
-          dst[d0 >> 2] = make_float4(o[d0], o[d0 + 1], o[d0 + 2], o[d0 + 3]);
-        p.part_ml[prow] = make_float2(m_run, l_run);
+      for (int c = 0; c < D / 16; ++c) {
+        float v[16];
+        tmem_ld16(o_tmem + lane_off + c * 16, v);
+        tmem_ld_wait();
+        if (my_tiles == 0) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] = 0.f;
+        }
+        if (row_ok) {
+          float4* o4 = reinterpret_cast<float4*>(p.part_o + prow * D + c * 16);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            o4[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        }
       }
+      if (row_ok) p.part_ml[prow] = make_float2(m_run, l_run);
       __threadfence();
       __syncthreads();
       if (t == 0) {
@@ -298,34 +406,43 @@ __global__ void __launch_bounds__(128, 1)
         flags[1] = last;
       }
       __syncthreads();
-      if (flags[1]) {
+      if (flags[1] && row_ok) {
         __threadfence();
-        if (row_ok) {
-          float mx = -FLT_MAX;
-          for (int c = 0; c < p.chunks; ++c) {
-            const float2 ml = __ldcg(&p.part_ml[(grp * p.chunks + c) * 128 + t]);
-            if (ml.y > 0.f) mx = fmaxf(mx, ml.x);
-          }
-          float lt = 0.f;
+        float mx = -FLT_MAX, lt = 0.f;
+        for (int c = 0; c < p.chunks; ++c) {
+          const float2 ml = __ldcg(&p.part_ml[(grp * p.chunks + c) * 128 + t]);
+          if (ml.y > 0.f) mx = fmaxf(mx, ml.x);
+        }
+        for (int c = 0; c < p.chunks; ++c) {
+          const float2 ml = __ldcg(&p.part_ml[(grp * p.chunks + c) * 128 + t]);
+          if (ml.y > 0.f) lt += exp2f(ml.x - mx) * ml.y;
+        }
+        const float inv = lt > 0.f ? 1.f / lt : 0.f;
+        // chunk-outer: each chunk's whole row is requested at once
+        float o[D];
 #pragma unroll
-          for (int i = 0; i < D; ++i) o[i] = 0.f;
-          for (int c = 0; c < p.chunks; ++c) {
-            const size_t cr = (grp * p.chunks + c) * 128 + t;
-            const float2 ml = __ldcg(&p.part_ml[cr]);
-            if (!(ml.y > 0.f)) continue;
-            const float w = exp2f(ml.x - mx);
-            lt += w * ml.y;
-            const float4* src = reinterpret_cast<const float4*>(p.part_o + cr * D);
+        for (int i = 0; i < D; ++i) o[i] = 0.f;
+        for (int c = 0; c < p.chunks; ++c) {
+          const size_t cr = (grp * p.chunks + c) * 128 + t;
+          const float2 ml = __ldcg(&p.part_ml[cr]);
+          if (!(ml.y > 0.f)) continue;
+          const float wgt = exp2f(ml.x - mx);
+          const float4* src = reinterpret_cast<const float4*>(p.part_o + cr * D);
 #pragma unroll
-            for (int d0 = 0; d0 < D; d0 += 4) {
-              const float4 x = __ldcg(src + (d0 >> 2));
-              o[d0] += w * x.x;
-              o[d0 + 1] += w * x.y;
-              o[d0 + 2] += w * x.z;
-              o[d0 + 3] += w * x.w;
-            }
+          for (int q = 0; q < D / 4; ++q) {
+            const float4 x = __ldcg(src + q);
+            o[4 * q] += wgt * x.x;
+            o[4 * q + 1] += wgt * x.y;
+            o[4 * q + 2] += wgt * x.z;
+            o[4 * q + 3] += wgt * x.w;
           }
-          if (lt > 0.f) store_row(o, 1.f / lt);
+        }
+#pragma unroll
+        for (int d0 = 0; d0 < D; d0 += 16) {
+          float v[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] = o[d0 + i];
+          store16(d0, v, inv);
         }
       }
     }
@@ -338,23 +455,15 @@ __global__ void __launch_bounds__(128, 1)
   }
 }
 
-template <int D>
+template <int D, int ST>
 static cudaError_t launch_attn_t(const CUtensorMap& qmap, const CUtensorMap& kmap,
                                  const CUtensorMap& vmap, const AttnParams& p, bool pdl,
                                  cudaStream_t s) {
-  auto kern = attn_kernel<D>;
-  const size_t smem = AttnCfg<D>::kSmem;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  auto kern = attn_kernel<D, ST>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.batch * p.Hkv * p.row_tiles * p.chunks);
   cfg.blockDim = dim3(128);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = AttnCfg<D, ST>::kSmem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -365,15 +474,32 @@ static cudaError_t launch_attn_t(const CUtensorMap& qmap, const CUtensorMap& kma
   return cudaLaunchKernelEx(&cfg, kern, qmap, kmap, vmap, p);
 }
 
-size_t attn_smem_bytes(int head_dim) {
-  return head_dim == 128 ? AttnCfg<128>::kSmem : AttnCfg<32>::kSmem;
+cudaError_t attn_prepare() {
+  cudaError_t e = cudaSuccess;
+#define DLLM_SET(D, ST)                                                                   \
+  if (e == cudaSuccess)                                                                  \
+    e = cudaFuncSetAttribute(attn_kernel<D, ST>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                             (int)AttnCfg<D, ST>::kSmem);
+  DLLM_SET(128, 1) DLLM_SET(128, 2) DLLM_SET(32, 1) DLLM_SET(32, 2)
+#undef DLLM_SET
+  return e;
 }
 
+size_t attn_smem_bytes(int head_dim) {
+  return head_dim == 128 ? AttnCfg<128, 2>::kSmem : AttnCfg<32, 2>::kSmem;
+}
+
+// One key tile per CTA keeps a single stage; longer chunks double-buffer.
 cudaError_t launch_attn(int head_dim, const CUtensorMap& qmap, const CUtensorMap& kmap,
                         const CUtensorMap& vmap, const AttnParams& p, bool pdl,
                         cudaStream_t s) {
-  if (head_dim == 128) return launch_attn_t<128>(qmap, kmap, vmap, p, pdl, s);
-  if (head_dim == 32) return launch_attn_t<32>(qmap, kmap, vmap, p, pdl, s);
+  const bool one = p.tiles_per_chunk <= 1;
+  if (head_dim == 128)
+    return one ? launch_attn_t<128, 1>(qmap, kmap, vmap, p, pdl, s)
+               : launch_attn_t<128, 2>(qmap, kmap, vmap, p, pdl, s);
+  if (head_dim == 32)
+    return one ? launch_attn_t<32, 1>(qmap, kmap, vmap, p, pdl, s)
+               : launch_attn_t<32, 2>(qmap, kmap, vmap, p, pdl, s);
   return cudaErrorInvalidValue;
 }
 

@@ -13,10 +13,11 @@
 //   EPI_OPROJ  residual add in fp32, bf16 copy for the next projection
 //   EPI_LMHEAD per-row running max / sum-exp / argmax / second max over the
 //              CTA's vocabulary tiles; logits never leave the SM
-// When (weight tiles x row tiles) would leave SMs idle, K is split; each split
-// writes an fp32 partial to a scratch slot and the last split to arrive (a
-// per-tile counter) sums the slots in split order and runs the epilogue, so
-// the result does not depend on arrival order.
+// When (weight tiles x row tiles) would leave SMs idle, K is split: the
+// splits of a tile run as one thread-block cluster, one unit per CTA, and
+// their fp32 partials are summed in rank order in the shared memory of rank
+// 0 through distributed shared memory, so the result does not depend on
+// timing and no partial goes through global memory.
 #include <float.h>
 #include <limits.h>
 
@@ -27,7 +28,10 @@ namespace dllm {
 
 template <int NT>
 struct GemmCfg {
-  static constexpr int kStages = NT <= 32 ? 8 : NT <= 64 ? 6 : NT <= 128 ? 5 : 4;
+  // Decode tiles (NT <= 64) keep the CTA near 70 KB of shared memory so that
+  // two CTAs of the next GEMM fit beside a running one and start streaming
+  // their weights before it finishes.
+  static constexpr int kStages = NT <= 64 ? 3 : 4;
   static constexpr int kWBytes = 128 * 64 * 2;
   static constexpr int kXBytes = NT * 64 * 2;
   static constexpr int kTmemCols = 2 * NT;
@@ -82,21 +86,45 @@ __device__ __forceinline__ float column_sum16(const float* stage, int et) {
   return s;
 }
 
-// Per-unit preparation of the final epilogue (QKV: the RMS scale of each
-// activation row, from the partial sums of squares, into inv[NT]).
+// Per-unit preparation of the final epilogue.  The epilogue warps run it
+// while the unit's mainloop is still streaming: it reads only what earlier
+// kernels wrote.  QKV, per activation row c of the tile: inv[c] = RMS scale
+// (from the partial sums of squares), rp[c] = rotary position, and the row
+// parts of the destination offsets in units of head_dim, qoff[c] into q and
+// koff[c] into the caches (the head / kv-head parts are added per weight row).
 template <int NT, int EPI>
-__device__ __forceinline__ void epi_prepare(const GemmParams& p, int n, int et, float* inv) {
+__device__ __forceinline__ void epi_prepare(const GemmParams& p, int n, int et, float* inv,
+                                            int* rp) {
   if constexpr (EPI == EPI_QKV) {
-    for (int c = et; c < NT; c += 128) {
+    int* qoff = rp + NT;
+    int* koff = qoff + NT;
+    constexpr int TPC = NT >= 128 ? 1 : 128 / NT;  // threads per column
+    const int sub = et % TPC;
+    for (int c = et / TPC; c < NT; c += 128 / TPC) {
       const int xrow = n * NT + c;
-      float r = 1.f;
+      float s = 0.f;
       if (p.sumsq_in != nullptr && xrow < p.R) {
         const float* src = p.sumsq_in + (size_t)xrow * p.npart;
-        float s = 0.f;
-        for (int k = 0; k < p.npart; ++k) s += src[k];
-        r = rsqrtf(s / (float)p.d_norm + p.rms_eps);
+#pragma unroll 8
+        for (int k = sub; k < p.npart; k += TPC) s += src[k];
       }
-      inv[c] = r;
+#pragma unroll
+      for (int o = 1; o < TPC; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      if (sub == 0) {
+        inv[c] = p.sumsq_in != nullptr ? rsqrtf(s / (float)p.d_norm + p.rms_eps) : 1.f;
+        int r = 0, qo = 0, ko = 0;
+        if (xrow < p.R) {
+          const int b = xrow / p.n_rows;
+          const int ii = xrow - b * p.n_rows;
+          const int pos = p.row0 + ii;
+          if (p.rope_tab != nullptr) r = pos - p.seq_start[b];
+          qo = b * p.Hq * p.n_rows + ii;                       // in units of D
+          ko = (p.layer * p.batch + b) * p.Hkv * p.S + pos;    // in units of D
+        }
+        rp[c] = r < 0 ? 0 : r;
+        qoff[c] = qo;
+        koff[c] = ko;
+      }
     }
     named_bar_sync(1, 128);
   }
@@ -109,13 +137,20 @@ __device__ __forceinline__ void epi_chunk(const GemmParams& p, int m, int n, int
                                           LmStat* run) {
   if constexpr (EPI == EPI_OPROJ) {
     const int wrow = m * 128 + wl;
+    // all residual loads first: stores to x below would otherwise order them
+    float xo[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int xrow = n * NT + c0 + i;
+      xo[i] = xrow < p.R ? p.x[(size_t)xrow * p.d_model + wrow] : 0.f;
+    }
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const int xrow = n * NT + c0 + i;
       float sq = 0.f;
       if (xrow < p.R) {
         const size_t off = (size_t)xrow * p.d_model + wrow;
-        const float nx = p.x[off] + v[i];
+        const float nx = xo[i] + v[i];
         p.x[off] = nx;
         p.xb[off] = __float2bfloat16_rn(nx);
         sq = nx * nx;
@@ -131,44 +166,54 @@ __device__ __forceinline__ void epi_chunk(const GemmParams& p, int m, int n, int
     }
   } else if constexpr (EPI == EPI_QKV) {
     const float* inv = reinterpret_cast<const float*>(run);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) stage[i * 128 + wl] = v[i] * inv[c0 + i];
-    named_bar_sync(1, 128);
+    const int* rpos = reinterpret_cast<const int*>(inv + NT);
+    const int* qoff = rpos + NT;
+    const int* koff = qoff + NT;
     const int D = p.D, half = D >> 1;
     const int wrow = m * 128 + wl;
     const int head = wrow / D;
     const int dd = wrow - head * D;
     const bool is_q = head < p.Hq;
     const bool is_k = !is_q && head < p.Hq + p.Hkv;
-    const bool rope = (p.rope_tab != nullptr) && (is_q || is_k);
-    const int partner = wl + (dd < half ? half : -half);
-    const int j = dd < half ? dd : dd - half;
+    const bool has_rope = p.rope_tab != nullptr;  // uniform over the CTA
+    float val[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) val[i] = v[i] * inv[c0 + i];
+    if (has_rope) {
+      // rotate-half pairs live in lanes dd and dd +- D/2 of the same tile
+#pragma unroll
+      for (int i = 0; i < 16; ++i) stage[i * 128 + wl] = val[i];
+      named_bar_sync(1, 128);
+      if (is_q || is_k) {
+        const int partner = wl + (dd < half ? half : -half);
+        const int j = dd < half ? dd : dd - half;
+        float2 cs[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) cs[i] = p.rope_tab[(size_t)rpos[c0 + i] * half + j];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float o = stage[i * 128 + partner];
+          val[i] = dd < half ? (val[i] * cs[i].x - o * cs[i].y) : (val[i] * cs[i].x + o * cs[i].y);
+        }
+      }
+      named_bar_sync(1, 128);
+    }
+    __nv_bfloat16* dst;
+    size_t hoff;
+    if (is_q) {
+      dst = p.q_out;
+      hoff = (size_t)head * p.n_rows * D + dd;
+    } else {
+      const int kvh = is_k ? head - p.Hq : head - p.Hq - p.Hkv;
+      dst = is_k ? p.k_cache : p.v_cache;
+      hoff = (size_t)kvh * p.S * D + dd;
+    }
+    const int* roff = is_q ? qoff : koff;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      const int xrow = n * NT + c0 + i;
-      if (xrow >= p.R) continue;
-      const int b = xrow / p.n_rows;
-      const int ii = xrow - b * p.n_rows;
-      const int pos = p.row0 + ii;
-      float val = stage[i * 128 + wl];
-      if (rope) {
-        int rp = pos - p.seq_start[b];
-        rp = rp < 0 ? 0 : rp;
-        const float2 cs = p.rope_tab[(size_t)rp * half + j];
-        const float o = stage[i * 128 + partner];
-        val = dd < half ? (val * cs.x - o * cs.y) : (val * cs.x + o * cs.y);
-      }
-      const __nv_bfloat16 bv = __float2bfloat16_rn(val);
-      if (is_q) {
-        p.q_out[(((size_t)b * p.Hq + head) * p.n_rows + ii) * D + dd] = bv;
-      } else {
-        const int kvh = is_k ? head - p.Hq : head - p.Hq - p.Hkv;
-        const size_t off =
-            ((((size_t)p.layer * p.batch + b) * p.Hkv + kvh) * p.S + pos) * (size_t)D + dd;
-        (is_k ? p.k_cache : p.v_cache)[off] = bv;
-      }
+      if (n * NT + c0 + i < p.R)
+        dst[(size_t)roff[c0 + i] * D + hoff] = __float2bfloat16_rn(val[i]);
     }
-    named_bar_sync(1, 128);
   } else {  // EPI_LMHEAD
 #pragma unroll
     for (int i = 0; i < 16; ++i) stage[i * 128 + wl] = v[i];
@@ -203,7 +248,7 @@ __device__ __forceinline__ void epi_chunk(const GemmParams& p, int m, int n, int
 }
 
 template <int NT, int EPI>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(192, NT <= 32 ? 3 : NT <= 64 ? 2 : 1)
     gemm_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap xmap,
                 const GemmParams p) {
   using C = GemmCfg<NT>;
@@ -224,6 +269,9 @@ __global__ void __launch_bounds__(192, 1)
   volatile int* flags = reinterpret_cast<volatile int*>(tmem_slot + 2);  // [0] abort, [1] last
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // Split K is reduced inside a thread-block cluster for decode tiles.
+  constexpr bool kClusterSplit = NT <= 64;
+  float part[kClusterSplit ? NT : 1];
   if (threadIdx.x == 0) {
     for (int s = 0; s < ST; ++s) {
       mbar_init(&full[s], 1);
@@ -252,15 +300,34 @@ __global__ void __launch_bounds__(192, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    grid_dep_wait();
     if (lane == 0) {
       const uint64_t pol_w = policy_evict_first();
+      // The weights do not depend on the previous kernel: the first stages of
+      // the first unit are requested before waiting for it to finish.
+      int pre = 0, pre_kb0 = 0, pre_n = 0;
+      if ((int)blockIdx.x < p.units) {
+        int m, n, tile, kb0, kb1;
+        decode_unit(p, blockIdx.x, m, n, tile, kb0, kb1);
+        pre = min(ST, kb1 - kb0);
+        pre_kb0 = kb0;
+        pre_n = n;
+        for (int i = 0; i < pre; ++i) {
+          mbar_arrive_expect_tx(&full[i], C::kWBytes + C::kXBytes);
+          tma_load_3d_hint(w_st + i * C::kWBytes, &wmap, &full[i], (kb0 + i) * 64, m * 128,
+                           p.layer, pol_w);
+        }
+      }
+      grid_dep_wait();
+      for (int i = 0; i < pre; ++i)
+        tma_load_3d(x_st + i * C::kXBytes, &xmap, &full[i], ((pre_kb0 + i) % p.kx_blocks) * 64,
+                    pre_n * NT, 0);
       int it = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
         int m, n, tile, kb0, kb1;
         decode_unit(p, u, m, n, tile, kb0, kb1);
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          if (it < pre) continue;  // issued before the dependency wait
           const int s = it % ST;
           const uint32_t ph = (it / ST) & 1;
           if (!mbar_wait(&empty[s], ph ^ 1, p.status) || flags[0]) {
@@ -282,7 +349,10 @@ __global__ void __launch_bounds__(192, 1)
           mbar_wait(&full[j % ST], (j / ST) & 1, nullptr);
         }
       }
+    } else {
+      grid_dep_wait();
     }
+    __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     grid_dep_wait();
@@ -344,56 +414,38 @@ __global__ void __launch_bounds__(192, 1)
       decode_unit(p, u, m, n, tile, kb0, kb1);
       const int acc = j & 1;
       const uint32_t aph = (j >> 1) & 1;
+      float* inv = reinterpret_cast<float*>(run);
+      epi_prepare<NT, EPI>(p, n, et, inv, reinterpret_cast<int*>(inv + NT));
       const bool bad = !mbar_wait(&tfull[acc], aph, p.status) || flags[0];
       if (named_bar_or(1, 128, bad)) {
         flags[0] = 1;
         break;
       }
       tc_fence_after();
-      const bool split = p.splits > 1;
-      if (!split) epi_prepare<NT, EPI>(p, n, et, reinterpret_cast<float*>(run));
+      if constexpr (kClusterSplit) {
+        if (p.splits > 1) {
+          // cluster split-K: keep this CTA's partial for the reduction below
+#pragma unroll
+          for (int c0 = 0; c0 < NT; c0 += 16) {
+            float v[16];
+            tmem_ld16(tmem + ((uint32_t)lane_base << 16) + acc * NT + c0, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) part[c0 + i] = v[i];
+          }
+          tc_fence_before();
+          mbar_arrive(&tempty[acc]);
+          continue;
+        }
+      }
       for (int c0 = 0; c0 < NT; c0 += 16) {
         float v[16];
         tmem_ld16(tmem + ((uint32_t)lane_base << 16) + acc * NT + c0, v);
         tmem_ld_wait();
-        if (split) {
-          float* slot = p.slots + ((size_t)u * NT + c0) * 128;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) slot[i * 128 + wl] = v[i];
-        } else {
-          epi_chunk<NT, EPI>(p, m, n, c0, wl, et, v, stage, run);
-        }
+        epi_chunk<NT, EPI>(p, m, n, c0, wl, et, v, stage, run);
       }
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
-      if (split) {
-        __threadfence();
-        named_bar_sync(1, 128);
-        if (et == 0) {
-          const int old = atomicAdd(&p.counters[tile], 1);
-          const int last = (old == p.splits - 1);
-          if (last) p.counters[tile] = 0;
-          flags[1] = last;
-        }
-        named_bar_sync(1, 128);
-        const int last = flags[1];
-        named_bar_sync(1, 128);
-        if (last) {
-          __threadfence();
-          epi_prepare<NT, EPI>(p, n, et, reinterpret_cast<float*>(run));
-          for (int c0 = 0; c0 < NT; c0 += 16) {
-            float v[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] = 0.f;
-            for (int sp = 0; sp < p.splits; ++sp) {
-              const float* slot = p.slots + ((size_t)(tile * p.splits + sp) * NT + c0) * 128;
-#pragma unroll
-              for (int i = 0; i < 16; ++i) v[i] += __ldcg(slot + i * 128 + wl);
-            }
-            epi_chunk<NT, EPI>(p, m, n, c0, wl, et, v, stage, run);
-          }
-        }
-      }
     }
     if constexpr (EPI == EPI_LMHEAD) {
       named_bar_sync(1, 128);
@@ -402,6 +454,43 @@ __global__ void __launch_bounds__(192, 1)
       for (int c = et; c < NT; c += 128) {
         const int xrow = n * NT + c;
         if (xrow < p.R) p.stats[(size_t)xrow * p.stat_slots + slot] = run[c];
+      }
+    }
+  }
+  __syncthreads();
+  if constexpr (kClusterSplit) {
+    if (p.splits > 1) {
+      // The splits of a tile form one cluster (one unit per CTA).  After
+      // every mainloop is done, ranks 1.. store their partial into rank 0's
+      // (now idle) stage buffers through distributed shared memory; rank 0
+      // adds them in rank order and runs the epilogue.
+      cluster_sync();
+      const uint32_t rank = cluster_ctarank();
+      const bool epi = warp >= 2;
+      const int et = threadIdx.x - 64;
+      const int wl = 32 * (warp & 3) + (threadIdx.x & 31);
+      float* red = reinterpret_cast<float*>(w_st);  // [rank-1][NT columns][128 lanes]
+      if (epi && rank != 0) {
+        const uint32_t dst = map_to_rank(smem_u32(red + (size_t)(rank - 1) * NT * 128 + wl), 0);
+#pragma unroll
+        for (int c = 0; c < NT; ++c) st_cluster_f32(dst + c * 128 * 4, part[c]);
+      }
+      cluster_sync();
+      if (epi && rank == 0 && !flags[0]) {
+        int m, n, tile, kb0, kb1;
+        decode_unit(p, blockIdx.x, m, n, tile, kb0, kb1);
+        for (int r = 1; r < p.splits; ++r) {
+          const float* src = red + (size_t)(r - 1) * NT * 128 + wl;
+#pragma unroll
+          for (int c = 0; c < NT; ++c) part[c] += src[c * 128];
+        }
+#pragma unroll
+        for (int c0 = 0; c0 < NT; c0 += 16) {
+          float v[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] = part[c0 + i];
+          epi_chunk<NT, EPI>(p, m, n, c0, wl, et, v, stage, run);
+        }
       }
     }
   }
@@ -417,25 +506,46 @@ static cudaError_t launch_t(const CUtensorMap& wmap, const CUtensorMap& xmap, co
                             int grid, bool pdl, cudaStream_t s) {
   auto kern = gemm_kernel<NT, EPI>;
   const size_t smem = GemmCfg<NT>::kSmem;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(192);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (p.splits > 1) {
+    if (NT > 64 || grid != p.units) return cudaErrorInvalidValue;
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = p.splits;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
+  cfg.numAttrs = na;
   count_launch();
   return cudaLaunchKernelEx(&cfg, kern, wmap, xmap, p);
+}
+
+// Opt every kernel variant into its dynamic shared memory size up front, so
+// that no attribute call happens while a launch sequence is being captured.
+cudaError_t gemm_prepare() {
+  cudaError_t e = cudaSuccess;
+#define DLLM_SET(NT, EPI)                                                                      \
+  if (e == cudaSuccess)                                                                       \
+    e = cudaFuncSetAttribute(gemm_kernel<NT, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                             (int)GemmCfg<NT>::kSmem);
+  DLLM_SET(32, 0) DLLM_SET(32, 1) DLLM_SET(32, 2)
+  DLLM_SET(64, 0) DLLM_SET(64, 1) DLLM_SET(64, 2)
+  DLLM_SET(128, 0) DLLM_SET(128, 1) DLLM_SET(128, 2)
+  DLLM_SET(256, 0) DLLM_SET(256, 1) DLLM_SET(256, 2)
+#undef DLLM_SET
+  return e;
 }
 
 int gemm_stages(int nt) {

@@ -28,9 +28,6 @@ struct GemmParams {
   int m_tiles, n_tiles, splits, kb_per_split, units;
   int layer;
   int* status;
-  // split-K scratch: slots[unit][NT][128] fp32, counters[tile]
-  float* slots;
-  int* counters;
   // rows are (sequence, i) with position row0 + i, n_rows per sequence
   int n_rows, row0;
   const int* seq_start;
@@ -61,7 +58,10 @@ struct AttnParams {
   int row_tiles;    // ceil(group_rows / 128)
   int chunks;       // key chunks per (sequence, kv head, row tile)
   int tiles_per_chunk;
-  const int* segs;  // [b][2][2] (start, len)
+  const int* segs;  // [b][2][2] (start, len), or null: derived from the fields below
+  int mode, blk_start, blk_len, window, seg_end;
+  const int* seq_start;
+  int dep_lo, dep_hi;  // key positions the preceding kernel writes (load after the wait)
   __nv_bfloat16* out;  // [b*n_rows][Hq*D]
   float* part_o;       // [b][Hkv][row_tiles][chunks][128][D]
   float2* part_ml;     // [b][Hkv][row_tiles][chunks][128]
@@ -74,6 +74,8 @@ struct AttnParams {
 cudaError_t launch_gemm(int epi, int nt, const CUtensorMap& wmap, const CUtensorMap& xmap,
                         const GemmParams& p, int grid, bool pdl, cudaStream_t s);
 int gemm_stages(int nt);
+cudaError_t gemm_prepare();
+cudaError_t attn_prepare();
 size_t gemm_smem_bytes(int nt);
 
 cudaError_t launch_attn(int head_dim, const CUtensorMap& qmap, const CUtensorMap& kmap,

@@ -10,9 +10,10 @@
 
 namespace dllm {
 
-static unsigned long long g_launches = 0;
+static long long g_launches = 0;
 void count_launch() { ++g_launches; }
-unsigned long long launch_count() { return g_launches; }
+void add_launches(long long n) { g_launches += n; }
+unsigned long long launch_count() { return (unsigned long long)g_launches; }
 
 template <class K, class... A>
 static cudaError_t launch_simple(K kern, dim3 grid, dim3 block, bool pdl, cudaStream_t s,
@@ -177,11 +178,12 @@ __device__ __forceinline__ LmStat merge_stat(const LmStat& a, const LmStat& b) {
   return r;
 }
 
-// One CTA (256 threads) per sequence.  Phase 1: merge the per-CTA vocabulary
-// statistics of each block row into conf = 1 / sum exp(l - max), tok, gap.
+// One CTA (1024 threads) per sequence.  Phase 1: one warp per block row
+// merges the per-CTA vocabulary statistics into conf = 1 / sum exp(l - max),
+// tok and gap.
 // Phase 2 (warp 0): commit masked rows with conf > tau, plus the most
 // confident masked row (lowest position on ties).
-__global__ void __launch_bounds__(256) commit_kernel(const CommitParams p) {
+__global__ void __launch_bounds__(1024) commit_kernel(const CommitParams p) {
   grid_dep_wait();
   grid_dep_launch();
   __shared__ float s_conf[64];
@@ -189,14 +191,23 @@ __global__ void __launch_bounds__(256) commit_kernel(const CommitParams p) {
   const int b = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (p.stats != nullptr) {
-    for (int i = warp; i < p.B; i += 8) {
+    const int nwarps = blockDim.x >> 5;
+    for (int i = warp; i < p.B; i += nwarps) {
       const LmStat* src = p.stats + (size_t)(b * p.B + i) * p.stat_slots;
       LmStat st;
       st.m = -FLT_MAX;
       st.s = 0.f;
       st.m2 = -FLT_MAX;
       st.idx = INT_MAX;
-      for (int k = lane; k < p.stat_slots; k += 32) st = merge_stat(st, src[k]);
+      LmStat buf[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {  // issue the loads before merging
+        const int k = lane + 32 * q;
+        buf[q] = k < p.stat_slots ? src[k] : st;
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) st = merge_stat(st, buf[q]);
+      for (int k = lane + 256; k < p.stat_slots; k += 32) st = merge_stat(st, src[k]);
 #pragma unroll
       for (int mask = 16; mask > 0; mask >>= 1) {
         LmStat o;
@@ -267,7 +278,7 @@ __global__ void __launch_bounds__(256) commit_kernel(const CommitParams p) {
 }
 
 cudaError_t launch_commit(const CommitParams& p, bool pdl, cudaStream_t s) {
-  return launch_simple(commit_kernel, dim3(p.batch), dim3(256), pdl, s, p);
+  return launch_simple(commit_kernel, dim3(p.batch), dim3(1024), pdl, s, p);
 }
 
 // ------------------------------------------------------------------ tables

@@ -208,8 +208,16 @@ dllm_status dllm_step_outputs(const dllm_config* cfg, void* ws, size_t ws_bytes,
 /* Copy the workspace's device status word to *code (host); synchronises stream. */
 dllm_status dllm_device_status(void* ws, int32_t* code, dllm_stream stream);
 
-/* Number of kernels this library has launched in this process. */
+/* Number of kernels this library has launched in this process (kernels run
+ * by a replayed graph included). */
 uint64_t dllm_launch_count(void);
+
+/* dllm_prefill, dllm_decode_step, dllm_kv_cache_refresh and dllm_decode_block
+ * record their launch sequence once per (configuration, weight, state and
+ * workspace pointers, block) as a CUDA graph and replay it afterwards.  The
+ * cache holds at most 256 graphs; this call destroys them all (call it before
+ * freeing buffers that a cached graph references, or to bound memory). */
+void dllm_graph_cache_clear(void);
 
 const char* dllm_status_string(dllm_status s);
 
