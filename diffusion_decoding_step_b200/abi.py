@@ -59,6 +59,7 @@ SIGNATURES = {
     "dllm_o_proj": (C.c_int, [_CFG, _W, _I, _P, _I, _I, _P, _P, _P, _P, C.c_size_t, _P]),
     "dllm_final_norm": (C.c_int, [_CFG, _P, _I, _I, _I, _P, _P, _P, _P]),
     "dllm_lmhead_confidence": (C.c_int, [_CFG, _W, _P, _I, _P, _P, _P, _P, C.c_size_t, _P]),
+    "dllm_lmhead_confidence_noalloc": (C.c_int, [_CFG, _W, _P, _I, _P, _P, _P, _P]),
     "dllm_threshold_commit": (C.c_int, [_CFG, _I, _P, _P, _P, _P, _P, _P, _P]),
     "dllm_prefill": (C.c_int, [_CFG, _W, _ST, _P, C.c_size_t, _P]),
     "dllm_decode_step": (C.c_int, [_CFG, _W, _ST, _I, _P, C.c_size_t, _P]),

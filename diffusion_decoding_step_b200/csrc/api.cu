@@ -950,6 +950,92 @@ dllm_status dllm_device_status(void* ws, int32_t* code, dllm_stream stream) {
   return DLLM_OK;
 }
 
+// ---------------------------------------------------------------------------
+// LM head + confidence without a caller workspace.
+//
+// Some callers cannot hand this library device memory: they run under an
+// inference server or plugin host whose allocator owns the whole device pool
+// and forbids cudaMalloc on the request path, or they sit behind a binding
+// that can pass tensors but not an extra workspace buffer.  This entry point
+// serves them: its only scratch, the per-CTA vocabulary statistics, lives in
+// the fixed-size array below, which every GPU that loads the library keeps
+// until the process exits.  Nothing here allocates.
+// ---------------------------------------------------------------------------
+namespace {
+constexpr int kNoAllocMaxSlots = 160;  // persistent LM-head CTAs per row tile (<= SM count)
+}
+static __device__ __align__(256) dllm::LmStat
+    g_noalloc_stats[DLLM_NOALLOC_MAX_ROWS * kNoAllocMaxSlots];
+
+namespace {
+// Device address of g_noalloc_stats on the current device, looked up once per
+// device (host code may not use the symbol itself as a device address).
+dllm::LmStat* noalloc_scratch() {
+  static std::mutex mu;
+  static dllm::LmStat* addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_stats) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<dllm::LmStat*>(ptr);
+  }
+  return addr[dev];
+}
+}  // namespace
+
+dllm_status dllm_lmhead_confidence_noalloc(const dllm_config* cfg, const dllm_weights* w,
+                                           const void* h, int32_t n_rows, float* conf,
+                                           int32_t* tok, float* gap, dllm_stream stream) {
+  Shape s;
+  DLLM_TRY(check_cfg(cfg, &s));
+  if (!w || !w->w_lm || !h || !conf || !tok) return DLLM_ERR_INVALID;
+  if (n_rows < 1) return DLLM_ERR_INVALID;
+  if (n_rows > DLLM_NOALLOC_MAX_ROWS) return DLLM_ERR_UNSUPPORTED;  // scratch holds 256 rows
+  DLLM_TRY(prepare_device());
+  const GemmPlan g = plan_lmhead(s.V, n_rows, s.Kw);
+  const int slots = g.grid / g.n_tiles;
+  if (slots > kNoAllocMaxSlots) return DLLM_ERR_UNSUPPORTED;
+  LmStat* scratch = noalloc_scratch();
+  if (!scratch) return DLLM_ERR_CUDA;
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  CUtensorMap wm, xm;
+  if (!make_map(&wm, w->w_lm, s.Kw, s.V, 1, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&xm, h, s.d, n_rows, 1, 64, g.nt, CU_TENSOR_MAP_SWIZZLE_128B))
+    return DLLM_ERR_CUDA;
+  GemmParams p{};
+  p.M = s.V;
+  p.R = n_rows;
+  p.K = s.Kw;
+  p.kx_blocks = s.d / 64;
+  p.m_tiles = g.m_tiles;
+  p.n_tiles = g.n_tiles;
+  p.splits = 1;
+  p.kb_per_split = g.kbps;
+  p.units = g.units;
+  p.layer = 0;
+  p.status = nullptr;
+  p.stats = scratch;  // every slot a later read needs is written by this launch
+  p.stat_slots = slots;
+  DLLM_TRY(cuda_status(launch_gemm(EPI_LMHEAD, g.nt, wm, xm, p, g.grid, false, st)));
+  for (int r0 = 0; r0 < n_rows; r0 += 64) {  // the reduce kernel takes 64 rows per CTA
+    CommitParams q{};
+    q.batch = 1;
+    q.B = std::min(64, n_rows - r0);
+    q.stat_slots = slots;
+    q.vocab = s.V;
+    q.tau = s.tau;
+    q.stats = scratch + (size_t)r0 * slots;
+    q.conf = conf + r0;
+    q.tok = tok + r0;
+    q.gap = gap ? gap + r0 : nullptr;
+    q.do_commit = 0;
+    DLLM_TRY(cuda_status(launch_commit(q, false, st)));
+  }
+  return DLLM_OK;
+}
+
 uint64_t dllm_launch_count(void) { return dllm::launch_count(); }
 
 const char* dllm_status_string(dllm_status s) {

@@ -165,6 +165,28 @@ dllm_status dllm_lmhead_confidence(const dllm_config* cfg, const dllm_weights* w
                                    const void* h, int32_t n_rows, float* conf, int32_t* tok,
                                    float* gap, void* ws, size_t ws_bytes, dllm_stream stream);
 
+/* Largest n_rows dllm_lmhead_confidence_noalloc accepts. */
+#define DLLM_NOALLOC_MAX_ROWS 256
+
+/* The same computation as dllm_lmhead_confidence for callers that cannot
+ * give the library any device memory (an allocator that owns the device pool
+ * and forbids cudaMalloc on the request path, or a binding that passes only
+ * tensors).  It allocates nothing and takes no workspace: its scratch is a
+ * fixed 640 KiB array in the library's device image, held by every GPU that
+ * loads the library until the process exits.  This call has no counterpart on
+ * the method's pages; it only changes where the scratch lives.
+ *  - n_rows must be <= DLLM_NOALLOC_MAX_ROWS; larger values return
+ *    DLLM_ERR_UNSUPPORTED and launch nothing.
+ *  - The first call on each device looks up the scratch's device address
+ *    (cudaGetSymbolAddress); make that first call before any stream capture.
+ *  - All calls share the one scratch array, whatever their stream: calls that
+ *    overlap on the GPU race and give wrong results.  Each call writes every
+ *    scratch entry it reads, so nothing needs clearing between calls.
+ *  - conf/tok/gap as in dllm_lmhead_confidence (gap may be NULL). */
+dllm_status dllm_lmhead_confidence_noalloc(const dllm_config* cfg, const dllm_weights* w,
+                                           const void* h, int32_t n_rows, float* conf,
+                                           int32_t* tok, float* gap, dllm_stream stream);
+
 /* Threshold commit of the block at block_start for every sequence: masked
  * rows with conf > tau commit, and the most confident masked row always does
  * (lowest position on ties).  conf/tok [b][B].  Updates tokens and masked;
