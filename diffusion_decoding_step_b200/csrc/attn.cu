@@ -28,7 +28,15 @@
 
 namespace dllm {
 
-constexpr int kKeys = 128;  // keys per tile
+constexpr int kKeys = 128;     // keys per tile
+constexpr int kMaxMerge = 4;   // key chunks per row tile (the merge keeps them all in flight)
+
+// 2^x with the SFU instruction (relative error ~2^-22; P is rounded to bf16).
+DLLM_DEV float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 template <int D, int ST>
 struct AttnCfg {
@@ -273,7 +281,7 @@ __global__ void __launch_bounds__(128, 1)
     for (int i = 0; i < kKeys; ++i)
       if (i < nvalid) tmax = fmaxf(tmax, s[i]);
     const float m_new = fmaxf(m_run, tmax * p.scale_log2);
-    const float alpha = exp2f(m_run - m_new);
+    const float alpha = fast_exp2(m_run - m_new);
     float lsum = 0.f;
 #pragma unroll
     for (int c = 0; c < kKeys / 8; ++c) {  // 8 keys = one 16-byte chunk of P
@@ -281,8 +289,8 @@ __global__ void __launch_bounds__(128, 1)
 #pragma unroll
       for (int i = 0; i < 8; i += 2) {
         const int k0 = c * 8 + i;
-        const float p0 = k0 < nvalid ? exp2f(s[k0] * p.scale_log2 - m_new) : 0.f;
-        const float p1 = k0 + 1 < nvalid ? exp2f(s[k0 + 1] * p.scale_log2 - m_new) : 0.f;
+        const float p0 = k0 < nvalid ? fast_exp2(s[k0] * p.scale_log2 - m_new) : 0.f;
+        const float p1 = k0 + 1 < nvalid ? fast_exp2(s[k0 + 1] * p.scale_log2 - m_new) : 0.f;
         const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
         lsum += __low2float(h2) + __high2float(h2);
         pk[i >> 1] = *reinterpret_cast<const uint32_t*>(&h2);
@@ -406,43 +414,79 @@ __global__ void __launch_bounds__(128, 1)
         flags[1] = last;
       }
       __syncthreads();
-      if (flags[1] && row_ok) {
+      if (flags[1]) {
         __threadfence();
-        float mx = -FLT_MAX, lt = 0.f;
-        for (int c = 0; c < p.chunks; ++c) {
-          const float2 ml = __ldcg(&p.part_ml[(grp * p.chunks + c) * 128 + t]);
-          if (ml.y > 0.f) mx = fmaxf(mx, ml.x);
-        }
-        for (int c = 0; c < p.chunks; ++c) {
-          const float2 ml = __ldcg(&p.part_ml[(grp * p.chunks + c) * 128 + t]);
-          if (ml.y > 0.f) lt += exp2f(ml.x - mx) * ml.y;
-        }
-        const float inv = lt > 0.f ? 1.f / lt : 0.f;
-        // chunk-outer: each chunk's whole row is requested at once
-        float o[D];
+        // The tile's existing rows are spread over all 128 threads (up to 4
+        // threads per row); every chunk's partial of a 16-column group is
+        // requested before any of it is used.
+        const int nv_rows = min(128, p.group_rows - rt * 128);
+        // each thread owns a multiple of 16 columns (D/16 threads per row at most)
+        const int tpr = min(nv_rows <= 32 ? 4 : nv_rows <= 64 ? 2 : 1, D / 16);
+        const int row = t / tpr, part = t % tpr;
+        if (row < nv_rows) {
+          const size_t base_r = grp * p.chunks * 128 + row;  // + c * 128
+          float2 ml[kMaxMerge];
 #pragma unroll
-        for (int i = 0; i < D; ++i) o[i] = 0.f;
-        for (int c = 0; c < p.chunks; ++c) {
-          const size_t cr = (grp * p.chunks + c) * 128 + t;
-          const float2 ml = __ldcg(&p.part_ml[cr]);
-          if (!(ml.y > 0.f)) continue;
-          const float wgt = exp2f(ml.x - mx);
-          const float4* src = reinterpret_cast<const float4*>(p.part_o + cr * D);
+          for (int c = 0; c < kMaxMerge; ++c)
+            ml[c] = c < p.chunks ? __ldcg(&p.part_ml[base_r + (size_t)c * 128])
+                                 : make_float2(-FLT_MAX, 0.f);
+          float mx = -FLT_MAX;
 #pragma unroll
-          for (int q = 0; q < D / 4; ++q) {
-            const float4 x = __ldcg(src + q);
-            o[4 * q] += wgt * x.x;
-            o[4 * q + 1] += wgt * x.y;
-            o[4 * q + 2] += wgt * x.z;
-            o[4 * q + 3] += wgt * x.w;
+          for (int c = 0; c < kMaxMerge; ++c)
+            if (ml[c].y > 0.f) mx = fmaxf(mx, ml[c].x);
+          float wgt[kMaxMerge], lt = 0.f;
+#pragma unroll
+          for (int c = 0; c < kMaxMerge; ++c) {
+            wgt[c] = ml[c].y > 0.f ? fast_exp2(ml[c].x - mx) : 0.f;
+            lt += wgt[c] * ml[c].y;
           }
-        }
+          const float inv = lt > 0.f ? 1.f / lt : 0.f;
+          const int rr = rt * 128 + row;
+          const int hl2 = rr / p.n_rows;
+          const int ii2 = rr - hl2 * p.n_rows;
+          __nv_bfloat16* dst2 =
+              p.out + ((size_t)(b * p.n_rows + ii2) * p.Hq + (kvh * g + hl2)) * D;
+          const int ncol = D / tpr;
+          for (int d0 = part * ncol; d0 < (part + 1) * ncol; d0 += 16) {
+            float4 x[kMaxMerge][4];
 #pragma unroll
-        for (int d0 = 0; d0 < D; d0 += 16) {
-          float v[16];
+            for (int c = 0; c < kMaxMerge; ++c) {
+              const float4* src = reinterpret_cast<const float4*>(
+                  p.part_o + (base_r + (size_t)c * 128) * D + d0);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) v[i] = o[d0 + i];
-          store16(d0, v, inv);
+              for (int q = 0; q < 4; ++q)
+                x[c][q] = c < p.chunks ? __ldcg(src + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+            float v[16];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+              for (int c = 0; c < kMaxMerge; ++c) {
+                acc.x += wgt[c] * x[c][q].x;
+                acc.y += wgt[c] * x[c][q].y;
+                acc.z += wgt[c] * x[c][q].z;
+                acc.w += wgt[c] * x[c][q].w;
+              }
+              v[4 * q] = acc.x * inv;
+              v[4 * q + 1] = acc.y * inv;
+              v[4 * q + 2] = acc.z * inv;
+              v[4 * q + 3] = acc.w * inv;
+            }
+#pragma unroll
+            for (int q = 0; q < 16; q += 8) {
+              __nv_bfloat162 a0 = __floats2bfloat162_rn(v[q], v[q + 1]);
+              __nv_bfloat162 a1 = __floats2bfloat162_rn(v[q + 2], v[q + 3]);
+              __nv_bfloat162 a2 = __floats2bfloat162_rn(v[q + 4], v[q + 5]);
+              __nv_bfloat162 a3 = __floats2bfloat162_rn(v[q + 6], v[q + 7]);
+              uint4 wv;
+              wv.x = *reinterpret_cast<uint32_t*>(&a0);
+              wv.y = *reinterpret_cast<uint32_t*>(&a1);
+              wv.z = *reinterpret_cast<uint32_t*>(&a2);
+              wv.w = *reinterpret_cast<uint32_t*>(&a3);
+              *reinterpret_cast<uint4*>(dst2 + d0 + q) = wv;
+            }
+          }
         }
       }
     }
