@@ -96,6 +96,73 @@ def workload_config(w, data_note):
             "l2": data_note}
 
 
+def step_key_counts(w, s):
+    """Keys each sequence attends to in a step of the block at position s."""
+    starts = [int(x) for x in _seq_starts(w)]
+    end = s + w.block
+    out = []
+    for st in starts:
+        if w.mode == 2:                       # DualCache: the whole valid range
+            n = w.seq_len - st
+        elif w.mode == 3:                     # pruned suffix window + trailing position
+            wend = min(end + w.window, w.seq_len)
+            n = wend - st + (1 if end < w.seq_len and w.seq_len - 1 >= wend else 0)
+        else:                                 # no cache / prefix cache
+            n = end - st
+        out.append(n)
+    return out
+
+
+def _seq_starts(w):
+    from diffusion_decoding_step_b200 import workload as wl
+    return wl.seq_starts(w)
+
+
+def step_algorithmic_bytes(w, s):
+    """Bytes one denoising step of the block at s must move through HBM once:
+    every layer's projection weights, the keys/values it attends to, the new
+    K/V rows it writes and the activations between kernels, then the LM-head
+    weights.  Logits are never stored, so they are not counted."""
+    d, D, Hq, Hkv = w.hidden, w.head_dim, w.n_q_heads, w.n_kv_heads
+    rows = w.batch * ((s + w.block) if w.mode == 0 else w.block)
+    per_layer = (w.qkv_rows * d * 2 + d * Hq * D * 2            # W_qkv, W_o
+                 + sum(step_key_counts(w, s)) * Hkv * D * 2 * 2  # K, V read
+                 + rows * (Hq + 2 * Hkv) * D * 2                 # q, k, v written
+                 + rows * d * 2                                  # xb read by QKV
+                 + rows * Hq * D * 2 * 3                         # q read, out written, out read
+                 + rows * d * (4 + 4 + 2))                       # x read + written, xb written
+    lm_rows = w.batch * w.block
+    return (w.n_layers * per_layer + w.vocab * d * 2 + lm_rows * d * 2
+            + lm_rows * d * (4 + 2))
+
+
+def gemm_source_sha1():
+    """Digest of the GEMM kernel's sources, to tie stored ncu counters to them."""
+    import hashlib
+    h = hashlib.sha1()
+    for name in ("gemm.cu", "kernels.cuh", "ptx.cuh"):
+        with open(os.path.join(ROOT, "diffusion_decoding_step_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def max_over_ranks(value, world, device=None):
+    """The slowest rank's figure; every rank must call this in the same order."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_env():
+    """(rank, world, local_rank) from the launcher's environment."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
     def __init__(self, index: int):
@@ -260,11 +327,7 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     launches = abi.dllm_launch_count() - launches0
     clk = clocks.stop() if clocks else None
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t)
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     tokens_total = world * w.batch * w.gen_len * args.steps
     value = tokens_total / (ms / 1000.0)
     assert dec.device_status() == 0
@@ -292,6 +355,8 @@ def run_ours(args, rank, world, local_rank):
 
     # dominant kernel: the Q/K/V projection of one layer, same launch shape as a step
     hbm, tflops, peak_kind = peaks()
+    step_bytes = step_algorithmic_bytes(w, w.prompt_len)
+    step_gbs = step_bytes / (statistics.median(step_us) * 1e-6) / 1e9
     rows = w.batch * w.block
     cfg_p = C.byref(dec.cfg)
     q = torch.empty(rows * w.n_q_heads * w.head_dim, dtype=torch.bfloat16, device=dev)
@@ -323,7 +388,10 @@ def run_ours(args, rank, world, local_rank):
     traffic = None
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
-            traffic = json.load(f).get(f"{w.name}:qkv_proj")
+            tj = json.load(f)
+        # counters only count while the kernel source they were taken on is unchanged
+        if tj.get("_gemm_source_sha1") == gemm_source_sha1():
+            traffic = tj.get(f"{w.name}:qkv_proj")
     except Exception:
         pass
 
@@ -354,11 +422,7 @@ def run_ours(args, rank, world, local_rank):
         e2e_generation()
     x1.record(stream)
     barrier()
-    e2e_ms = x0.elapsed_time(x1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t)
+    e2e_ms = max_over_ranks(x0.elapsed_time(x1), world, dev)
     e2e_value = tokens_total / (e2e_ms / 1000.0)
 
     cpu = None
@@ -384,6 +448,10 @@ def run_ours(args, rank, world, local_rank):
                                "isolated_max": max(step_us)},
             "denoising_steps_per_generation": denoise_steps / args.steps,
             "prefill_ms": prefill_ms,
+            "step_roofline": {"bound": "hbm", "algorithmic_bytes": step_bytes,
+                              "isolated_p50_us": statistics.median(step_us),
+                              "achieved": step_gbs, "peak": hbm, "unit": "GB/s",
+                              "frac": step_gbs / hbm, "peak_kind": peak_kind},
             "roofline": {"bound": "hbm", "kernel": "qkv_proj (tcgen05 GEMM, fused RoPE + "
                          "cache write)", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                          "frac": achieved / hbm, "traffic": traffic,
@@ -400,9 +468,7 @@ def run_ours(args, rank, world, local_rank):
 
 def main():
     args = parse()
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local_rank = rank_env()
     if args.impl == "reference":
         run_reference(args, rank, world)
         return

@@ -97,7 +97,7 @@ typedef struct {
   const int32_t* seq_start; /* [b] first valid position (left padding before it) */
   void* k_cache;            /* bf16 [L][b][Hkv][S][D]; must hold finite values */
   void* v_cache;            /* bf16 [L][b][Hkv][S][D] */
-  const void* plants;       /* bf16 [b][G][hidden] layer-0 input of masked generated rows */
+  const void* plants;       /* bf16 [b][G][hidden] planted LM-head offsets of generated rows */
 } dllm_state;
 
 /* Bytes of workspace a configuration needs (host call, no GPU work). */
