@@ -72,6 +72,7 @@ SIGNATURES = {
     "dllm_device_status": (C.c_int, [_P, C.POINTER(C.c_int32), _P]),
     "dllm_launch_count": (C.c_uint64, []),
     "dllm_graph_cache_clear": (None, []),
+    "dllm_set_l2_prefetch": (C.c_int, [C.c_int64, C.c_int64, C.c_int32]),
     "dllm_status_string": (C.c_char_p, [C.c_int]),
 }
 

@@ -161,7 +161,7 @@ AttnPlan plan_attn(const Shape& s, int n_rows, int ntile_bound) {
   const int g = s.Hq / s.Hkv;
   a.row_tiles = cdiv(g * n_rows, 128);
   const int base = s.b * s.Hkv * a.row_tiles;
-  // at most 4 key chunks per row tile: the merge holds them all in registers
+  // at most 4 key chunks per row tile: the chunks form one cluster and merge on chip
   int chunks = std::max(1, std::min({ntile_bound, cdiv(kNumSMs, base), 4}));
   if (base >= kNumSMs) chunks = 1;
   a.tpc = cdiv(ntile_bound, chunks);
@@ -188,9 +188,9 @@ int key_tiles_bound(const Shape& s, int blk, int seg_end) {
 
 // ------------------------------------------------------------------ workspace
 struct Layout {
-  size_t status, acnt, x, xb, sumsq, q, attn, h, stats, part_o, part_ml, conf, tok, gap, commit,
+  size_t status, x, xb, sumsq, q, attn, h, stats, conf, tok, gap, commit,
       remaining, segs, rope, total;
-  int rmax, lm_slots, acnt_n;
+  int rmax, lm_slots;
 };
 
 // Row counts (per sequence) a configuration uses: decode steps and prefill.
@@ -215,30 +215,11 @@ Layout layout(const Shape& s) {
   };
   const std::vector<int> rows = row_counts(s);
   int max_rows = 0;
-  size_t part_rows = 0;
-  int acnt = 1;
   for (int n : rows) max_rows = std::max(max_rows, n);
-  // attention partials: every decode step, plus the unit-level entry point
-  // (block rows against up to ceil(S/128)+1 key tiles)
-  auto need_attn = [&](int n_rows, int ntb) {
-    const AttnPlan a = plan_attn(s, n_rows, ntb);
-    if (a.chunks > 1)
-      part_rows = std::max(part_rows, (size_t)s.b * s.Hkv * a.row_tiles * a.chunks * 128);
-    acnt = std::max(acnt, s.b * s.Hkv * a.row_tiles);
-  };
-  for (int blk = s.P; blk < s.S; blk += s.B) {
-    if (s.mode == DLLM_CACHE_NONE)
-      need_attn(blk + s.B, key_tiles_bound(s, blk, blk + s.B));
-    else
-      need_attn(s.B, key_tiles_bound(s, blk, 0));
-  }
-  need_attn(s.B, cdiv(s.S, kKeyTile) + 1);
   l.rmax = s.b * max_rows;
   const GemmPlan gl = plan_lmhead(s.V, s.b * s.B, s.Kw);
   l.lm_slots = gl.grid / gl.n_tiles;
-  l.acnt_n = acnt;
   l.status = take(256);
-  l.acnt = take((size_t)acnt * 4);
   l.x = take((size_t)l.rmax * s.d * 4);
   l.xb = take((size_t)l.rmax * s.d * 2);
   l.sumsq = take((size_t)l.rmax * (s.d / 128) * 4);
@@ -246,8 +227,6 @@ Layout layout(const Shape& s) {
   l.attn = take((size_t)l.rmax * s.Hq * s.D * 2);
   l.h = take((size_t)s.b * s.B * s.d * 2);
   l.stats = take((size_t)s.b * s.B * l.lm_slots * sizeof(LmStat));
-  l.part_o = take(std::max<size_t>(part_rows * s.D * 4, 256));
-  l.part_ml = take(std::max<size_t>(part_rows * 8, 256));
   l.conf = take((size_t)s.b * s.B * 4);
   l.tok = take((size_t)s.b * s.B * 4);
   l.gap = take((size_t)s.b * s.B * 4);
@@ -312,7 +291,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 // ------------------------------------------------------------------ launches
 dllm_status run_qkv(const Ctx& c, const void* wqkv, int layer, const void* xb,
                     const float* sumsq, int row0, int n_rows, const int* seq_start, void* q_out,
-                    void* kc, void* vc, bool pdl) {
+                    void* kc, void* vc, bool pdl, const L2Prefetch& pf = L2Prefetch{}) {
   const Shape& s = c.s;
   const int R = s.b * n_rows;
   const GemmPlan g = plan_gemm(s.qkv_rows, R, s.Kw, true);
@@ -348,11 +327,13 @@ dllm_status run_qkv(const Ctx& c, const void* wqkv, int layer, const void* xb,
   p.q_out = static_cast<__nv_bfloat16*>(q_out);
   p.k_cache = static_cast<__nv_bfloat16*>(kc);
   p.v_cache = static_cast<__nv_bfloat16*>(vc);
+  p.pf = pf;
   return cuda_status(launch_gemm(EPI_QKV, g.nt, wm, xm, p, g.grid, pdl, c.st));
 }
 
 dllm_status run_oproj(const Ctx& c, const void* wo, int layer, const void* attn, int row0,
-                      int n_rows, float* x, void* xb, float* sumsq, bool pdl) {
+                      int n_rows, float* x, void* xb, float* sumsq, bool pdl,
+                      const L2Prefetch& pf = L2Prefetch{}) {
   const Shape& s = c.s;
   const int R = s.b * n_rows;
   const GemmPlan g = plan_gemm(s.d, R, s.Ko, true);
@@ -380,6 +361,7 @@ dllm_status run_oproj(const Ctx& c, const void* wo, int layer, const void* attn,
   p.sumsq_out = sumsq;
   p.npart = s.d / 128;
   p.d_norm = s.d;
+  p.pf = pf;
   return cuda_status(launch_gemm(EPI_OPROJ, g.nt, wm, xm, p, g.grid, pdl, c.st));
 }
 
@@ -391,20 +373,10 @@ struct AttnKeys {
 
 dllm_status run_attn(const Ctx& c, int layer, int n_rows, const void* q, const void* kc,
                      const void* vc, const AttnKeys& keys, void* out, int ntile_bound,
-                     bool pdl) {
+                     bool pdl, const L2Prefetch& pf = L2Prefetch{}) {
   const Shape& s = c.s;
   const int g = s.Hq / s.Hkv;
-  AttnPlan a = plan_attn(s, n_rows, ntile_bound);
-  if (a.chunks > 1) {
-    // The partial buffers are sized for the decode row counts; larger row
-    // counts have enough (row tile) CTAs without splitting the keys.
-    const size_t need = (size_t)s.b * s.Hkv * a.row_tiles * a.chunks * 128;
-    const size_t have = (c.l.part_ml - c.l.part_o) / (4 * (size_t)s.D);
-    if (need > have || (size_t)s.b * s.Hkv * a.row_tiles > (size_t)c.l.acnt_n) {
-      a.chunks = 1;
-      a.tpc = ntile_bound;
-    }
-  }
+  const AttnPlan a = plan_attn(s, n_rows, ntile_bound);
   const int box_d = s.D >= 64 ? 64 : s.D;
   const CUtensorMapSwizzle sw = s.D >= 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   CUtensorMap qm, km, vm;
@@ -434,11 +406,9 @@ dllm_status run_attn(const Ctx& c, int layer, int n_rows, const void* q, const v
   p.dep_lo = keys.dep_lo;
   p.dep_hi = keys.dep_hi;
   p.out = static_cast<__nv_bfloat16*>(out);
-  p.part_o = c.at<float>(c.l.part_o);
-  p.part_ml = c.at<float2>(c.l.part_ml);
-  p.counters = c.at<int>(c.l.acnt);
   p.status = c.at<int>(c.l.status);
   p.scale_log2 = 1.4426950408889634f / sqrtf((float)s.D);
+  p.pf = pf;
   return cuda_status(launch_attn(s.D, qm, km, vm, p, pdl, c.st));
 }
 
@@ -472,20 +442,66 @@ dllm_status run_embed(const Ctx& c, const dllm_weights* w, const dllm_state* stt
   return cuda_status(launch_embed(e, pdl, c.st));
 }
 
-// Embed + L pre-norm layers for n_rows rows per sequence at row0.
+// How much of the weights that come next the layer stack pulls into L2 ahead
+// of use.  The attention kernel moves little data, so while it runs HBM
+// would idle: it can prefetch its own layer's W_o and the start of the next
+// weights (the next layer's W_qkv, or the LM head after the last layer);
+// the O-projection can prefetch a further part.  Off by default: on the
+// 8B-shaped stacks the projections' time goes to their ramp-up and tail, not
+// to the weight stream, and the extra traffic cost more than it saved.
+struct PrefetchTune {
+  long long attn_next = 0;
+  long long oproj_next = 0;
+  bool attn_wo = false;
+};
+PrefetchTune g_pf_tune;
+
+long long round16(long long v) { return v < 0 ? 0 : v & ~15ll; }
+
+// Embed + L pre-norm layers for n_rows rows per sequence at row0.  lm_next:
+// the LM head follows the last layer.
 dllm_status run_forward(const Ctx& c, const dllm_weights* w, const dllm_state* stt, int row0,
-                        int n_rows, int blk_start, int seg_end) {
+                        int n_rows, int blk_start, int seg_end, bool lm_next) {
   const Shape& s = c.s;
   DLLM_TRY(run_embed(c, w, stt, row0, n_rows, blk_start, seg_end, true));
   const int ntb = key_tiles_bound(s, blk_start, seg_end);
+  const long long qkv_bytes = (long long)s.qkv_rows * s.Kw * 2;
+  const long long wo_bytes = (long long)s.d * s.Ko * 2;
+  const auto* wqkv = static_cast<const uint8_t*>(w->wqkv);
+  const auto* wo = static_cast<const uint8_t*>(w->wo);
+  const PrefetchTune tune = g_pf_tune;
   for (int l = 0; l < s.L; ++l) {
+    const uint8_t* next = nullptr;
+    long long next_bytes = 0;
+    if (l + 1 < s.L) {
+      next = wqkv + (l + 1) * qkv_bytes;
+      next_bytes = qkv_bytes;
+    } else if (lm_next) {
+      next = static_cast<const uint8_t*>(w->w_lm);
+      next_bytes = (long long)s.V * s.Kw * 2;
+    }
+    const long long a = round16(std::min(tune.attn_next, next_bytes));
+    const long long o = round16(std::min(tune.oproj_next, next_bytes - a));
+    L2Prefetch pf_attn{}, pf_oproj{};
+    if (tune.attn_wo) {
+      pf_attn.ptr[0] = wo + l * wo_bytes;
+      pf_attn.bytes[0] = wo_bytes;
+    }
+    if (next && a > 0) {
+      pf_attn.ptr[1] = next;
+      pf_attn.bytes[1] = a;
+    }
+    if (next && o > 0) {
+      pf_oproj.ptr[0] = next + a;
+      pf_oproj.bytes[0] = o;
+    }
     DLLM_TRY(run_qkv(c, w->wqkv, l, c.at<void>(c.l.xb), c.at<float>(c.l.sumsq), row0, n_rows,
                      stt->seq_start, c.at<void>(c.l.q), stt->k_cache, stt->v_cache, true));
     const AttnKeys keys{nullptr, stt->seq_start, blk_start, seg_end, row0, row0 + n_rows};
     DLLM_TRY(run_attn(c, l, n_rows, c.at<void>(c.l.q), stt->k_cache, stt->v_cache, keys,
-                      c.at<void>(c.l.attn), ntb, true));
+                      c.at<void>(c.l.attn), ntb, true, pf_attn));
     DLLM_TRY(run_oproj(c, w->wo, l, c.at<void>(c.l.attn), row0, n_rows, c.at<float>(c.l.x),
-                       c.at<void>(c.l.xb), c.at<float>(c.l.sumsq), true));
+                       c.at<void>(c.l.xb), c.at<float>(c.l.sumsq), true, pf_oproj));
   }
   return DLLM_OK;
 }
@@ -581,7 +597,8 @@ dllm_status step(const Ctx& c, const dllm_weights* w, const dllm_state* st, int 
   if (!st->plants || !aligned16(st->plants)) return DLLM_ERR_INVALID;
   const int row0 = s.mode == DLLM_CACHE_NONE ? 0 : blk;
   const int n_rows = s.mode == DLLM_CACHE_NONE ? blk + s.B : s.B;
-  DLLM_TRY(run_forward(c, w, st, row0, n_rows, blk, s.mode == DLLM_CACHE_NONE ? blk + s.B : 0));
+  DLLM_TRY(run_forward(c, w, st, row0, n_rows, blk, s.mode == DLLM_CACHE_NONE ? blk + s.B : 0,
+                       true));
   DLLM_TRY(run_final_norm(c, c.at<float>(c.l.x), row0, n_rows, blk, st->masked, st->plants,
                           c.at<void>(c.l.h), true));
   DLLM_TRY(run_lmhead(c, w->w_lm, c.at<void>(c.l.h), s.b * s.B, true));
@@ -685,7 +702,7 @@ dllm_status refresh_graph(const Ctx& c, const dllm_config* cfg, const dllm_weigh
   if (c.s.mode == DLLM_CACHE_NONE) return DLLM_OK;
   const GraphKey key = make_key(cfg, w, st, ws, ws_bytes, kGraphRefresh, blk);
   return run_graph(c, key, [&](const Ctx& cc) {
-    return run_forward(cc, w, st, blk, cc.s.B, blk, 0);
+    return run_forward(cc, w, st, blk, cc.s.B, blk, 0, false);
   });
 }
 
@@ -706,7 +723,7 @@ dllm_status dllm_workspace_init(const dllm_config* cfg, void* ws, size_t ws_byte
                                 dllm_stream stream) {
   Ctx c;
   DLLM_TRY(make_ctx(cfg, ws, ws_bytes, stream, &c));
-  // status word, counters: zero
+  // status word: zero
   if (cudaMemsetAsync(c.ws, 0, c.l.x, c.st) != cudaSuccess) return DLLM_ERR_CUDA;
   if (c.s.theta > 0.f)
     return cuda_status(launch_rope_table(c.at<float2>(c.l.rope), c.s.S, c.s.D, c.s.theta, c.st));
@@ -872,7 +889,8 @@ dllm_status dllm_prefill(const dllm_config* cfg, const dllm_weights* w, const dl
   const int end = c.s.mode == DLLM_CACHE_PREFIX ? c.s.P : c.s.S;
   if (end < 1) return DLLM_OK;
   const GraphKey key = make_key(cfg, w, st, ws, ws_bytes, kGraphPrefill, 0);
-  return run_graph(c, key, [&](const Ctx& cc) { return run_forward(cc, w, st, 0, end, -1, end); });
+  return run_graph(c, key,
+                   [&](const Ctx& cc) { return run_forward(cc, w, st, 0, end, -1, end, false); });
 }
 
 dllm_status dllm_decode_step(const dllm_config* cfg, const dllm_weights* w, const dllm_state* st,
@@ -923,6 +941,16 @@ dllm_status dllm_decode_block(const dllm_config* cfg, const dllm_weights* w, con
   }
   if (steps_taken) *steps_taken = n;
   return refresh_graph(c, cfg, w, st, ws, ws_bytes, block_start);
+}
+
+dllm_status dllm_set_l2_prefetch(int64_t attn_next_bytes, int64_t oproj_next_bytes,
+                                 int32_t attn_prefetch_wo) {
+  if (attn_next_bytes < 0 || oproj_next_bytes < 0) return DLLM_ERR_INVALID;
+  g_pf_tune.attn_next = attn_next_bytes;
+  g_pf_tune.oproj_next = oproj_next_bytes;
+  g_pf_tune.attn_wo = attn_prefetch_wo != 0;
+  dllm_graph_cache_clear();  // cached graphs hold the old prefetch ranges
+  return DLLM_OK;
 }
 
 void dllm_graph_cache_clear(void) {

@@ -19,8 +19,11 @@
 // so for a decode step the prefix/suffix cache is already in flight while the
 // Q/K/V projection finishes.  Keys outside the sequence's segments are
 // masked inside the tile.  When a row tile is split over several key
-// chunks, each chunk writes an unnormalised partial (O, max, sum) and the
-// last chunk to finish merges them in chunk order.
+// chunks, the chunks run as one thread-block cluster: every CTA sends its
+// rows' (max, sum) to all others through distributed shared memory, scales
+// its O by its share of the merged softmax and sends each 16-column group to
+// the CTA that owns the group, which adds the chunks' contributions in chunk
+// order and writes the bf16 output.  No partial goes through global memory.
 #include <float.h>
 
 #include "kernels.cuh"
@@ -29,7 +32,7 @@
 namespace dllm {
 
 constexpr int kKeys = 128;     // keys per tile
-constexpr int kMaxMerge = 4;   // key chunks per row tile (the merge keeps them all in flight)
+constexpr int kMaxMerge = 4;   // key chunks (cluster size) per row tile
 
 // 2^x with the SFU instruction (relative error ~2^-22; P is rounded to bf16).
 DLLM_DEV float fast_exp2(float x) {
@@ -49,8 +52,26 @@ struct AttnCfg {
   static constexpr int kKVBytes = kKeys * D * 2;      // K or V tile
   static constexpr int kPBytes = 128 * kKeys * 2;     // two 128B-swizzle atom columns
   static constexpr int kTmemCols = 256;               // S [0,128), O [128,128+D)
-  static constexpr size_t kSmem = 1024 + kQBytes + ST * 2 * kKVBytes + kPBytes + 128 + 64;
+  static constexpr int kMlBytes = kMaxMerge * 128 * 8;  // (max, sum) of every chunk's rows
+  static constexpr size_t kSmem =
+      1024 + kQBytes + ST * 2 * kKVBytes + kPBytes + kMlBytes + 128 + 64;
+  // The merge reuses the K/V/P region once every chunk's last P V is done:
+  // [src chunk][owned group][4 float4][128 rows] fp32 for up to kMaxMerge chunks.
+  static constexpr int kGroups = D / 16;
+  static constexpr int kRegion = ST * 2 * kKVBytes + kPBytes;
 };
+
+template <int D>
+constexpr int merge_bytes(int n) {
+  return n * ((D / 16 + n - 1) / n) * 4 * 128 * 16;
+}
+static_assert(merge_bytes<128>(2) <= AttnCfg<128, 1>::kRegion &&
+                  merge_bytes<128>(3) <= AttnCfg<128, 1>::kRegion &&
+                  merge_bytes<128>(4) <= AttnCfg<128, 1>::kRegion &&
+                  merge_bytes<32>(2) <= AttnCfg<32, 1>::kRegion &&
+                  merge_bytes<32>(3) <= AttnCfg<32, 1>::kRegion &&
+                  merge_bytes<32>(4) <= AttnCfg<32, 1>::kRegion,
+              "the chunk merge buffer must fit in the K/V/P region");
 
 // Key segments (start, len) x 2 of sequence b: given explicitly, or derived
 // from the cache mode, the block and the sequence start.
@@ -138,7 +159,8 @@ __global__ void __launch_bounds__(128, 1)
   uint8_t* k_s = q_s + C::kQBytes;                 // [ST]
   uint8_t* v_s = k_s + ST * C::kKVBytes;           // [ST]
   uint8_t* p_s = v_s + ST * C::kKVBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(p_s + C::kPBytes);
+  float2* ml_s = reinterpret_cast<float2*>(p_s + C::kPBytes);  // [kMaxMerge][128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(p_s + C::kPBytes + C::kMlBytes);
   uint64_t* bar_q = bars;
   uint64_t* bar_s = bars + 1;
   uint64_t* bar_o = bars + 2;
@@ -209,6 +231,7 @@ __global__ void __launch_bounds__(128, 1)
       }
     }
   }
+  if (warp == 3) l2_prefetch_share(p.pf, blockIdx.x, gridDim.x, t - 96, 32);
   grid_dep_wait();
   if (p.segs != nullptr) seq_segments(p, b, sg);
   int t0, my_tiles;
@@ -276,13 +299,16 @@ __global__ void __launch_bounds__(128, 1)
 #pragma unroll
     for (int c = 0; c < kKeys / 32; ++c) tmem_ld32(s_tmem + lane_off + c * 32, s + c * 32);
     tmem_ld_wait();
-    float tmax = -FLT_MAX;
+    // independent partial maxima and sums: one warp per scheduler has no
+    // other work to hide a serial dependency chain behind
+    float tm[4] = {-FLT_MAX, -FLT_MAX, -FLT_MAX, -FLT_MAX};
 #pragma unroll
     for (int i = 0; i < kKeys; ++i)
-      if (i < nvalid) tmax = fmaxf(tmax, s[i]);
+      if (i < nvalid) tm[i & 3] = fmaxf(tm[i & 3], s[i]);
+    const float tmax = fmaxf(fmaxf(tm[0], tm[1]), fmaxf(tm[2], tm[3]));
     const float m_new = fmaxf(m_run, tmax * p.scale_log2);
     const float alpha = fast_exp2(m_run - m_new);
-    float lsum = 0.f;
+    float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int c = 0; c < kKeys / 8; ++c) {  // 8 keys = one 16-byte chunk of P
       uint32_t pk[4];
@@ -292,7 +318,7 @@ __global__ void __launch_bounds__(128, 1)
         const float p0 = k0 < nvalid ? fast_exp2(s[k0] * p.scale_log2 - m_new) : 0.f;
         const float p1 = k0 + 1 < nvalid ? fast_exp2(s[k0 + 1] * p.scale_log2 - m_new) : 0.f;
         const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-        lsum += __low2float(h2) + __high2float(h2);
+        ls[c & 3] += __low2float(h2) + __high2float(h2);
         pk[i >> 1] = *reinterpret_cast<const uint32_t*>(&h2);
       }
       // keys 64h..64h+63 form atom column h; row t holds 8 chunks of 16 bytes
@@ -314,7 +340,7 @@ __global__ void __launch_bounds__(128, 1)
       }
       tmem_st_wait();
     }
-    l_run = l_run * alpha + lsum;
+    l_run = l_run * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
     m_run = m_new;
     fence_proxy_async_smem();
     tc_fence_before();
@@ -375,8 +401,8 @@ __global__ void __launch_bounds__(128, 1)
     }
   };
 
-  if (ok) {
-    if (p.chunks == 1) {
+  if (p.chunks == 1) {
+    if (ok) {
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
 #pragma unroll
       for (int c = 0; c < D / 16; ++c) {
@@ -385,109 +411,73 @@ __global__ void __launch_bounds__(128, 1)
         tmem_ld_wait();
         if (row_ok && my_tiles > 0) store16(c * 16, v, inv);
       }
-    } else {
-      const size_t grp = ((size_t)(b * p.Hkv + kvh) * p.row_tiles + rt);
-      const size_t prow = (grp * p.chunks + chunk) * 128 + t;
+    }
+  } else {
+    // ---- merge of the key chunks inside the cluster (rank = chunk).  Every
+    // CTA reaches both cluster barriers, whatever happened before.
+    const int nch = p.chunks;
+    const uint32_t rank = (uint32_t)chunk;
+    const bool have = ok && my_tiles > 0 && l_run > 0.f;
+    const float2 mine = have ? make_float2(m_run, l_run) : make_float2(-FLT_MAX, 0.f);
+    const uint32_t ml_addr = smem_u32(&ml_s[rank * 128 + t]);
+    for (int q = 0; q < nch; ++q)
+      st_cluster_v2(map_to_rank(ml_addr, (uint32_t)q), mine.x, mine.y);
+    cluster_sync();  // (max, sum) everywhere; every chunk's P V is done
+    float mx = -FLT_MAX;
+    for (int c = 0; c < nch; ++c) {
+      const float2 e = ml_s[c * 128 + t];
+      if (e.y > 0.f) mx = fmaxf(mx, e.x);
+    }
+    float lt = 0.f;
+    for (int c = 0; c < nch; ++c) {
+      const float2 e = ml_s[c * 128 + t];
+      if (e.y > 0.f) lt += fast_exp2(e.x - mx) * e.y;
+    }
+    const float wmine = have && lt > 0.f ? fast_exp2(mine.x - mx) / lt : 0.f;
+    // groups of 16 columns are dealt round robin to the ranks; the owner's
+    // buffer is [src][owned group][4][128 rows] float4 over the K/V/P region
+    const int gpo = (C::kGroups + nch - 1) / nch;
+    float4* red = reinterpret_cast<float4*>(k_s);
+    const uint32_t red_addr = smem_u32(red);
 #pragma unroll
-      for (int c = 0; c < D / 16; ++c) {
+    for (int gi = 0; gi < C::kGroups; ++gi) {
+      float v[16];
+      tmem_ld16(o_tmem + lane_off + gi * 16, v);
+      tmem_ld_wait();
+      if (row_ok) {
+        const uint32_t owner = (uint32_t)(gi % nch);
+        const int lg = gi / nch;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int slot = ((int)(rank * gpo + lg) * 4 + q) * 128 + t;
+          const uint32_t dst = map_to_rank(red_addr + slot * 16, owner);
+          if (wmine != 0.f)
+            st_cluster_v4(dst, v[4 * q] * wmine, v[4 * q + 1] * wmine, v[4 * q + 2] * wmine,
+                          v[4 * q + 3] * wmine);
+          else
+            st_cluster_v4(dst, 0.f, 0.f, 0.f, 0.f);
+        }
+      }
+    }
+    cluster_sync();  // every contribution has landed
+    if (ok && row_ok) {
+      for (int lg = 0; lg < gpo; ++lg) {
+        const int gi = lg * nch + (int)rank;
+        if (gi >= C::kGroups) break;
         float v[16];
-        tmem_ld16(o_tmem + lane_off + c * 16, v);
-        tmem_ld_wait();
-        if (my_tiles == 0) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) v[i] = 0.f;
-        }
-        if (row_ok) {
-          float4* o4 = reinterpret_cast<float4*>(p.part_o + prow * D + c * 16);
+        for (int i = 0; i < 16; ++i) v[i] = 0.f;
+        for (int c = 0; c < nch; ++c) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            o4[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-        }
-      }
-      if (row_ok) p.part_ml[prow] = make_float2(m_run, l_run);
-      __threadfence();
-      __syncthreads();
-      if (t == 0) {
-        const int old = atomicAdd(&p.counters[grp], 1);
-        const int last = old == p.chunks - 1;
-        if (last) p.counters[grp] = 0;
-        flags[1] = last;
-      }
-      __syncthreads();
-      if (flags[1]) {
-        __threadfence();
-        // The tile's existing rows are spread over all 128 threads (up to 4
-        // threads per row); every chunk's partial of a 16-column group is
-        // requested before any of it is used.
-        const int nv_rows = min(128, p.group_rows - rt * 128);
-        // each thread owns a multiple of 16 columns (D/16 threads per row at most)
-        const int tpr = min(nv_rows <= 32 ? 4 : nv_rows <= 64 ? 2 : 1, D / 16);
-        const int row = t / tpr, part = t % tpr;
-        if (row < nv_rows) {
-          const size_t base_r = grp * p.chunks * 128 + row;  // + c * 128
-          float2 ml[kMaxMerge];
-#pragma unroll
-          for (int c = 0; c < kMaxMerge; ++c)
-            ml[c] = c < p.chunks ? __ldcg(&p.part_ml[base_r + (size_t)c * 128])
-                                 : make_float2(-FLT_MAX, 0.f);
-          float mx = -FLT_MAX;
-#pragma unroll
-          for (int c = 0; c < kMaxMerge; ++c)
-            if (ml[c].y > 0.f) mx = fmaxf(mx, ml[c].x);
-          float wgt[kMaxMerge], lt = 0.f;
-#pragma unroll
-          for (int c = 0; c < kMaxMerge; ++c) {
-            wgt[c] = ml[c].y > 0.f ? fast_exp2(ml[c].x - mx) : 0.f;
-            lt += wgt[c] * ml[c].y;
-          }
-          const float inv = lt > 0.f ? 1.f / lt : 0.f;
-          const int rr = rt * 128 + row;
-          const int hl2 = rr / p.n_rows;
-          const int ii2 = rr - hl2 * p.n_rows;
-          __nv_bfloat16* dst2 =
-              p.out + ((size_t)(b * p.n_rows + ii2) * p.Hq + (kvh * g + hl2)) * D;
-          const int ncol = D / tpr;
-          for (int d0 = part * ncol; d0 < (part + 1) * ncol; d0 += 16) {
-            float4 x[kMaxMerge][4];
-#pragma unroll
-            for (int c = 0; c < kMaxMerge; ++c) {
-              const float4* src = reinterpret_cast<const float4*>(
-                  p.part_o + (base_r + (size_t)c * 128) * D + d0);
-#pragma unroll
-              for (int q = 0; q < 4; ++q)
-                x[c][q] = c < p.chunks ? __ldcg(src + q) : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-            float v[16];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-              for (int c = 0; c < kMaxMerge; ++c) {
-                acc.x += wgt[c] * x[c][q].x;
-                acc.y += wgt[c] * x[c][q].y;
-                acc.z += wgt[c] * x[c][q].z;
-                acc.w += wgt[c] * x[c][q].w;
-              }
-              v[4 * q] = acc.x * inv;
-              v[4 * q + 1] = acc.y * inv;
-              v[4 * q + 2] = acc.z * inv;
-              v[4 * q + 3] = acc.w * inv;
-            }
-#pragma unroll
-            for (int q = 0; q < 16; q += 8) {
-              __nv_bfloat162 a0 = __floats2bfloat162_rn(v[q], v[q + 1]);
-              __nv_bfloat162 a1 = __floats2bfloat162_rn(v[q + 2], v[q + 3]);
-              __nv_bfloat162 a2 = __floats2bfloat162_rn(v[q + 4], v[q + 5]);
-              __nv_bfloat162 a3 = __floats2bfloat162_rn(v[q + 6], v[q + 7]);
-              uint4 wv;
-              wv.x = *reinterpret_cast<uint32_t*>(&a0);
-              wv.y = *reinterpret_cast<uint32_t*>(&a1);
-              wv.z = *reinterpret_cast<uint32_t*>(&a2);
-              wv.w = *reinterpret_cast<uint32_t*>(&a3);
-              *reinterpret_cast<uint4*>(dst2 + d0 + q) = wv;
-            }
+          for (int q = 0; q < 4; ++q) {
+            const float4 x = red[((c * gpo + lg) * 4 + q) * 128 + t];
+            v[4 * q] += x.x;
+            v[4 * q + 1] += x.y;
+            v[4 * q + 2] += x.z;
+            v[4 * q + 3] += x.w;
           }
         }
+        store16(gi * 16, v, 1.f);
       }
     }
   }
@@ -509,11 +499,22 @@ static cudaError_t launch_attn_t(const CUtensorMap& qmap, const CUtensorMap& kma
   cfg.blockDim = dim3(128);
   cfg.dynamicSmemBytes = AttnCfg<D, ST>::kSmem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  if (p.chunks > 1) {  // the chunks of a row tile merge through distributed shared memory
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = p.chunks;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
+  cfg.numAttrs = na;
   count_launch();
   return cudaLaunchKernelEx(&cfg, kern, qmap, kmap, vmap, p);
 }

@@ -350,6 +350,8 @@ __global__ void __launch_bounds__(192, NT <= 32 ? 3 : NT <= 64 ? 2 : 1)
         }
       }
     } else {
+      // lanes 1..31 warm L2 for a later kernel while the weights stream
+      l2_prefetch_share(p.pf, blockIdx.x, gridDim.x, lane - 1, 31);
       grid_dep_wait();
     }
     __syncwarp();

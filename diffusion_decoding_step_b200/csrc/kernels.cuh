@@ -19,6 +19,14 @@ struct __align__(16) LmStat {
   int idx;
 };
 
+// Bytes a later kernel of the sequence will read, fetched into L2 while
+// this kernel runs: ranges [ptr[i], ptr[i] + bytes[i]), split over the CTAs.
+// Nothing waits for them; a prefetch only warms the cache.
+struct L2Prefetch {
+  const uint8_t* ptr[2];
+  long long bytes[2];
+};
+
 struct GemmParams {
   // D^T[wrow][xrow] = sum_k W[layer][wrow][k] * X[xrow][k mod kx]
   int M;          // weight rows (multiple of 128)
@@ -49,6 +57,7 @@ struct GemmParams {
   // LM-head epilogue: stats[xrow][slot]
   LmStat* stats;
   int stat_slots;
+  L2Prefetch pf;
 };
 
 struct AttnParams {
@@ -56,19 +65,41 @@ struct AttnParams {
   int n_rows;       // query rows per sequence and head
   int group_rows;   // (Hq/Hkv) * n_rows
   int row_tiles;    // ceil(group_rows / 128)
-  int chunks;       // key chunks per (sequence, kv head, row tile)
+  int chunks;       // key chunks per (sequence, kv head, row tile) = cluster size
   int tiles_per_chunk;
   const int* segs;  // [b][2][2] (start, len), or null: derived from the fields below
   int mode, blk_start, blk_len, window, seg_end;
   const int* seq_start;
   int dep_lo, dep_hi;  // key positions the preceding kernel writes (load after the wait)
   __nv_bfloat16* out;  // [b*n_rows][Hq*D]
-  float* part_o;       // [b][Hkv][row_tiles][chunks][128][D]
-  float2* part_ml;     // [b][Hkv][row_tiles][chunks][128]
-  int* counters;       // [b][Hkv][row_tiles]
   int* status;
   float scale_log2;    // log2(e) / sqrt(D)
+  L2Prefetch pf;
 };
+
+#ifdef __CUDACC__
+// This CTA's share of a prefetch: the ranges are cut into 32 KB chunks, dealt
+// round robin over the CTAs and issued by `lanes` threads of the CTA.
+__device__ __forceinline__ void l2_prefetch_share(const L2Prefetch& pf, int cta, int ctas,
+                                                  int lane, int lanes) {
+  constexpr long long kChunk = 32768;
+  long long c0 = 0;  // chunks of the earlier ranges
+  for (int r = 0; r < 2; ++r) {
+    const long long nb = pf.bytes[r];
+    if (pf.ptr[r] == nullptr || nb <= 0) continue;
+    const long long nc = (nb + kChunk - 1) / kChunk;
+    const long long first = ((cta - c0) % ctas + ctas) % ctas;
+    for (long long i = first + (long long)lane * ctas; i < nc; i += (long long)lanes * ctas) {
+      const long long off = i * kChunk;
+      const long long n = nb - off < kChunk ? nb - off : kChunk;
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(pf.ptr[r] + off),
+                   "r"((uint32_t)n)
+                   : "memory");
+    }
+    c0 += nc;
+  }
+}
+#endif
 
 // Launch helpers (return cudaError_t of the launch).
 cudaError_t launch_gemm(int epi, int nt, const CUtensorMap& wmap, const CUtensorMap& xmap,

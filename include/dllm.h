@@ -241,6 +241,17 @@ uint64_t dllm_launch_count(void);
  * freeing buffers that a cached graph references, or to bound memory). */
 void dllm_graph_cache_clear(void);
 
+/* L2 prefetch of upcoming weights inside the layer stack (a tuning knob; no
+ * counterpart on the pages).  While layer l's attention runs, HBM has little
+ * to do: the attention kernel asks L2 for layer l's W_o (attn_prefetch_wo != 0)
+ * and the first attn_next_bytes of the weights read next (layer l+1's W_qkv,
+ * or the LM head after the last layer of a step); layer l's O-projection asks
+ * for the following oproj_next_bytes.  Only the cache is affected, never a
+ * result.  Process-wide; clears the graph cache.  Negative sizes are
+ * rejected (DLLM_ERR_INVALID).  Defaults: 0, 0, off. */
+dllm_status dllm_set_l2_prefetch(int64_t attn_next_bytes, int64_t oproj_next_bytes,
+                                 int32_t attn_prefetch_wo);
+
 const char* dllm_status_string(dllm_status s);
 
 #ifdef __cplusplus
