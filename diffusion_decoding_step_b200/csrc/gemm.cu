@@ -130,20 +130,28 @@ __device__ __forceinline__ void epi_prepare(const GemmParams& p, int n, int et, 
   }
 }
 
+// O-projection: the residual entries x[n*NT + c0 + i][m*128 + wl] a chunk
+// adds to.  The previous kernels are complete once the dependency wait has
+// returned, so these loads may run while the mainloop is still streaming.
+template <int NT>
+__device__ __forceinline__ void oproj_load_x(const GemmParams& p, int m, int n, int c0, int wl,
+                                             float (&xo)[16]) {
+  const int wrow = m * 128 + wl;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int xrow = n * NT + c0 + i;
+    xo[i] = xrow < p.R ? p.x[(size_t)xrow * p.d_model + wrow] : 0.f;
+  }
+}
+
 // Epilogue of one 16-column chunk; v[i] = D^T[m*128 + wl][n*NT + c0 + i].
+// xo: the O-projection's residual entries of the chunk (oproj_load_x).
 template <int NT, int EPI>
 __device__ __forceinline__ void epi_chunk(const GemmParams& p, int m, int n, int c0, int wl,
-                                          int et, const float (&v)[16], float* stage,
-                                          LmStat* run) {
+                                          int et, const float (&v)[16], const float (&xo)[16],
+                                          float* stage, LmStat* run) {
   if constexpr (EPI == EPI_OPROJ) {
     const int wrow = m * 128 + wl;
-    // all residual loads first: stores to x below would otherwise order them
-    float xo[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int xrow = n * NT + c0 + i;
-      xo[i] = xrow < p.R ? p.x[(size_t)xrow * p.d_model + wrow] : 0.f;
-    }
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const int xrow = n * NT + c0 + i;
@@ -272,6 +280,10 @@ __global__ void __launch_bounds__(192, NT <= 32 ? 3 : NT <= 64 ? 2 : 1)
   // Split K is reduced inside a thread-block cluster for decode tiles.
   constexpr bool kClusterSplit = NT <= 64;
   float part[kClusterSplit ? NT : 1];
+  // 16-column chunks of a split tile are dealt round robin to the cluster's
+  // ranks; at most kOwnMax per rank (splits >= 2)
+  constexpr int kOwnMax = kClusterSplit ? (NT / 16 + 1) / 2 : 1;
+  float xpre[kOwnMax][16];
   if (threadIdx.x == 0) {
     for (int s = 0; s < ST; ++s) {
       mbar_init(&full[s], 1);
@@ -418,6 +430,16 @@ __global__ void __launch_bounds__(192, NT <= 32 ? 3 : NT <= 64 ? 2 : 1)
       const uint32_t aph = (j >> 1) & 1;
       float* inv = reinterpret_cast<float*>(run);
       epi_prepare<NT, EPI>(p, n, et, inv, reinterpret_cast<int*>(inv + NT));
+      if constexpr (kClusterSplit && EPI == EPI_OPROJ) {
+        if (p.splits > 1) {  // residual rows of the chunks this rank will finish
+          const int rank = (int)cluster_ctarank();
+#pragma unroll
+          for (int lq = 0; lq < kOwnMax; ++lq) {
+            const int q = lq * p.splits + rank;
+            if (q < NT / 16) oproj_load_x<NT>(p, m, n, q * 16, wl, xpre[lq]);
+          }
+        }
+      }
       const bool bad = !mbar_wait(&tfull[acc], aph, p.status) || flags[0];
       if (named_bar_or(1, 128, bad)) {
         flags[0] = 1;
@@ -441,10 +463,11 @@ __global__ void __launch_bounds__(192, NT <= 32 ? 3 : NT <= 64 ? 2 : 1)
         }
       }
       for (int c0 = 0; c0 < NT; c0 += 16) {
-        float v[16];
+        float v[16], xo[16];
+        if constexpr (EPI == EPI_OPROJ) oproj_load_x<NT>(p, m, n, c0, wl, xo);
         tmem_ld16(tmem + ((uint32_t)lane_base << 16) + acc * NT + c0, v);
         tmem_ld_wait();
-        epi_chunk<NT, EPI>(p, m, n, c0, wl, et, v, stage, run);
+        epi_chunk<NT, EPI>(p, m, n, c0, wl, et, v, xo, stage, run);
       }
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
@@ -463,35 +486,58 @@ __global__ void __launch_bounds__(192, NT <= 32 ? 3 : NT <= 64 ? 2 : 1)
   if constexpr (kClusterSplit) {
     if (p.splits > 1) {
       // The splits of a tile form one cluster (one unit per CTA).  After
-      // every mainloop is done, ranks 1.. store their partial into rank 0's
-      // (now idle) stage buffers through distributed shared memory; rank 0
-      // adds them in rank order and runs the epilogue.
+      // every mainloop is done, the tile's 16-column chunks are dealt round
+      // robin to the ranks: each rank sends its partial of chunk q into the
+      // (now idle) stage buffers of rank q % splits through distributed
+      // shared memory, and every owner adds the partials of its chunks in
+      // rank order and runs their epilogue.
       cluster_sync();
-      const uint32_t rank = cluster_ctarank();
+      const int rank = (int)cluster_ctarank();
       const bool epi = warp >= 2;
       const int et = threadIdx.x - 64;
       const int wl = 32 * (warp & 3) + (threadIdx.x & 31);
-      float* red = reinterpret_cast<float*>(w_st);  // [rank-1][NT columns][128 lanes]
-      if (epi && rank != 0) {
-        const uint32_t dst = map_to_rank(smem_u32(red + (size_t)(rank - 1) * NT * 128 + wl), 0);
+      const int sp = p.splits;
+      const int own = (NT / 16 + sp - 1) / sp;  // chunk slots per owner
+      // [src rank][owned chunk][128 lanes][4 float4], float4 j at j ^ ((wl >> 1) & 3)
+      float* red = reinterpret_cast<float*>(w_st);
+      const int sw = (wl >> 1) & 3;
+      if (epi) {
 #pragma unroll
-        for (int c = 0; c < NT; ++c) st_cluster_f32(dst + c * 128 * 4, part[c]);
+        for (int q = 0; q < NT / 16; ++q) {
+          const uint32_t owner = (uint32_t)(q % sp);
+          const int lq = q / sp;
+          const uint32_t base = smem_u32(red + ((size_t)(rank * own + lq) * 128 + wl) * 16);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            st_cluster_v4(map_to_rank(base + ((j ^ sw) << 4), owner), part[q * 16 + 4 * j],
+                          part[q * 16 + 4 * j + 1], part[q * 16 + 4 * j + 2],
+                          part[q * 16 + 4 * j + 3]);
+        }
       }
       cluster_sync();
-      if (epi && rank == 0 && !flags[0]) {
+      if (epi && !flags[0]) {
         int m, n, tile, kb0, kb1;
         decode_unit(p, blockIdx.x, m, n, tile, kb0, kb1);
-        for (int r = 1; r < p.splits; ++r) {
-          const float* src = red + (size_t)(r - 1) * NT * 128 + wl;
 #pragma unroll
-          for (int c = 0; c < NT; ++c) part[c] += src[c * 128];
-        }
-#pragma unroll
-        for (int c0 = 0; c0 < NT; c0 += 16) {
+        for (int lq = 0; lq < kOwnMax; ++lq) {
+          const int q = lq * sp + rank;
+          if (q >= NT / 16) break;
           float v[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) v[i] = part[c0 + i];
-          epi_chunk<NT, EPI>(p, m, n, c0, wl, et, v, stage, run);
+          for (int i = 0; i < 16; ++i) v[i] = 0.f;
+          for (int r = 0; r < sp; ++r) {
+            const float4* src =
+                reinterpret_cast<const float4*>(red + ((size_t)(r * own + lq) * 128 + wl) * 16);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float4 x = src[j ^ sw];
+              v[4 * j] += x.x;
+              v[4 * j + 1] += x.y;
+              v[4 * j + 2] += x.z;
+              v[4 * j + 3] += x.w;
+            }
+          }
+          epi_chunk<NT, EPI>(p, m, n, q * 16, wl, et, v, xpre[lq], stage, run);
         }
       }
     }

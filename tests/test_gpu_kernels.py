@@ -184,13 +184,17 @@ OPROJ_CASES = [  # (hidden, Hq, D, batch, n_rows, block_start)
     (512, 8, 128, 16, 32, 0),
     (4096, 32, 128, 1, 512, 0),
     (4096, 32, 128, 1, 128, 0),
+    (4096, 32, 128, 2, 32, 256),   # 64-row tiles, K split over a 3-CTA cluster
+    (1024, 8, 128, 1, 48, 64),     # ragged 64-row tile, 3-CTA cluster
+    (8192, 64, 128, 1, 32, 0),     # 2-CTA cluster
 ]
 
 
 @pytest.mark.parametrize("d,Hq,D,b,nr,blk", OPROJ_CASES)
 def test_output_projection_residual(d, Hq, D, b, nr, blk):
     w = wl.Workload("t", batch=b, n_layers=2, hidden=d, n_q_heads=Hq, n_kv_heads=Hq, head_dim=D,
-                    vocab=1024, prompt_len=max(blk, 32), gen_len=max(nr, 32), block=32)
+                    vocab=1024, prompt_len=max(blk, 32), gen_len=max(32, -(-nr // 32) * 32),
+                    block=32)
     abi, cfg, ws, n = _ws(w)
     g = _gen(d + nr)
     Wo = (torch.randn(2, d, Hq * D, generator=g, device=DEV) * 0.02).to(torch.bfloat16)
