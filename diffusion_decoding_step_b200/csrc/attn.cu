@@ -193,7 +193,6 @@ __global__ void __launch_bounds__(128, 1)
     prefetch_tmap(&vmap);
   }
   __syncthreads();
-  grid_dep_launch();
 
   // Segments come from the sequence start (an input of the step) unless an
   // explicit list is given, which may be produced by earlier kernels.
@@ -439,21 +438,23 @@ __global__ void __launch_bounds__(128, 1)
     const int gpo = (C::kGroups + nch - 1) / nch;
     float4* red = reinterpret_cast<float4*>(k_s);
     const uint32_t red_addr = smem_u32(red);
+    // the whole O row is read from TMEM with one wait, then sent out
+    float o[D];
 #pragma unroll
-    for (int gi = 0; gi < C::kGroups; ++gi) {
-      float v[16];
-      tmem_ld16(o_tmem + lane_off + gi * 16, v);
-      tmem_ld_wait();
-      if (row_ok) {
+    for (int c = 0; c < D / 32; ++c) tmem_ld32(o_tmem + lane_off + c * 32, o + c * 32);
+    tmem_ld_wait();
+    if (row_ok) {
+#pragma unroll
+      for (int gi = 0; gi < C::kGroups; ++gi) {
         const uint32_t owner = (uint32_t)(gi % nch);
         const int lg = gi / nch;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int slot = ((int)(rank * gpo + lg) * 4 + q) * 128 + t;
           const uint32_t dst = map_to_rank(red_addr + slot * 16, owner);
+          const float* v = o + gi * 16 + 4 * q;
           if (wmine != 0.f)
-            st_cluster_v4(dst, v[4 * q] * wmine, v[4 * q + 1] * wmine, v[4 * q + 2] * wmine,
-                          v[4 * q + 3] * wmine);
+            st_cluster_v4(dst, v[0] * wmine, v[1] * wmine, v[2] * wmine, v[3] * wmine);
           else
             st_cluster_v4(dst, 0.f, 0.f, 0.f, 0.f);
         }
@@ -481,6 +482,9 @@ __global__ void __launch_bounds__(128, 1)
       }
     }
   }
+  // The next kernel is released only now: its CTAs, resident beside this
+  // one while they wait, slowed this kernel's softmax and merge measurably.
+  grid_dep_launch();
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {

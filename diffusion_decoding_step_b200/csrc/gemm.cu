@@ -26,12 +26,17 @@
 
 namespace dllm {
 
-template <int NT>
+template <int NT, int EPI>
 struct GemmCfg {
-  // Decode tiles (NT <= 64) keep the CTA near 70 KB of shared memory so that
-  // two CTAs of the next GEMM fit beside a running one and start streaming
-  // their weights before it finishes.
-  static constexpr int kStages = NT <= 64 ? 3 : 4;
+  // Bytes in flight per SM bound a weight stream: the LM head runs alone with
+  // one CTA per SM and a deep ring.  The O-projection keeps a ring small
+  // enough (about 90 KB) to sit beside the attention kernel it follows, so it
+  // can load weights before that kernel ends; the Q/K/V projection (two or
+  // three CTAs per SM) keeps about 70 KB per CTA so that two fit beside the
+  // O-projection before it.
+  static constexpr int kStages = EPI == EPI_LMHEAD ? (NT <= 64 ? 8 : NT <= 128 ? 6 : 4)
+                                 : EPI == EPI_OPROJ ? (NT <= 64 ? 4 : 4)
+                                                    : (NT <= 64 ? 3 : 4);
   static constexpr int kWBytes = 128 * 64 * 2;
   static constexpr int kXBytes = NT * 64 * 2;
   static constexpr int kTmemCols = 2 * NT;
@@ -39,6 +44,7 @@ struct GemmCfg {
   static constexpr size_t kSmem = 1024 + (size_t)kStages * (kWBytes + kXBytes) +
                                   kChunk * 128 * 4 + NT * sizeof(LmStat) +
                                   (2 * kStages + 4) * 8 + 64;
+  static_assert(kSmem <= 227 * 1024, "GEMM shared memory");
 };
 
 __device__ __forceinline__ void decode_unit(const GemmParams& p, int u, int& m, int& n, int& tile,
@@ -259,7 +265,7 @@ template <int NT, int EPI>
 __global__ void __launch_bounds__(192, NT <= 32 ? 3 : NT <= 64 ? 2 : 1)
     gemm_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap xmap,
                 const GemmParams p) {
-  using C = GemmCfg<NT>;
+  using C = GemmCfg<NT, EPI>;
   constexpr int ST = C::kStages;
   constexpr uint32_t kIdesc = idesc_bf16(128, NT, 0, 0);
   extern __shared__ uint8_t smem_raw[];
@@ -308,7 +314,6 @@ __global__ void __launch_bounds__(192, NT <= 32 ? 3 : NT <= 64 ? 2 : 1)
     prefetch_tmap(&xmap);
   }
   __syncthreads();
-  grid_dep_launch();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -483,6 +488,9 @@ __global__ void __launch_bounds__(192, NT <= 32 ? 3 : NT <= 64 ? 2 : 1)
     }
   }
   __syncthreads();
+  // Every mainloop of this CTA is done: the next kernel may start loading
+  // its weights during the reduction and epilogue below.
+  grid_dep_launch();
   if constexpr (kClusterSplit) {
     if (p.splits > 1) {
       // The splits of a tile form one cluster (one unit per CTA).  After
@@ -553,7 +561,7 @@ template <int NT, int EPI>
 static cudaError_t launch_t(const CUtensorMap& wmap, const CUtensorMap& xmap, const GemmParams& p,
                             int grid, bool pdl, cudaStream_t s) {
   auto kern = gemm_kernel<NT, EPI>;
-  const size_t smem = GemmCfg<NT>::kSmem;
+  const size_t smem = GemmCfg<NT, EPI>::kSmem;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(192);
@@ -587,7 +595,7 @@ cudaError_t gemm_prepare() {
 #define DLLM_SET(NT, EPI)                                                                      \
   if (e == cudaSuccess)                                                                       \
     e = cudaFuncSetAttribute(gemm_kernel<NT, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                             (int)GemmCfg<NT>::kSmem);
+                             (int)GemmCfg<NT, EPI>::kSmem);
   DLLM_SET(32, 0) DLLM_SET(32, 1) DLLM_SET(32, 2)
   DLLM_SET(64, 0) DLLM_SET(64, 1) DLLM_SET(64, 2)
   DLLM_SET(128, 0) DLLM_SET(128, 1) DLLM_SET(128, 2)
@@ -596,23 +604,6 @@ cudaError_t gemm_prepare() {
   return e;
 }
 
-int gemm_stages(int nt) {
-  switch (nt) {
-    case 32: return GemmCfg<32>::kStages;
-    case 64: return GemmCfg<64>::kStages;
-    case 128: return GemmCfg<128>::kStages;
-    default: return GemmCfg<256>::kStages;
-  }
-}
-
-size_t gemm_smem_bytes(int nt) {
-  switch (nt) {
-    case 32: return GemmCfg<32>::kSmem;
-    case 64: return GemmCfg<64>::kSmem;
-    case 128: return GemmCfg<128>::kSmem;
-    default: return GemmCfg<256>::kSmem;
-  }
-}
 
 template <int EPI>
 static cudaError_t launch_e(int nt, const CUtensorMap& wmap, const CUtensorMap& xmap,

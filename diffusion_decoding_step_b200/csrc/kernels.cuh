@@ -104,10 +104,8 @@ __device__ __forceinline__ void l2_prefetch_share(const L2Prefetch& pf, int cta,
 // Launch helpers (return cudaError_t of the launch).
 cudaError_t launch_gemm(int epi, int nt, const CUtensorMap& wmap, const CUtensorMap& xmap,
                         const GemmParams& p, int grid, bool pdl, cudaStream_t s);
-int gemm_stages(int nt);
 cudaError_t gemm_prepare();
 cudaError_t attn_prepare();
-size_t gemm_smem_bytes(int nt);
 
 cudaError_t launch_attn(int head_dim, const CUtensorMap& qmap, const CUtensorMap& kmap,
                         const CUtensorMap& vmap, const AttnParams& p, bool pdl,
