@@ -328,6 +328,7 @@ dllm_status run_qkv(const Ctx& c, const void* wqkv, int layer, const void* xb,
   p.k_cache = static_cast<__nv_bfloat16*>(kc);
   p.v_cache = static_cast<__nv_bfloat16*>(vc);
   p.pf = pf;
+  p.recv_in_ring = g.grid > kNumSMs;
   return cuda_status(launch_gemm(EPI_QKV, g.nt, wm, xm, p, g.grid, pdl, c.st));
 }
 
@@ -362,6 +363,7 @@ dllm_status run_oproj(const Ctx& c, const void* wo, int layer, const void* attn,
   p.npart = s.d / 128;
   p.d_norm = s.d;
   p.pf = pf;
+  p.recv_in_ring = g.grid > kNumSMs;
   return cuda_status(launch_gemm(EPI_OPROJ, g.nt, wm, xm, p, g.grid, pdl, c.st));
 }
 

@@ -165,7 +165,8 @@ __global__ void __launch_bounds__(128, 1)
   uint64_t* bar_s = bars + 1;
   uint64_t* bar_o = bars + 2;
   uint64_t* bar_kv = bars + 3;  // [ST]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 + ST);
+  uint64_t* dep_bar = bars + 3 + ST;  // thread 0 passes the dependency wait, the rest sleep
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4 + ST);
   volatile int* flags = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
   const int t = threadIdx.x;
@@ -185,6 +186,7 @@ __global__ void __launch_bounds__(128, 1)
     mbar_init(bar_s, 1);
     mbar_init(bar_o, 1);
     for (int s = 0; s < ST; ++s) mbar_init(&bar_kv[s], 1);
+    mbar_init(dep_bar, 1);
     flags[0] = 0;
     flags[1] = 0;
     fence_barrier_init();
@@ -231,7 +233,12 @@ __global__ void __launch_bounds__(128, 1)
     }
   }
   if (warp == 3) l2_prefetch_share(p.pf, blockIdx.x, gridDim.x, t - 96, 32);
-  grid_dep_wait();
+  if (t == 0) {
+    grid_dep_wait();
+    mbar_arrive(dep_bar);
+  } else {
+    mbar_wait_sleep(dep_bar, 0, p.status);
+  }
   if (p.segs != nullptr) seq_segments(p, b, sg);
   int t0, my_tiles;
   chunk_range(t0, my_tiles);

@@ -29,21 +29,31 @@ namespace dllm {
 template <int NT, int EPI>
 struct GemmCfg {
   // Bytes in flight per SM bound a weight stream: the LM head runs alone with
-  // one CTA per SM and a deep ring.  The O-projection keeps a ring small
-  // enough (about 90 KB) to sit beside the attention kernel it follows, so it
-  // can load weights before that kernel ends; the Q/K/V projection (two or
-  // three CTAs per SM) keeps about 70 KB per CTA so that two fit beside the
-  // O-projection before it.
+  // one CTA per SM and a deep ring.  The O-projection (one CTA per SM) takes
+  // four stages (about 90 KB), which still fits beside the attention kernel
+  // before it; the Q/K/V projection keeps about 70 KB per CTA so that it runs
+  // two or three CTAs per SM.  (Three O-projection stages, which would let
+  // two Q/K/V CTAs start beside it, measured slower.)
   static constexpr int kStages = EPI == EPI_LMHEAD ? (NT <= 64 ? 8 : NT <= 128 ? 6 : 4)
-                                 : EPI == EPI_OPROJ ? (NT <= 64 ? 4 : 4)
+                                 : EPI == EPI_OPROJ ? 4
                                                     : (NT <= 64 ? 3 : 4);
   static constexpr int kWBytes = 128 * 64 * 2;
   static constexpr int kXBytes = NT * 64 * 2;
   static constexpr int kTmemCols = 2 * NT;
   static constexpr int kChunk = 16;
-  static constexpr size_t kSmem = 1024 + (size_t)kStages * (kWBytes + kXBytes) +
-                                  kChunk * 128 * 4 + NT * sizeof(LmStat) +
-                                  (2 * kStages + 4) * 8 + 64;
+  // Split-K partials received from the other ranks of a cluster: [src slot
+  // (splits - 1)][owned chunk][128 lanes][16 fp32]; splits <= 4 for NT 32 and
+  // <= 3 for NT 64 (two owned chunks at most).
+  static constexpr int kRecvSlots = NT <= 32 ? 3 : 2;
+  static constexpr int kRecvOwn = NT <= 32 ? 1 : 2;
+  static constexpr int kRecvBytes =
+      (NT <= 64 && EPI != EPI_LMHEAD) ? kRecvSlots * kRecvOwn * 128 * 64 : 0;
+  // the receive buffer sits last, so a launch that keeps it in the (then
+  // idle) weight ring simply asks for kSmemBase bytes
+  static constexpr size_t kSmemBase = 1024 + (size_t)kStages * (kWBytes + kXBytes) +
+                                      kChunk * 128 * 4 + NT * sizeof(LmStat) +
+                                      (2 * kStages + 4) * 8 + 64;
+  static constexpr size_t kSmem = kSmemBase + kRecvBytes;
   static_assert(kSmem <= 227 * 1024, "GEMM shared memory");
 };
 
@@ -279,7 +289,16 @@ __global__ void __launch_bounds__(192, NT <= 32 ? 3 : NT <= 64 ? 2 : 1)
   uint64_t* empty = full + ST;
   uint64_t* tfull = empty + ST;
   uint64_t* tempty = tfull + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  // dep_bar: one thread passes the programmatic-dependency wait and releases
+  // the others through it (they sleep instead of polling beside the kernel
+  // still running on this SM)
+  uint64_t* dep_bar = tempty + 2;
+  uint64_t* red_bar = dep_bar + 1;  // split-K partials received from the cluster
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red_bar + 1);
+  // split-K receive buffer: its own region when the launch has one CTA per SM
+  // at most, else the weight ring once every mainloop of the cluster is done
+  float* recv = p.recv_in_ring ? reinterpret_cast<float*>(w_st)
+                               : reinterpret_cast<float*>(base + C::kSmemBase - 1024);
   volatile int* flags = reinterpret_cast<volatile int*>(tmem_slot + 2);  // [0] abort, [1] last
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -299,6 +318,8 @@ __global__ void __launch_bounds__(192, NT <= 32 ? 3 : NT <= 64 ? 2 : 1)
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], 128);
     }
+    mbar_init(dep_bar, 1);
+    mbar_init(red_bar, 1);
     flags[0] = 0;
     flags[1] = 0;
     fence_barrier_init();
@@ -314,6 +335,17 @@ __global__ void __launch_bounds__(192, NT <= 32 ? 3 : NT <= 64 ? 2 : 1)
     prefetch_tmap(&xmap);
   }
   __syncthreads();
+  if constexpr (kClusterSplit) {
+    if (p.splits > 1) {
+      // Owners of split-K chunks expect the other ranks' partials; the
+      // cluster barrier (waited for in the tail) publishes the armed barriers.
+      const int rank = (int)cluster_ctarank();
+      const int owned = (NT / 16 - rank + p.splits - 1) / p.splits;
+      if (threadIdx.x == 0 && owned > 0)
+        mbar_arrive_expect_tx(red_bar, (uint32_t)((p.splits - 1) * owned * 128 * 64));
+      cluster_arrive_relaxed();
+    }
+  }
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -335,6 +367,7 @@ __global__ void __launch_bounds__(192, NT <= 32 ? 3 : NT <= 64 ? 2 : 1)
         }
       }
       grid_dep_wait();
+      mbar_arrive(dep_bar);
       for (int i = 0; i < pre; ++i)
         tma_load_3d(x_st + i * C::kXBytes, &xmap, &full[i], ((pre_kb0 + i) % p.kx_blocks) * 64,
                     pre_n * NT, 0);
@@ -369,12 +402,11 @@ __global__ void __launch_bounds__(192, NT <= 32 ? 3 : NT <= 64 ? 2 : 1)
     } else {
       // lanes 1..31 warm L2 for a later kernel while the weights stream
       l2_prefetch_share(p.pf, blockIdx.x, gridDim.x, lane - 1, 31);
-      grid_dep_wait();
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    grid_dep_wait();
+    mbar_wait_sleep(dep_bar, 0, p.status);
     tmem_alloc(tmem_slot, C::kTmemCols);
     tc_fence_before();
     named_bar_sync(2, 160);
@@ -420,7 +452,7 @@ __global__ void __launch_bounds__(192, NT <= 32 ? 3 : NT <= 64 ? 2 : 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
-    grid_dep_wait();
+    mbar_wait_sleep(dep_bar, 0, p.status);
     named_bar_sync(2, 160);
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
@@ -493,61 +525,86 @@ __global__ void __launch_bounds__(192, NT <= 32 ? 3 : NT <= 64 ? 2 : 1)
   grid_dep_launch();
   if constexpr (kClusterSplit) {
     if (p.splits > 1) {
-      // The splits of a tile form one cluster (one unit per CTA).  After
-      // every mainloop is done, the tile's 16-column chunks are dealt round
-      // robin to the ranks: each rank sends its partial of chunk q into the
-      // (now idle) stage buffers of rank q % splits through distributed
-      // shared memory, and every owner adds the partials of its chunks in
-      // rank order and runs their epilogue.
-      cluster_sync();
+      // The splits of a tile form one cluster (one unit per CTA).  The tile's
+      // 16-column chunks are dealt round robin to the ranks; every rank sends
+      // its partial of each chunk it does not own to the owner's receive
+      // buffer with st.async (the bytes complete on the owner's red_bar), and
+      // each owner adds the partials of its chunks in rank order and runs
+      // their epilogue.  The final cluster barrier keeps every CTA alive
+      // until the transfers into it have landed.
+      cluster_wait();
+      if (p.recv_in_ring) {  // the owners' rings must be idle before they receive
+        cluster_arrive();
+        cluster_wait();
+      }
       const int rank = (int)cluster_ctarank();
       const bool epi = warp >= 2;
       const int et = threadIdx.x - 64;
       const int wl = 32 * (warp & 3) + (threadIdx.x & 31);
       const int sp = p.splits;
       const int own = (NT / 16 + sp - 1) / sp;  // chunk slots per owner
-      // [src rank][owned chunk][128 lanes][4 float4], float4 j at j ^ ((wl >> 1) & 3)
-      float* red = reinterpret_cast<float*>(w_st);
-      const int sw = (wl >> 1) & 3;
+      const int sw = (wl >> 1) & 3;              // float4 j of a lane sits at j ^ sw
       if (epi) {
 #pragma unroll
         for (int q = 0; q < NT / 16; ++q) {
-          const uint32_t owner = (uint32_t)(q % sp);
-          const int lq = q / sp;
-          const uint32_t base = smem_u32(red + ((size_t)(rank * own + lq) * 128 + wl) * 16);
+          const int owner = q % sp;
+          if (owner == rank) continue;
+          const int slot = rank < owner ? rank : rank - 1;
+          const uint32_t base =
+              smem_u32(recv + ((size_t)(slot * own + q / sp) * 128 + wl) * 16);
+          const uint32_t rbar = map_to_rank(smem_u32(red_bar), (uint32_t)owner);
 #pragma unroll
           for (int j = 0; j < 4; ++j)
-            st_cluster_v4(map_to_rank(base + ((j ^ sw) << 4), owner), part[q * 16 + 4 * j],
-                          part[q * 16 + 4 * j + 1], part[q * 16 + 4 * j + 2],
-                          part[q * 16 + 4 * j + 3]);
+            st_async_v4(map_to_rank(base + ((j ^ sw) << 4), (uint32_t)owner),
+                        part[q * 16 + 4 * j], part[q * 16 + 4 * j + 1],
+                        part[q * 16 + 4 * j + 2], part[q * 16 + 4 * j + 3], rbar);
         }
       }
-      cluster_sync();
-      if (epi && !flags[0]) {
-        int m, n, tile, kb0, kb1;
-        decode_unit(p, blockIdx.x, m, n, tile, kb0, kb1);
+      if (epi && rank < NT / 16) {
+        const bool got = mbar_wait_cluster(red_bar, 0, p.status);
+        cluster_arrive();
+        if (got && !flags[0]) {
+          int m, n, tile, kb0, kb1;
+          decode_unit(p, blockIdx.x, m, n, tile, kb0, kb1);
 #pragma unroll
-        for (int lq = 0; lq < kOwnMax; ++lq) {
-          const int q = lq * sp + rank;
-          if (q >= NT / 16) break;
-          float v[16];
+          for (int lq = 0; lq < kOwnMax; ++lq) {
+            const int q = lq * sp + rank;
+            if (q >= NT / 16) break;
+            float mine[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) v[i] = 0.f;
-          for (int r = 0; r < sp; ++r) {
-            const float4* src =
-                reinterpret_cast<const float4*>(red + ((size_t)(r * own + lq) * 128 + wl) * 16);
+            for (int qq = 0; qq < NT / 16; ++qq)
+              if (qq == q) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const float4 x = src[j ^ sw];
-              v[4 * j] += x.x;
-              v[4 * j + 1] += x.y;
-              v[4 * j + 2] += x.z;
-              v[4 * j + 3] += x.w;
+                for (int i = 0; i < 16; ++i) mine[i] = part[qq * 16 + i];
+              }
+            float v[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] = 0.f;
+            for (int r = 0; r < sp; ++r) {
+              if (r == rank) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[i] += mine[i];
+                continue;
+              }
+              const int slot = r < rank ? r : r - 1;
+              const float4* src = reinterpret_cast<const float4*>(
+                  recv + ((size_t)(slot * own + lq) * 128 + wl) * 16);
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const float4 x = src[j ^ sw];
+                v[4 * j] += x.x;
+                v[4 * j + 1] += x.y;
+                v[4 * j + 2] += x.z;
+                v[4 * j + 3] += x.w;
+              }
             }
+            epi_chunk<NT, EPI>(p, m, n, q * 16, wl, et, v, xpre[lq], stage, run);
           }
-          epi_chunk<NT, EPI>(p, m, n, q * 16, wl, et, v, xpre[lq], stage, run);
         }
+      } else {
+        cluster_arrive();
       }
+      cluster_wait();
     }
   }
   __syncthreads();
@@ -561,7 +618,7 @@ template <int NT, int EPI>
 static cudaError_t launch_t(const CUtensorMap& wmap, const CUtensorMap& xmap, const GemmParams& p,
                             int grid, bool pdl, cudaStream_t s) {
   auto kern = gemm_kernel<NT, EPI>;
-  const size_t smem = GemmCfg<NT, EPI>::kSmem;
+  const size_t smem = p.recv_in_ring ? GemmCfg<NT, EPI>::kSmemBase : GemmCfg<NT, EPI>::kSmem;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(192);
@@ -571,6 +628,9 @@ static cudaError_t launch_t(const CUtensorMap& wmap, const CUtensorMap& xmap, co
   int na = 0;
   if (p.splits > 1) {
     if (NT > 64 || grid != p.units) return cudaErrorInvalidValue;
+    if (p.recv_in_ring &&
+        (size_t)GemmCfg<NT, EPI>::kStages * GemmCfg<NT, EPI>::kWBytes < GemmCfg<NT, EPI>::kRecvBytes)
+      return cudaErrorInvalidValue;
     attr[na].id = cudaLaunchAttributeClusterDimension;
     attr[na].val.clusterDim.x = p.splits;
     attr[na].val.clusterDim.y = 1;

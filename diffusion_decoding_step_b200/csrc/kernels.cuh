@@ -57,6 +57,7 @@ struct GemmParams {
   // LM-head epilogue: stats[xrow][slot]
   LmStat* stats;
   int stat_slots;
+  int recv_in_ring;  // split K: partials go into the weight ring (grid > SM count)
   L2Prefetch pf;
 };
 

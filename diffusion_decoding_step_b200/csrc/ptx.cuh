@@ -53,6 +53,18 @@ DLLM_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// try_wait that lets the thread sleep up to hint_ns while the phase is open.
+DLLM_DEV bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
 // Wait for the phase with the given parity to complete.  Gives up after
 // kWaitLimitNs, sets kErrTimeout in *status and returns false.
 DLLM_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, int* status) {
@@ -61,6 +73,19 @@ DLLM_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, int* status) {
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 255u) == 0u && global_ns() - t0 > kWaitLimitNs) {
+      if (status) atomicOr(status, kErrTimeout);
+      return false;
+    }
+  }
+}
+
+// A long wait (for a preceding kernel): the thread sleeps between polls, so
+// a CTA started early beside a running kernel takes no issue slots from it.
+DLLM_DEV bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, int* status) {
+  const unsigned long long t0 = global_ns();
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+    if (global_ns() - t0 > kWaitLimitNs) {
       if (status) atomicOr(status, kErrTimeout);
       return false;
     }
@@ -195,6 +220,40 @@ DLLM_DEV uint32_t cluster_ctarank() {
 DLLM_DEV void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Split cluster barrier: arrive (no ordering) now, wait later.
+DLLM_DEV void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+DLLM_DEV void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+DLLM_DEV void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+// 16-byte store into another CTA's shared memory that completes its bytes
+// on that CTA's mbarrier (both addresses from map_to_rank).
+DLLM_DEV void st_async_v4(uint32_t addr, float a, float b, float c, float d, uint32_t bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::
+          "r"(addr),
+      "f"(a), "f"(b), "f"(c), "f"(d), "r"(bar)
+      : "memory");
+}
+// Bounded wait on a local mbarrier whose bytes come from other CTAs.
+DLLM_DEV bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, int* status) {
+  const unsigned long long t0 = global_ns();
+  for (uint32_t i = 0;; ++i) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    if (ok) return true;
+    if ((i & 255u) == 255u && global_ns() - t0 > kWaitLimitNs) {
+      if (status) atomicOr(status, kErrTimeout);
+      return false;
+    }
+  }
 }
 // Address of the same shared-memory offset in CTA `rank` of this cluster.
 DLLM_DEV uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
