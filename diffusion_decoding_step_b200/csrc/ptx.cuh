@@ -236,6 +236,13 @@ DLLM_DEV void st_async_v4(uint32_t addr, float a, float b, float c, float d, uin
       "f"(a), "f"(b), "f"(c), "f"(d), "r"(bar)
       : "memory");
 }
+DLLM_DEV void st_async_v2(uint32_t addr, float a, float b, uint32_t bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(
+          addr),
+      "f"(a), "f"(b), "r"(bar)
+      : "memory");
+}
 // Bounded wait on a local mbarrier whose bytes come from other CTAs.
 DLLM_DEV bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, int* status) {
   const unsigned long long t0 = global_ns();
