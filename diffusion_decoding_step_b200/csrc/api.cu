@@ -161,8 +161,8 @@ AttnPlan plan_attn(const Shape& s, int n_rows, int ntile_bound) {
   const int g = s.Hq / s.Hkv;
   a.row_tiles = cdiv(g * n_rows, 128);
   const int base = s.b * s.Hkv * a.row_tiles;
-  // at most 4 key chunks per row tile: the chunks form one cluster and merge on chip
-  int chunks = std::max(1, std::min({ntile_bound, cdiv(kNumSMs, base), 4}));
+  // at most 6 key chunks per row tile: the chunks form one cluster and merge on chip
+  int chunks = std::max(1, std::min({ntile_bound, cdiv(kNumSMs, base), 6}));
   if (base >= kNumSMs) chunks = 1;
   a.tpc = cdiv(ntile_bound, chunks);
   a.chunks = cdiv(ntile_bound, a.tpc);

@@ -32,7 +32,7 @@
 namespace dllm {
 
 constexpr int kKeys = 128;     // keys per tile
-constexpr int kMaxMerge = 4;   // key chunks (cluster size) per row tile
+constexpr int kMaxMerge = 6;   // key chunks (cluster size) per row tile
 
 // 2^x with the SFU instruction (relative error ~2^-22; P is rounded to bf16).
 DLLM_DEV float fast_exp2(float x) {
@@ -68,9 +68,13 @@ constexpr int merge_bytes(int n) {
 static_assert(merge_bytes<128>(2) <= AttnCfg<128, 1>::kRegion &&
                   merge_bytes<128>(3) <= AttnCfg<128, 1>::kRegion &&
                   merge_bytes<128>(4) <= AttnCfg<128, 1>::kRegion &&
+                  merge_bytes<128>(5) <= AttnCfg<128, 1>::kRegion &&
+                  merge_bytes<128>(6) <= AttnCfg<128, 1>::kRegion &&
                   merge_bytes<32>(2) <= AttnCfg<32, 1>::kRegion &&
                   merge_bytes<32>(3) <= AttnCfg<32, 1>::kRegion &&
-                  merge_bytes<32>(4) <= AttnCfg<32, 1>::kRegion,
+                  merge_bytes<32>(4) <= AttnCfg<32, 1>::kRegion &&
+                  merge_bytes<32>(5) <= AttnCfg<32, 1>::kRegion &&
+                  merge_bytes<32>(6) <= AttnCfg<32, 1>::kRegion,
               "the chunk merge buffer must fit in the K/V/P region");
 
 // Key segments (start, len) x 2 of sequence b: given explicitly, or derived

@@ -282,6 +282,9 @@ ATTN_CASES = [  # (Hq, Hkv, D, batch, n_rows, S, segs per sequence, layer)
     (8, 8, 128, 3, 32, 1280, [[(300, 980), (0, 0)], [(0, 1280), (0, 0)], [(512, 768), (0, 0)]], 1),
     (4, 2, 128, 1, 700, 700, [[(0, 700), (0, 0)]], 0),
     (32, 32, 128, 1, 512, 512, [[(0, 512), (0, 0)]], 1),   # prefill shape
+    (28, 4, 128, 1, 32, 640, [[(0, 544), (639, 1)]], 0),   # 6 key chunks
+    (28, 4, 128, 1, 32, 1024, [[(5, 539), (0, 0)]], 1),    # 5 chunks of 2 tiles
+    (8, 8, 32, 1, 16, 640, [[(0, 600), (0, 0)]], 0),       # head_dim 32, 6 chunks
 ]
 
 
