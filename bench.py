@@ -333,15 +333,22 @@ def run_ours(args, rank, world, local_rank):
     assert dec.device_status() == 0
     assert not bool(dec.masked.any())
 
-    # prefill share and per-step latency (separate untimed measurement)
+    # prefill share, decode-only rate and per-step latency (separate measurement)
     p0 = torch.cuda.Event(enable_timing=True)
     p1 = torch.cuda.Event(enable_timing=True)
+    p2 = torch.cuda.Event(enable_timing=True)
     dec.reset()
     p0.record(stream)
     dec.prefill()
     p1.record(stream)
+    for s_ in range(w.prompt_len, w.seq_len, w.block):
+        dec.decode_block(s_)
+    p2.record(stream)
     torch.cuda.synchronize(dev)
     prefill_ms = p0.elapsed_time(p1)
+    decode_ms = p1.elapsed_time(p2)
+    dec.reset()
+    dec.prefill()
     step_us = []
     s = w.prompt_len
     for _ in range(min(6, w.block)):
@@ -448,6 +455,10 @@ def run_ours(args, rank, world, local_rank):
                                "isolated_max": max(step_us)},
             "denoising_steps_per_generation": denoise_steps / args.steps,
             "prefill_ms": prefill_ms,
+            "decode_only": {"tokens_per_s": w.batch * w.gen_len / (decode_ms / 1000.0),
+                            "ms": decode_ms,
+                            "what": "committed tokens / decode time of one generation, "
+                                    "steps and block refreshes, prefill excluded"},
             "step_roofline": {"bound": "hbm", "algorithmic_bytes": step_bytes,
                               "isolated_p50_us": statistics.median(step_us),
                               "achieved": step_gbs, "peak": hbm, "unit": "GB/s",

@@ -128,3 +128,34 @@ def lockstep(dec, case, max_blocks: int | None = None, max_steps: int | None = N
             assert n <= cfg.block
         compare_refresh(dec, case, s)
     return rep
+
+
+def compare_step_sampled(dec, case, s: int, seqs, rep: Report) -> None:
+    """One GPU step of the whole batch, checked on the sequences `seqs` only:
+    the oracle recomputes each of them alone from its GPU state (sequences of
+    a batch are independent, which the oracle's own pins establish)."""
+    cfg1 = dataclasses.replace(case.cfg, batch=1)
+    refs = {}
+    for bi in seqs:
+        st = O.State(tokens=dec.tokens[bi:bi + 1].cpu().numpy().astype(np.int64),
+                     masked=dec.masked[bi:bi + 1].cpu().numpy().astype(bool),
+                     kcache=f64(dec.k_cache[:, bi:bi + 1]), vcache=f64(dec.v_cache[:, bi:bi + 1]),
+                     starts=dec.seq_start[bi:bi + 1].cpu().numpy().astype(np.int64))
+        refs[bi] = O.decode_step(cfg1, case.W, st, case.plants64[bi:bi + 1], s, apply=False)
+        del st
+    dec.step(s)
+    torch.cuda.synchronize()
+    assert dec.device_status() == 0
+    conf, tok, gap, commit = (t.cpu().numpy() for t in dec.step_outputs())
+    for bi, r in refs.items():
+        m = ~np.isnan(r.conf[0])
+        rep.rows += int(m.sum())
+        err = np.abs(conf[bi][m] - r.conf[0][m])
+        rep.max_conf_err = max(rep.max_conf_err, float(err.max()))
+        assert err.max() <= CONF_TOL, f"seq {bi}: conf error {err.max()}"
+        flag = r.amb_tok[0] | r.amb_commit[0]
+        rep.flagged += int(flag.sum())
+        bad = (m & (tok[bi] != r.tok[0])) | (commit[bi].astype(bool) != r.commit[0])
+        assert not (bad & ~flag).any(), f"seq {bi}: unflagged mismatch rows {np.where(bad & ~flag)[0]}"
+        rep.flagged_mismatch += int(bad.sum())
+    rep.steps += 1

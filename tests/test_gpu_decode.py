@@ -143,3 +143,34 @@ def test_full_size_first_steps_lockstep(name):
     for _ in range(2):
         compare_step(dec, case, w.prompt_len, rep, check_kv=False)
     assert rep.steps == 2
+
+
+# ---------------------------------------------------------------- full-size batches
+BATCHED = ["llada8b_dual_b16", "qwen7b_long_pruned"]
+
+
+@pytest.mark.parametrize("name", BATCHED)
+def test_full_size_batched_step_sampled_sequences(name):
+    """Batched full-size shapes (16 ragged LLaDA-8B-shaped sequences with
+    DualCache; 4 long Qwen-shaped sequences with the pruned suffix): prefill,
+    then one step of the first block on the GPU, the first and the last
+    sequence recomputed alone by the oracle from the GPU's state."""
+    from tests.lockstep import Report, compare_step_sampled
+    w = wl.WORKLOADS[name]
+    ensure_lib()
+    case = Case(w, device="cuda")
+    dec = make_decoder(case)
+    dec.prefill()
+    torch.cuda.synchronize()
+    assert dec.device_status() == 0
+    for l in (0, w.n_layers - 1):
+        assert bool(torch.isfinite(dec.k_cache[l]).all())
+        assert bool(torch.isfinite(dec.v_cache[l]).all())
+    rep = Report()
+    compare_step_sampled(dec, case, w.prompt_len, [0, w.batch - 1], rep)
+    assert rep.steps == 1 and rep.rows > 0
+    # every sequence committed at least one row and nothing outside the block
+    commit = dec.step_outputs()[3].cpu().numpy()
+    assert (commit.sum(1) >= 1).all()
+    masked = dec.masked.cpu().numpy()
+    assert masked[:, w.prompt_len + w.block:].all()
