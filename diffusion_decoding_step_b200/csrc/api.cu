@@ -144,6 +144,17 @@ GemmPlan plan_gemm(int M, int R, int K, bool allow_split) {
   return g;
 }
 
+// The same GEMM with K split into exactly sp parts (one unit per CTA).
+GemmPlan plan_gemm_splits(int M, int R, int K, int sp) {
+  GemmPlan g = plan_gemm(M, R, K, false);
+  const int kbt = K / 64;
+  g.kbps = cdiv(kbt, sp);
+  g.splits = cdiv(kbt, g.kbps);
+  g.units = g.m_tiles * g.n_tiles * g.splits;
+  g.grid = g.splits > 1 ? g.units : std::min(g.units, kNumSMs);
+  return g;
+}
+
 GemmPlan plan_lmhead(int V, int R, int K) {
   GemmPlan g = plan_gemm(V, R, K, false);
   int grid = std::min(g.units, kNumSMs);
@@ -294,7 +305,14 @@ dllm_status run_qkv(const Ctx& c, const void* wqkv, int layer, const void* xb,
                     void* kc, void* vc, bool pdl, const L2Prefetch& pf = L2Prefetch{}) {
   const Shape& s = c.s;
   const int R = s.b * n_rows;
-  const GemmPlan g = plan_gemm(s.qkv_rows, R, s.Kw, true);
+  GemmPlan g = plan_gemm(s.qkv_rows, R, s.Kw, true);
+  // More split CTAs than SMs start partly late (beside the O-projection
+  // still running); two splits on a deeper ring measured faster than three.
+  int epi = EPI_QKV;
+  if (g.nt <= 64 && g.splits > 2 && g.grid > kNumSMs) {
+    g = plan_gemm_splits(s.qkv_rows, R, s.Kw, 2);
+    epi = EPI_QKV_DEEP;
+  }
   CUtensorMap wm, xm;
   if (!make_map(&wm, wqkv, s.Kw, s.qkv_rows, s.L, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map(&xm, xb, s.d, R, 1, 64, g.nt, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -329,7 +347,7 @@ dllm_status run_qkv(const Ctx& c, const void* wqkv, int layer, const void* xb,
   p.v_cache = static_cast<__nv_bfloat16*>(vc);
   p.pf = pf;
   p.recv_in_ring = g.grid > kNumSMs;
-  return cuda_status(launch_gemm(EPI_QKV, g.nt, wm, xm, p, g.grid, pdl, c.st));
+  return cuda_status(launch_gemm(epi, g.nt, wm, xm, p, g.grid, pdl, c.st));
 }
 
 dllm_status run_oproj(const Ctx& c, const void* wo, int layer, const void* attn, int row0,

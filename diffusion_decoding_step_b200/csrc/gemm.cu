@@ -34,9 +34,10 @@ struct GemmCfg {
   // before it; the Q/K/V projection keeps about 70 KB per CTA so that it runs
   // two or three CTAs per SM.  (Three O-projection stages, which would let
   // two Q/K/V CTAs start beside it, measured slower.)
-  static constexpr int kStages = EPI == EPI_LMHEAD ? (NT <= 64 ? 8 : NT <= 128 ? 6 : 4)
-                                 : EPI == EPI_OPROJ ? 4
-                                                    : (NT <= 64 ? 3 : 4);
+  static constexpr int kStages = EPI == EPI_LMHEAD     ? (NT <= 64 ? 8 : NT <= 128 ? 6 : 4)
+                                 : EPI == EPI_OPROJ   ? 4
+                                 : EPI == EPI_QKV_DEEP ? 4
+                                                      : (NT <= 64 ? 3 : 4);
   static constexpr int kWBytes = 128 * 64 * 2;
   static constexpr int kXBytes = NT * 64 * 2;
   static constexpr int kTmemCols = 2 * NT;
@@ -277,6 +278,7 @@ __global__ void __launch_bounds__(192, NT <= 32 ? 3 : NT <= 64 ? 2 : 1)
                 const GemmParams p) {
   using C = GemmCfg<NT, EPI>;
   constexpr int ST = C::kStages;
+  constexpr int kEpi = EPI == EPI_QKV_DEEP ? EPI_QKV : EPI;  // epilogue kind
   constexpr uint32_t kIdesc = idesc_bf16(128, NT, 0, 0);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -466,8 +468,8 @@ __global__ void __launch_bounds__(192, NT <= 32 ? 3 : NT <= 64 ? 2 : 1)
       const int acc = j & 1;
       const uint32_t aph = (j >> 1) & 1;
       float* inv = reinterpret_cast<float*>(run);
-      epi_prepare<NT, EPI>(p, n, et, inv, reinterpret_cast<int*>(inv + NT));
-      if constexpr (kClusterSplit && EPI == EPI_OPROJ) {
+      epi_prepare<NT, kEpi>(p, n, et, inv, reinterpret_cast<int*>(inv + NT));
+      if constexpr (kClusterSplit && kEpi == EPI_OPROJ) {
         if (p.splits > 1) {  // residual rows of the chunks this rank will finish
           const int rank = (int)cluster_ctarank();
 #pragma unroll
@@ -501,15 +503,15 @@ __global__ void __launch_bounds__(192, NT <= 32 ? 3 : NT <= 64 ? 2 : 1)
       }
       for (int c0 = 0; c0 < NT; c0 += 16) {
         float v[16], xo[16];
-        if constexpr (EPI == EPI_OPROJ) oproj_load_x<NT>(p, m, n, c0, wl, xo);
+        if constexpr (kEpi == EPI_OPROJ) oproj_load_x<NT>(p, m, n, c0, wl, xo);
         tmem_ld16(tmem + ((uint32_t)lane_base << 16) + acc * NT + c0, v);
         tmem_ld_wait();
-        epi_chunk<NT, EPI>(p, m, n, c0, wl, et, v, xo, stage, run);
+        epi_chunk<NT, kEpi>(p, m, n, c0, wl, et, v, xo, stage, run);
       }
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
     }
-    if constexpr (EPI == EPI_LMHEAD) {
+    if constexpr (kEpi == EPI_LMHEAD) {
       named_bar_sync(1, 128);
       const int n = blockIdx.x % p.n_tiles;
       const int slot = blockIdx.x / p.n_tiles;
@@ -598,7 +600,7 @@ __global__ void __launch_bounds__(192, NT <= 32 ? 3 : NT <= 64 ? 2 : 1)
                 v[4 * j + 3] += x.w;
               }
             }
-            epi_chunk<NT, EPI>(p, m, n, q * 16, wl, et, v, xpre[lq], stage, run);
+            epi_chunk<NT, kEpi>(p, m, n, q * 16, wl, et, v, xpre[lq], stage, run);
           }
         }
       } else {
@@ -656,8 +658,8 @@ cudaError_t gemm_prepare() {
   if (e == cudaSuccess)                                                                       \
     e = cudaFuncSetAttribute(gemm_kernel<NT, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                              (int)GemmCfg<NT, EPI>::kSmem);
-  DLLM_SET(32, 0) DLLM_SET(32, 1) DLLM_SET(32, 2)
-  DLLM_SET(64, 0) DLLM_SET(64, 1) DLLM_SET(64, 2)
+  DLLM_SET(32, 0) DLLM_SET(32, 1) DLLM_SET(32, 2) DLLM_SET(32, 3)
+  DLLM_SET(64, 0) DLLM_SET(64, 1) DLLM_SET(64, 2) DLLM_SET(64, 3)
   DLLM_SET(128, 0) DLLM_SET(128, 1) DLLM_SET(128, 2)
   DLLM_SET(256, 0) DLLM_SET(256, 1) DLLM_SET(256, 2)
 #undef DLLM_SET
@@ -668,6 +670,13 @@ cudaError_t gemm_prepare() {
 template <int EPI>
 static cudaError_t launch_e(int nt, const CUtensorMap& wmap, const CUtensorMap& xmap,
                             const GemmParams& p, int grid, bool pdl, cudaStream_t s) {
+  if constexpr (EPI == EPI_QKV_DEEP) {
+    switch (nt) {
+      case 32: return launch_t<32, EPI>(wmap, xmap, p, grid, pdl, s);
+      case 64: return launch_t<64, EPI>(wmap, xmap, p, grid, pdl, s);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   switch (nt) {
     case 32: return launch_t<32, EPI>(wmap, xmap, p, grid, pdl, s);
     case 64: return launch_t<64, EPI>(wmap, xmap, p, grid, pdl, s);
@@ -683,6 +692,7 @@ cudaError_t launch_gemm(int epi, int nt, const CUtensorMap& wmap, const CUtensor
     case EPI_QKV: return launch_e<EPI_QKV>(nt, wmap, xmap, p, grid, pdl, s);
     case EPI_OPROJ: return launch_e<EPI_OPROJ>(nt, wmap, xmap, p, grid, pdl, s);
     case EPI_LMHEAD: return launch_e<EPI_LMHEAD>(nt, wmap, xmap, p, grid, pdl, s);
+    case EPI_QKV_DEEP: return launch_e<EPI_QKV_DEEP>(nt, wmap, xmap, p, grid, pdl, s);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -10,7 +10,9 @@ namespace dllm {
 
 constexpr int kNumSMs = 148;
 
-enum EpiKind : int { EPI_QKV = 0, EPI_OPROJ = 1, EPI_LMHEAD = 2 };
+// EPI_QKV_DEEP: the Q/K/V epilogue on a deeper weight ring (split tiles that
+// run two CTAs on some SMs)
+enum EpiKind : int { EPI_QKV = 0, EPI_OPROJ = 1, EPI_LMHEAD = 2, EPI_QKV_DEEP = 3 };
 
 // Running softmax statistics of a set of logits: max, sum of exp(l - max),
 // second largest (a tied maximum counts), index of the first maximum.
