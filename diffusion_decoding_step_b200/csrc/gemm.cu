@@ -5,8 +5,9 @@
 // rows per tile) and the activations the "B" operand (N = NT rows):
 //     D^T[wrow][xrow] = sum_k W[wrow][k] * X[xrow][k]
 // with both operands K-major in shared memory (128-byte swizzle, staged by
-// TMA) and the fp32 accumulator in TMEM.  A persistent CTA (one per SM) runs
-// three warp roles: warp 0 issues TMA loads through a STAGES-deep ring,
+// TMA) and the fp32 accumulator in TMEM.  A CTA (persistent over units when
+// K is not split) runs three warp roles: warp 0 issues TMA loads through a
+// ring of stages,
 // warp 1 issues the UMMAs, warps 2-5 drain TMEM (double-buffered
 // accumulator) and run one of three fused epilogues:
 //   EPI_QKV    RoPE on q/k, bf16 store of q and of k/v into the cache slots
@@ -14,10 +15,12 @@
 //   EPI_LMHEAD per-row running max / sum-exp / argmax / second max over the
 //              CTA's vocabulary tiles; logits never leave the SM
 // When (weight tiles x row tiles) would leave SMs idle, K is split: the
-// splits of a tile run as one thread-block cluster, one unit per CTA, and
-// their fp32 partials are summed in rank order in the shared memory of rank
-// 0 through distributed shared memory, so the result does not depend on
-// timing and no partial goes through global memory.
+// splits of a tile run as one thread-block cluster, one unit per CTA.  The
+// tile's 16-column chunks are dealt round robin to the ranks; each rank sends
+// its fp32 partials of the chunks it does not own to their owners with
+// st.async (completing on the owner's mbarrier), and every owner adds the
+// partials in rank order and runs the epilogue of its chunks.  The result
+// does not depend on timing and no partial goes through global memory.
 #include <float.h>
 #include <limits.h>
 
