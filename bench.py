@@ -220,7 +220,8 @@ def oracle_sample(w, weights, tokens, masked, starts, plants, budget_s=20.0):
     cfg = O.Config(batch=w.batch, n_layers=w.n_layers, hidden=w.hidden, n_q_heads=w.n_q_heads,
                    n_kv_heads=w.n_kv_heads, head_dim=w.head_dim, vocab=w.vocab,
                    prompt_len=w.prompt_len, gen_len=w.gen_len, block=w.block, tau=w.tau,
-                   mode=w.mode, window=w.window, rope_theta=w.rope_theta, mask_id=w.mask_id)
+                   mode=w.mode, window=w.window, rope_theta=w.rope_theta, mask_id=w.mask_id,
+                   commit_mode=w.commit_mode, steps_per_block=w.steps_per_block)
     W = O.Weights(lambda l: weights.wqkv[l].cpu().double().numpy(),
                   lambda l: weights.wo[l].cpu().double().numpy(),
                   weights.w_lm.cpu().double().numpy())

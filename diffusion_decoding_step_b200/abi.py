@@ -16,6 +16,7 @@ DLLM_OK, DLLM_ERR_INVALID, DLLM_ERR_UNSUPPORTED = 0, -1, -2
 DLLM_ERR_CUDA, DLLM_ERR_TIMEOUT, DLLM_ERR_WORKSPACE = -3, -4, -5
 DLLM_CACHE_NONE, DLLM_CACHE_PREFIX, DLLM_CACHE_DUAL, DLLM_CACHE_DUAL_PRUNED = 0, 1, 2, 3
 DLLM_W_BF16, DLLM_W_F32_SPLIT = 0, 1
+DLLM_COMMIT_THRESHOLD, DLLM_COMMIT_TOPK = 0, 1
 
 
 class DllmError(RuntimeError):
@@ -28,7 +29,8 @@ class dllm_config(C.Structure):
                 ("vocab", C.c_int32), ("prompt_len", C.c_int32), ("gen_len", C.c_int32),
                 ("block", C.c_int32), ("window", C.c_int32), ("mask_id", C.c_int32),
                 ("tau", C.c_float), ("rope_theta", C.c_float), ("mode", C.c_int32),
-                ("weight_format", C.c_int32)]
+                ("weight_format", C.c_int32), ("commit_mode", C.c_int32),
+                ("steps_per_block", C.c_int32)]
 
 
 class dllm_weights(C.Structure):

@@ -28,6 +28,7 @@ from typing import Optional
 import torch
 
 MODE_NONE, MODE_PREFIX, MODE_DUAL, MODE_DUAL_PRUNED = 0, 1, 2, 3
+COMMIT_THRESHOLD, COMMIT_TOPK = 0, 1  # conf > tau, or a fixed top-k budget per step
 MODE_NAMES = {MODE_NONE: "none", MODE_PREFIX: "prefix", MODE_DUAL: "dual",
               MODE_DUAL_PRUNED: "dual_pruned"}
 
@@ -57,6 +58,8 @@ class Workload:
     weight_f32: bool = False   # fp32 weights (tiny case) instead of bf16
     plant_a_max: float = 20.0
     prompt_len_min: Optional[int] = None  # ragged prompts: U[min, prompt_len]
+    commit_mode: int = COMMIT_THRESHOLD
+    steps_per_block: int = 0   # COMMIT_TOPK: a block is decoded in exactly this many steps
 
     def __post_init__(self):
         if self.mask_id < 0:

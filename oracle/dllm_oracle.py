@@ -53,6 +53,7 @@ from typing import Callable, Optional, Sequence
 import numpy as np
 
 MODE_NONE, MODE_PREFIX, MODE_DUAL, MODE_DUAL_PRUNED = 0, 1, 2, 3
+COMMIT_THRESHOLD, COMMIT_TOPK = 0, 1
 
 AMBIG_GAP = 1e-2     # top-2 logit gap below which an argmax is ambiguous
 AMBIG_CONF = 2e-3    # |conf - tau| (or forced-pick conf difference) band
@@ -174,6 +175,50 @@ def threshold_commit(conf: np.ndarray, masked: np.ndarray, tau: float) -> np.nda
     return commit
 
 
+def topk_budget(block: int, steps_per_block: int, n_masked: int) -> int:
+    """Rows a fixed-budget step commits (the low-confidence-remasking sampler).
+
+    Fast-dLLM's README sets the sampler's total steps (--steps) next to the
+    block length, and the Fast-dLLM overview page contrasts the cache plus
+    threshold with a standard diffusion sampler.  Plainest reading of that
+    sampler: a block of B masked positions is decoded in exactly S =
+    steps_per_block steps; step j (0-based) commits floor(B/S) rows, plus one
+    more while j < B mod S.  j is recovered from the rows already committed,
+    c = B - n_masked.  Never more than n_masked.
+    """
+    base, rem = divmod(block, steps_per_block)
+    c = block - n_masked
+    if c < rem * (base + 1):
+        j = c // (base + 1)
+    else:
+        j = rem + (c - rem * (base + 1)) // max(base, 1)
+    k = base + (1 if j < rem else 0)
+    return int(min(max(k, 1), n_masked))
+
+
+def topk_commit(conf: np.ndarray, masked: np.ndarray, k: int) -> np.ndarray:
+    """The k masked rows of highest confidence (lower position first on
+    equal confidence).  Returns a bool [B]."""
+    commit = np.zeros(masked.shape, dtype=bool)
+    idx = np.where(masked)[0]
+    order = sorted(idx, key=lambda i: (-conf[i], i))
+    commit[order[:k]] = True
+    return commit
+
+
+def topk_ambiguity(conf, masked, k):
+    """Top-k commit: the rows within AMBIG_CONF of the k-th / (k+1)-th
+    boundary may land on either side of it."""
+    amb = np.zeros(masked.shape, dtype=bool)
+    idx = np.where(masked)[0]
+    if 0 < k < len(idx):
+        c = np.sort(conf[idx])[::-1]
+        lo, hi = c[k], c[k - 1]
+        if hi - lo < AMBIG_CONF:
+            amb[idx[np.abs(conf[idx] - 0.5 * (hi + lo)) <= 0.5 * (hi - lo) + AMBIG_CONF]] = True
+    return amb
+
+
 def ambiguity_flags(conf, gap, masked, tau):
     """Rows whose outcome a correct implementation may decide either way.
 
@@ -214,6 +259,8 @@ class Config:
     window: int
     rope_theta: float
     mask_id: int
+    commit_mode: int = COMMIT_THRESHOLD
+    steps_per_block: int = 0
 
     @property
     def seq_len(self):
@@ -356,8 +403,9 @@ def decode_step(cfg: Config, W: Weights, st: State, plants: np.ndarray, s: int,
     """One denoising step of the block at [s, s+B).
 
     The block rows run through every layer (their keys/values overwrite the
-    cache at [s, s+B)), the LM head scores the masked rows, and the threshold
-    rule commits rows: tokens take the argmax, the mask bit goes to 0.
+    cache at [s, s+B)), the LM head scores the masked rows, and the commit
+    rule (threshold, or the fixed top-k budget) commits rows: tokens take the
+    argmax, the mask bit goes to 0.
     Without a cache (MODE_NONE) all positions [start, s+B) are recomputed.
     """
     B, b = cfg.block, cfg.batch
@@ -386,9 +434,15 @@ def decode_step(cfg: Config, W: Weights, st: State, plants: np.ndarray, s: int,
         if m.any():
             c, t, gp = lm_head_confidence(h[bi][m], W.w_lm())
             conf[bi, m], tok[bi, m], gap[bi, m] = c, t, gp
-            commit[bi] = threshold_commit(np.where(m, conf[bi], 0.0), m, cfg.tau)
-            amb_tok[bi], amb_commit[bi] = ambiguity_flags(
-                np.where(m, conf[bi], 0.0), gap[bi], m, cfg.tau)
+            cm = np.where(m, conf[bi], 0.0)
+            if cfg.commit_mode == COMMIT_TOPK:
+                k = topk_budget(B, cfg.steps_per_block, int(m.sum()))
+                commit[bi] = topk_commit(cm, m, k)
+                amb_tok[bi] = m & (gap[bi] < AMBIG_GAP)
+                amb_commit[bi] = topk_ambiguity(cm, m, k)
+            else:
+                commit[bi] = threshold_commit(cm, m, cfg.tau)
+                amb_tok[bi], amb_commit[bi] = ambiguity_flags(cm, gap[bi], m, cfg.tau)
         if apply:
             idx = np.where(commit[bi])[0]
             st.tokens[bi, s + idx] = tok[bi, idx]

@@ -13,7 +13,8 @@ def oracle_config(w: wl.Workload) -> O.Config:
                     n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads, head_dim=w.head_dim,
                     vocab=w.vocab, prompt_len=w.prompt_len, gen_len=w.gen_len,
                     block=w.block, tau=w.tau, mode=w.mode, window=w.window,
-                    rope_theta=w.rope_theta, mask_id=w.mask_id)
+                    rope_theta=w.rope_theta, mask_id=w.mask_id, commit_mode=w.commit_mode,
+                    steps_per_block=w.steps_per_block)
 
 
 def to64(t: torch.Tensor) -> np.ndarray:

@@ -416,3 +416,65 @@ def test_refresh_writes_committed_block_kv():
     k = (O.round_bf16(e) @ W.wqkv(0)[Hq * D:(Hq + Hkv) * D].T) * scale[:, None]
     want = O.round_bf16(k.reshape(w.block, Hkv, D).transpose(1, 0, 2))
     np.testing.assert_array_equal(st.kcache[0, 0][:, s:s + w.block], want)
+
+
+# ---------------------------------------------------------------- fixed-budget (top-k) commit
+def _schedule(B, S):
+    ks, m = [], B
+    while m:
+        k = O.topk_budget(B, S, m)
+        ks.append(k)
+        m -= k
+    return ks
+
+
+def test_topk_budget_spreads_the_block_over_the_steps():
+    assert _schedule(32, 5) == [7, 7, 6, 6, 6]
+    assert _schedule(32, 8) == [4] * 8
+    assert _schedule(32, 32) == [1] * 32
+    assert _schedule(32, 1) == [32]
+    assert _schedule(8, 3) == [3, 3, 2]
+    for B in (8, 32, 64):
+        for S in range(1, B + 1):
+            ks = _schedule(B, S)
+            assert len(ks) == S and sum(ks) == B and max(ks) - min(ks) <= 1
+
+
+def test_topk_commit_picks_the_most_confident_rows_lowest_position_first():
+    rng = np.random.default_rng(7)
+    for _ in range(200):
+        B = int(rng.integers(1, 65))
+        conf = np.round(rng.random(B), 1)            # coarse values: many ties
+        masked = rng.random(B) < 0.7
+        if not masked.any():
+            continue
+        k = int(rng.integers(1, masked.sum() + 1))
+        c = O.topk_commit(conf, masked, k)
+        assert c.sum() == k and not (c & ~masked).any()
+        # every committed row beats every masked row left out, (conf, -position) lexicographic
+        for i in np.where(c)[0]:
+            for j in np.where(masked & ~c)[0]:
+                assert conf[i] > conf[j] or (conf[i] == conf[j] and i < j)
+
+
+def test_topk_with_one_row_per_step_equals_tau_above_one():
+    w1 = TINY.replace(commit_mode=wl.COMMIT_TOPK, steps_per_block=TINY.block, gen_len=16)
+    w2 = TINY.replace(tau=1.5, gen_len=16)
+    t1, t2 = Case(w1).decode(), Case(w2).decode()
+    assert np.array_equal(t1.tokens, t2.tokens)
+    assert t1.steps_per_block == t2.steps_per_block == [TINY.block] * 2
+
+
+def test_topk_decode_takes_exactly_the_step_budget():
+    w = TINY.replace(commit_mode=wl.COMMIT_TOPK, steps_per_block=3, gen_len=16)
+    tr = Case(w).decode()
+    assert tr.steps_per_block == [3, 3]
+    per_step = [int(r.commit.sum()) for _, r in tr.steps]
+    assert per_step == [3, 3, 2, 3, 3, 2]
+    assert not (tr.tokens[:, w.prompt_len:] < 0).any()
+
+
+def test_topk_single_step_commits_the_whole_block():
+    w = TINY.replace(commit_mode=wl.COMMIT_TOPK, steps_per_block=1, gen_len=16)
+    tr = Case(w).decode()
+    assert tr.steps_per_block == [1, 1]
