@@ -38,6 +38,10 @@ def parse():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--commit", default="threshold", choices=["threshold", "topk"],
+                    help="commit rule: conf > tau (default) or a fixed top-k budget per step")
+    ap.add_argument("--steps-per-block", type=int, default=0,
+                    help="topk: steps a block takes (default block/4)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", action="store_true",
@@ -56,7 +60,7 @@ def run_profile(args):
     from diffusion_decoding_step_b200.runtime import Decoder
 
     build.build()
-    w = wl.WORKLOADS[args.workload]
+    w = selected_workload(args)
     if args.layers:
         w = w.replace(n_layers=args.layers)
     weights = wl.make_weights(w, device="cuda")
@@ -88,11 +92,22 @@ def peaks():
         return 6650.0, 1590.0, "fallback"
 
 
+def selected_workload(args):
+    from diffusion_decoding_step_b200 import workload as wl
+    w = wl.WORKLOADS[args.workload]
+    if args.commit == "topk":
+        w = w.replace(commit_mode=wl.COMMIT_TOPK,
+                      steps_per_block=args.steps_per_block or max(1, w.block // 4))
+    return w
+
+
 def workload_config(w, data_note):
     return {"workload": w.name, "batch": w.batch, "layers": w.n_layers, "hidden": w.hidden,
             "heads": f"{w.n_q_heads}/{w.n_kv_heads}x{w.head_dim}", "vocab": w.vocab,
             "prompt_len": w.prompt_len, "gen_len": w.gen_len, "block": w.block, "tau": w.tau,
             "cache": ["none", "prefix", "dual", "dual_pruned"][w.mode],
+            "commit": ("threshold" if w.commit_mode == 0
+                       else f"topk, {w.steps_per_block} steps per block"),
             "l2": data_note}
 
 
@@ -249,7 +264,7 @@ def run_reference(args, rank, world):
         return
     import torch
     from diffusion_decoding_step_b200 import workload as wl
-    w = wl.WORKLOADS[args.workload]
+    w = selected_workload(args)
     weights = wl.make_weights(w, device="cpu")
     tokens, masked = wl.make_tokens(w)
     starts = wl.seq_starts(w)
@@ -292,7 +307,7 @@ def run_ours(args, rank, world, local_rank):
     abi.lib()
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    w = wl.WORKLOADS[args.workload]
+    w = selected_workload(args)
     weights = wl.make_weights(w, device=dev)
     tokens, masked = wl.make_tokens(w)
     starts = wl.seq_starts(w)

@@ -54,7 +54,7 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_
 
 // ------------------------------------------------------------------ shapes
 struct Shape {
-  int b, L, d, Hq, Hkv, D, V, P, G, B, S, W, mode, wfmt;
+  int b, L, d, Hq, Hkv, D, V, P, G, B, S, W, mode, wfmt, commit_mode, spb;
   int qkv_rows, Kw, Ko;
   float tau, theta;
   int mask_id;
@@ -73,6 +73,11 @@ dllm_status check_cfg(const dllm_config* c, Shape* s) {
   if (c->gen_len % c->block) return DLLM_ERR_INVALID;
   if (c->mode == DLLM_CACHE_DUAL_PRUNED && c->window < 0) return DLLM_ERR_INVALID;
   if (c->mask_id < 0 || c->mask_id >= c->vocab) return DLLM_ERR_INVALID;
+  if (c->commit_mode != DLLM_COMMIT_THRESHOLD && c->commit_mode != DLLM_COMMIT_TOPK)
+    return DLLM_ERR_INVALID;
+  if (c->commit_mode == DLLM_COMMIT_TOPK &&
+      (c->steps_per_block < 1 || c->steps_per_block > c->block))
+    return DLLM_ERR_INVALID;
   if (!(c->tau == c->tau) || c->rope_theta < 0.f) return DLLM_ERR_INVALID;
   if (c->head_dim != 32 && c->head_dim != 128) return DLLM_ERR_UNSUPPORTED;
   const int qkv = (c->n_q_heads + 2 * c->n_kv_heads) * c->head_dim;
@@ -93,6 +98,8 @@ dllm_status check_cfg(const dllm_config* c, Shape* s) {
   s->W = c->window;
   s->mode = c->mode;
   s->wfmt = c->weight_format;
+  s->commit_mode = c->commit_mode;
+  s->spb = c->commit_mode == DLLM_COMMIT_TOPK ? c->steps_per_block : 0;
   s->qkv_rows = qkv;
   const int f = c->weight_format == DLLM_W_F32_SPLIT ? 2 : 1;
   s->Kw = f * c->hidden;
@@ -593,6 +600,8 @@ dllm_status run_commit(const Ctx& c, const dllm_state* stt, int blk_start, bool 
   p.commit = c.at<uint8_t>(c.l.commit);
   p.remaining = c.at<int>(c.l.remaining);
   p.do_commit = 1;
+  p.topk = s.commit_mode == DLLM_COMMIT_TOPK;
+  p.steps_per_block = s.spb;
   return cuda_status(launch_commit(p, pdl, c.st));
 }
 
@@ -897,6 +906,8 @@ dllm_status dllm_threshold_commit(const dllm_config* cfg, int32_t block_start, c
   p.commit = commit;
   p.remaining = remaining;
   p.do_commit = 1;
+  p.topk = s.commit_mode == DLLM_COMMIT_TOPK;
+  p.steps_per_block = s.spb;
   return cuda_status(launch_commit(p, false, reinterpret_cast<cudaStream_t>(stream)));
 }
 

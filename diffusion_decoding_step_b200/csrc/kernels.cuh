@@ -156,6 +156,8 @@ struct CommitParams {
   uint8_t* commit;
   int* remaining;
   int do_commit;
+  int topk;             // fixed-budget rule instead of the threshold
+  int steps_per_block;  // topk: steps a block takes
 };
 cudaError_t launch_commit(const CommitParams& p, bool pdl, cudaStream_t s);
 

@@ -258,8 +258,34 @@ __global__ void __launch_bounds__(1024) commit_kernel(const CommitParams p) {
     }
   }
   const bool any_masked = bc >= 0.f;
-  const bool k0 = m0 && (c0 > p.tau || (any_masked && bi == i0));
-  const bool k1 = m1 && (c1 > p.tau || (any_masked && bi == i1));
+  bool k0, k1;
+  if (p.topk) {
+    // fixed budget: this step's share of the block, then the rows whose rank
+    // (masked rows ahead of them: higher conf, or equal conf and lower
+    // position) is below it
+    const int nm = __popc(__ballot_sync(0xffffffffu, m0)) + __popc(__ballot_sync(0xffffffffu, m1));
+    const int base = p.B / p.steps_per_block, rem = p.B % p.steps_per_block;
+    const int done = p.B - nm;
+    const int j = done < rem * (base + 1) ? done / (base + 1)
+                                          : rem + (done - rem * (base + 1)) / max(base, 1);
+    const int k = min(max(base + (j < rem ? 1 : 0), 1), nm);
+    __shared__ float s_mc[64];  // conf of masked rows, -1 elsewhere
+    if (i0 < p.B) s_mc[i0] = c0;
+    if (i1 < p.B) s_mc[i1] = c1;
+    __syncwarp();
+    int r0 = 0, r1 = 0;
+    for (int q = 0; q < p.B; ++q) {
+      const float cq = s_mc[q];
+      if (cq < 0.f) continue;
+      r0 += (cq > c0 || (cq == c0 && q < i0)) ? 1 : 0;
+      r1 += (cq > c1 || (cq == c1 && q < i1)) ? 1 : 0;
+    }
+    k0 = m0 && r0 < k;
+    k1 = m1 && r1 < k;
+  } else {
+    k0 = m0 && (c0 > p.tau || (any_masked && bi == i0));
+    k1 = m1 && (c1 > p.tau || (any_masked && bi == i1));
+  }
   if (k0) {
     p.tokens[base + i0] = s_tok[i0];
     p.masked[base + i0] = 0;

@@ -73,6 +73,18 @@ typedef enum {
  * 2^-17 relative, and the embedding stays fp32. */
 typedef enum { DLLM_W_BF16 = 0, DLLM_W_F32_SPLIT = 1 } dllm_weight_format;
 
+/* Commit rule of a step (Fast-dLLM overview page, "The v1 Mechanism": the
+ * confidence-threshold rule; Fast-dLLM README, "Quick Start": the sampler's
+ * --steps knob next to the block length).
+ *   THRESHOLD  every masked row with conf > tau, and at least the most
+ *              confident masked row (lowest position on ties).
+ *   TOPK       a fixed budget: a block is decoded in exactly steps_per_block
+ *              steps; step j commits floor(B/steps) + [j < B mod steps] of
+ *              the most confident masked rows (lower position first on
+ *              equal confidence), j being inferred from the rows already
+ *              committed.  tau is not used. */
+typedef enum { DLLM_COMMIT_THRESHOLD = 0, DLLM_COMMIT_TOPK = 1 } dllm_commit_mode;
+
 typedef struct {
   int32_t batch, n_layers, hidden, n_q_heads, n_kv_heads, head_dim, vocab;
   int32_t prompt_len; /* P: longest prompt; shorter prompts are left-padded */
@@ -81,6 +93,8 @@ typedef struct {
   float rope_theta; /* rotate-half RoPE base; 0 disables RoPE */
   int32_t mode;          /* dllm_cache_mode */
   int32_t weight_format; /* dllm_weight_format */
+  int32_t commit_mode;   /* dllm_commit_mode */
+  int32_t steps_per_block; /* TOPK: 1 <= steps_per_block <= block; ignored otherwise */
 } dllm_config;
 
 /* Kw = hidden (BF16) or 2*hidden (F32_SPLIT); Ko = Hq*D or 2*Hq*D. */

@@ -174,3 +174,35 @@ def test_full_size_batched_step_sampled_sequences(name):
     assert (commit.sum(1) >= 1).all()
     masked = dec.masked.cpu().numpy()
     assert masked[:, w.prompt_len + w.block:].all()
+
+
+
+# ---------------------------------------------------------------- fixed-budget commits
+TOPK = {
+    "tiny_prefix_topk": TINY.replace(commit_mode=wl.COMMIT_TOPK, steps_per_block=3),
+    "llada_mid_dual_topk": MID["llada_mid_dual"].replace(commit_mode=wl.COMMIT_TOPK,
+                                                         steps_per_block=5),
+}
+
+
+@pytest.mark.parametrize("name", list(TOPK))
+def test_lockstep_decode_topk(name):
+    """The fixed-budget rule in lockstep with the oracle; every block takes
+    exactly steps_per_block steps."""
+    w = TOPK[name]
+    case = Case(w)
+    dec = make_decoder(case)
+    rep = lockstep(dec, case)
+    assert rep.steps == (w.gen_len // w.block) * w.steps_per_block
+    assert rep.flagged_mismatch <= max(2, rep.rows // 50)
+    assert not dec.masked.any()
+
+
+def test_decode_block_topk_takes_the_step_budget():
+    w = TOPK["llada_mid_dual_topk"]
+    case = Case(w)
+    dec = make_decoder(case)
+    steps = dec.generate()
+    torch.cuda.synchronize()
+    assert steps == [w.steps_per_block] * (w.gen_len // w.block)
+    assert not dec.masked.any()

@@ -359,3 +359,45 @@ def test_threshold_commit_bit_exact(b, B, tau):
         assert np.array_equal(t_tokens[bi].cpu().numpy(), want_tok)
         assert np.array_equal(t_masked[bi].cpu().numpy(), want_mask)
         assert int(remaining[bi]) == int(m.sum() - c_ref.sum())
+
+
+@pytest.mark.parametrize("b,B,spb,done", [(1, 8, 3, 0), (1, 32, 5, 14), (16, 32, 8, 0),
+                                          (4, 64, 7, 19), (3, 32, 32, 31), (2, 32, 1, 0)])
+def test_topk_commit_bit_exact(b, B, spb, done):
+    """Fixed-budget rule: every sequence commits its step's share of the
+    block (from the rows it has committed so far), by confidence, lower
+    position first on ties."""
+    w = wl.Workload("t", batch=b, n_layers=1, hidden=128, n_q_heads=4, n_kv_heads=4,
+                    head_dim=32, vocab=1024, prompt_len=64, gen_len=2 * B, block=B,
+                    commit_mode=wl.COMMIT_TOPK, steps_per_block=spb)
+    abi = ensure_lib()
+    cfg = make_config(w)
+    rng = np.random.default_rng(b * 1000 + B + spb)
+    S = w.seq_len
+    s = w.prompt_len + B
+    conf = np.round(rng.uniform(0, 1, (b, B)), 2).astype(np.float32)   # many ties
+    masked = np.zeros((b, S), dtype=np.uint8)
+    for bi in range(b):
+        left = rng.permutation(B)[:B - done] if bi % 2 == 0 else rng.permutation(B)[:max(1, B - done - bi)]
+        masked[bi, s + left] = 1
+    tok = rng.integers(0, 1024, (b, B)).astype(np.int32)
+    tokens = rng.integers(0, 1024, (b, S)).astype(np.int32)
+    t_tokens = torch.tensor(tokens, device=DEV)
+    t_masked = torch.tensor(masked, device=DEV)
+    commit = torch.zeros(b, B, dtype=torch.uint8, device=DEV)
+    remaining = torch.zeros(b, dtype=torch.int32, device=DEV)
+    t_conf = torch.tensor(conf, device=DEV)
+    t_tok = torch.tensor(tok, device=DEV)
+    abi.check(abi.dllm_threshold_commit(C.byref(cfg), s, ptr(t_conf), ptr(t_tok), ptr(t_tokens),
+                                        ptr(t_masked), ptr(commit), ptr(remaining), stream()),
+              "commit")
+    torch.cuda.synchronize()
+    for bi in range(b):
+        m = masked[bi, s:s + B].astype(bool)
+        k = O.topk_budget(B, spb, int(m.sum()))
+        c_ref = O.topk_commit(conf[bi].astype(np.float64), m, k)
+        assert np.array_equal(commit[bi].cpu().numpy().astype(bool), c_ref), f"seq {bi}"
+        want_tok = tokens[bi].copy()
+        want_tok[s:s + B][c_ref] = tok[bi][c_ref]
+        assert np.array_equal(t_tokens[bi].cpu().numpy(), want_tok)
+        assert int(remaining[bi]) == int(m.sum() - c_ref.sum())
