@@ -66,6 +66,18 @@ def test_rejects_bad_configs(lib):
     assert abi.dllm_workspace_size(None, None) == abi.DLLM_ERR_INVALID
 
 
+def test_commit_mode_validation(lib):
+    base = wl.WORKLOADS["tiny"]
+    topk = base.replace(commit_mode=wl.COMMIT_TOPK)
+    assert _status(topk.replace(steps_per_block=1)) == abi.DLLM_OK
+    assert _status(topk.replace(steps_per_block=base.block)) == abi.DLLM_OK
+    assert _status(topk.replace(steps_per_block=0)) == abi.DLLM_ERR_INVALID
+    assert _status(topk.replace(steps_per_block=base.block + 1)) == abi.DLLM_ERR_INVALID
+    assert _status(base.replace(commit_mode=2)) == abi.DLLM_ERR_INVALID
+    # the threshold rule ignores steps_per_block
+    assert _status(base.replace(steps_per_block=-3)) == abi.DLLM_OK
+
+
 def test_null_pointers_rejected_before_launch(lib):
     cfg = make_config(wl.WORKLOADS["tiny"])
     n = C.c_size_t(0)
