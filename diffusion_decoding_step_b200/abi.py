@@ -17,6 +17,7 @@ DLLM_ERR_CUDA, DLLM_ERR_TIMEOUT, DLLM_ERR_WORKSPACE = -3, -4, -5
 DLLM_CACHE_NONE, DLLM_CACHE_PREFIX, DLLM_CACHE_DUAL, DLLM_CACHE_DUAL_PRUNED = 0, 1, 2, 3
 DLLM_W_BF16, DLLM_W_F32_SPLIT = 0, 1
 DLLM_COMMIT_THRESHOLD, DLLM_COMMIT_TOPK = 0, 1
+DLLM_DEVICE_TIMEOUT = 1  # status-word bit of a device wait that gave up
 
 
 class DllmError(RuntimeError):
@@ -75,6 +76,7 @@ SIGNATURES = {
     "dllm_launch_count": (C.c_uint64, []),
     "dllm_graph_cache_clear": (None, []),
     "dllm_set_l2_prefetch": (C.c_int, [C.c_int64, C.c_int64, C.c_int32]),
+    "dllm_selftest_wait_timeout": (C.c_int, [_P, C.c_int32, _P]),
     "dllm_status_string": (C.c_char_p, [C.c_int]),
 }
 

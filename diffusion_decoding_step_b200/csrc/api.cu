@@ -8,6 +8,11 @@
 #include <mutex>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
+#include <chrono>
+#include <thread>
+
 #include "../../include/dllm.h"
 #include "kernels.cuh"
 
@@ -305,6 +310,31 @@ dllm_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DLLM_OK : DLL
   } while (0)
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// NVTX range over an entry point (free when no profiler is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
+
+// Wait for the work queued on st so far, giving up after deadline_s: the
+// kernels bound their own waits, this bounds the host side as well.
+dllm_status wait_stream(cudaStream_t st, double deadline_s) {
+  thread_local cudaEvent_t ev = nullptr;
+  if (!ev && cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess)
+    return DLLM_ERR_CUDA;
+  if (cudaEventRecord(ev, st) != cudaSuccess) return DLLM_ERR_CUDA;
+  const auto t0 = std::chrono::steady_clock::now();
+  for (;;) {
+    const cudaError_t q = cudaEventQuery(ev);
+    if (q == cudaSuccess) return DLLM_OK;
+    if (q != cudaErrorNotReady) return DLLM_ERR_CUDA;
+    const double el = std::chrono::duration<double>(std::chrono::steady_clock::now() - t0).count();
+    if (el > deadline_s) return DLLM_ERR_TIMEOUT;
+    if (el > 2e-3) std::this_thread::sleep_for(std::chrono::microseconds(20));
+  }
+}
+constexpr double kHostDeadlineS = 60.0;
 
 // ------------------------------------------------------------------ launches
 dllm_status run_qkv(const Ctx& c, const void* wqkv, int layer, const void* xb,
@@ -913,6 +943,7 @@ dllm_status dllm_threshold_commit(const dllm_config* cfg, int32_t block_start, c
 
 dllm_status dllm_prefill(const dllm_config* cfg, const dllm_weights* w, const dllm_state* st,
                          void* ws, size_t ws_bytes, dllm_stream stream) {
+  NvtxRange nv("dllm_prefill");
   Ctx c;
   DLLM_TRY(make_ctx(cfg, ws, ws_bytes, stream, &c));
   DLLM_TRY(check_state(c.s, w, st));
@@ -927,6 +958,7 @@ dllm_status dllm_prefill(const dllm_config* cfg, const dllm_weights* w, const dl
 dllm_status dllm_decode_step(const dllm_config* cfg, const dllm_weights* w, const dllm_state* st,
                              int32_t block_start, void* ws, size_t ws_bytes,
                              dllm_stream stream) {
+  NvtxRange nv("dllm_decode_step");
   Ctx c;
   DLLM_TRY(make_ctx(cfg, ws, ws_bytes, stream, &c));
   DLLM_TRY(check_state(c.s, w, st));
@@ -938,6 +970,7 @@ dllm_status dllm_decode_step(const dllm_config* cfg, const dllm_weights* w, cons
 dllm_status dllm_kv_cache_refresh(const dllm_config* cfg, const dllm_weights* w,
                                   const dllm_state* st, int32_t block_start, void* ws,
                                   size_t ws_bytes, dllm_stream stream) {
+  NvtxRange nv("dllm_kv_cache_refresh");
   Ctx c;
   DLLM_TRY(make_ctx(cfg, ws, ws_bytes, stream, &c));
   DLLM_TRY(check_state(c.s, w, st));
@@ -948,6 +981,7 @@ dllm_status dllm_kv_cache_refresh(const dllm_config* cfg, const dllm_weights* w,
 dllm_status dllm_decode_block(const dllm_config* cfg, const dllm_weights* w, const dllm_state* st,
                               int32_t block_start, int32_t max_steps, int32_t* steps_taken,
                               void* ws, size_t ws_bytes, dllm_stream stream) {
+  NvtxRange nv("dllm_decode_block");
   Ctx c;
   DLLM_TRY(make_ctx(cfg, ws, ws_bytes, stream, &c));
   DLLM_TRY(check_state(c.s, w, st));
@@ -962,9 +996,9 @@ dllm_status dllm_decode_block(const dllm_config* cfg, const dllm_weights* w, con
     if (cudaMemcpyAsync(rem.data(), c.at<int>(c.l.remaining), sizeof(int) * c.s.b,
                         cudaMemcpyDeviceToHost, c.st) != cudaSuccess ||
         cudaMemcpyAsync(rem.data() + c.s.b, c.at<int>(c.l.status), sizeof(int),
-                        cudaMemcpyDeviceToHost, c.st) != cudaSuccess ||
-        cudaStreamSynchronize(c.st) != cudaSuccess)
+                        cudaMemcpyDeviceToHost, c.st) != cudaSuccess)
       return DLLM_ERR_CUDA;
+    DLLM_TRY(wait_stream(c.st, kHostDeadlineS));
     if (rem[c.s.b] != 0) return DLLM_ERR_TIMEOUT;
     int left = 0;
     for (int i = 0; i < c.s.b; ++i) left += rem[i];
@@ -972,6 +1006,13 @@ dllm_status dllm_decode_block(const dllm_config* cfg, const dllm_weights* w, con
   }
   if (steps_taken) *steps_taken = n;
   return refresh_graph(c, cfg, w, st, ws, ws_bytes, block_start);
+}
+
+dllm_status dllm_selftest_wait_timeout(int32_t* status, int32_t limit_us, dllm_stream stream) {
+  if (!status) return DLLM_ERR_INVALID;
+  DLLM_TRY(prepare_device());
+  const long long us = std::min<long long>(std::max<long long>(limit_us, 1), 2000000);
+  return cuda_status(launch_wait_timeout(status, us * 1000, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 dllm_status dllm_set_l2_prefetch(int64_t attn_next_bytes, int64_t oproj_next_bytes,

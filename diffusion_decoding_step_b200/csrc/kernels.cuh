@@ -109,6 +109,7 @@ cudaError_t launch_gemm(int epi, int nt, const CUtensorMap& wmap, const CUtensor
                         const GemmParams& p, int grid, bool pdl, cudaStream_t s);
 cudaError_t gemm_prepare();
 cudaError_t attn_prepare();
+cudaError_t launch_wait_timeout(int* status, long long limit_ns, cudaStream_t s);
 
 cudaError_t launch_attn(int head_dim, const CUtensorMap& qmap, const CUtensorMap& kmap,
                         const CUtensorMap& vmap, const AttnParams& p, bool pdl,

@@ -66,17 +66,21 @@ DLLM_DEV bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_
   return ok != 0;
 }
 // Wait for the phase with the given parity to complete.  Gives up after
-// kWaitLimitNs, sets kErrTimeout in *status and returns false.
-DLLM_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, int* status) {
+// limit_ns, sets kErrTimeout in *status and returns false.
+DLLM_DEV bool mbar_wait_limit(uint64_t* bar, uint32_t parity, int* status,
+                              unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   unsigned long long t0 = global_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255u) == 0u && global_ns() - t0 > kWaitLimitNs) {
+    if ((i & 255u) == 0u && global_ns() - t0 > limit_ns) {
       if (status) atomicOr(status, kErrTimeout);
       return false;
     }
   }
+}
+DLLM_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, int* status) {
+  return mbar_wait_limit(bar, parity, status, kWaitLimitNs);
 }
 
 // A long wait (for a preceding kernel): the thread sleeps between polls, so

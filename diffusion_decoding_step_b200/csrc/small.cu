@@ -347,4 +347,24 @@ cudaError_t launch_split_f32(const float* src, __nv_bfloat16* dst, int64_t rows,
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ diagnostics
+// One CTA waits on an mbarrier that nothing arrives at: the bounded wait must
+// give up after limit_ns and report it in *status, and the kernel returns
+// normally (no trap, no fault), leaving the context usable.
+__global__ void wait_timeout_kernel(int* status, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait_limit(&bar, 0, status, limit_ns);
+}
+
+cudaError_t launch_wait_timeout(int* status, long long limit_ns, cudaStream_t s) {
+  count_launch();
+  wait_timeout_kernel<<<1, 32, 0, s>>>(status, (unsigned long long)limit_ns);
+  return cudaGetLastError();
+}
+
 }  // namespace dllm

@@ -266,6 +266,16 @@ void dllm_graph_cache_clear(void);
 dllm_status dllm_set_l2_prefetch(int64_t attn_next_bytes, int64_t oproj_next_bytes,
                                  int32_t attn_prefetch_wo);
 
+/* Failure-detection self-test (no counterpart on the pages).  Launches one
+ * CTA whose bounded device wait has nothing to wait for: after limit_us
+ * microseconds (clamped to [1, 2000000]) it gives up and ORs
+ * DLLM_DEVICE_TIMEOUT into *status (device int32), exactly as a wait inside
+ * the decode kernels reports a stalled producer, and returns without a trap
+ * or fault.  Lets tests check that a timed-out wait is reported and that the
+ * context stays usable afterwards. */
+#define DLLM_DEVICE_TIMEOUT 1
+dllm_status dllm_selftest_wait_timeout(int32_t* status, int32_t limit_us, dllm_stream stream);
+
 const char* dllm_status_string(dllm_status s);
 
 #ifdef __cplusplus
