@@ -11,7 +11,7 @@ import pytest
 import torch
 
 from tests.gpu_util import ensure_lib, ptr, stream
-from tests.test_gpu_kernels import test_block_attention_matches_oracle
+from tests.test_gpu_kernels import test_block_attention_matches_oracle as _attention_case
 
 pytestmark = pytest.mark.gpu
 
@@ -27,7 +27,7 @@ def test_bounded_wait_reports_timeout_and_context_stays_usable():
     assert int(status.item()) & abi.DLLM_DEVICE_TIMEOUT
     assert 0.015 <= waited < 5.0
     # the context is intact: kernels launched afterwards still agree with the oracle
-    test_block_attention_matches_oracle(4, 4, 32, 1, 8, 96, [[(0, 72), (0, 0)]], 0)
+    _attention_case(4, 4, 32, 1, 8, 96, [[(0, 72), (0, 0)]], 0)
 
 
 def test_selftest_rejects_a_null_status():
