@@ -28,9 +28,10 @@ from typing import Optional
 import torch
 
 MODE_NONE, MODE_PREFIX, MODE_DUAL, MODE_DUAL_PRUNED = 0, 1, 2, 3
+MODE_PREFIX_SUFFIXQ = 4    # prefix cache, block and suffix recomputed as queries each step
 COMMIT_THRESHOLD, COMMIT_TOPK = 0, 1  # conf > tau, or a fixed top-k budget per step
 MODE_NAMES = {MODE_NONE: "none", MODE_PREFIX: "prefix", MODE_DUAL: "dual",
-              MODE_DUAL_PRUNED: "dual_pruned"}
+              MODE_DUAL_PRUNED: "dual_pruned", MODE_PREFIX_SUFFIXQ: "prefix_suffixq"}
 
 SIGMA_W = 0.02
 SEED_WEIGHTS, SEED_PROMPTS, SEED_PLANTS, SEED_LENGTHS = 0, 1, 2, 3

@@ -53,6 +53,7 @@ from typing import Callable, Optional, Sequence
 import numpy as np
 
 MODE_NONE, MODE_PREFIX, MODE_DUAL, MODE_DUAL_PRUNED = 0, 1, 2, 3
+MODE_PREFIX_SUFFIXQ = 4   # prefix cache; block and suffix recomputed as queries every step
 COMMIT_THRESHOLD, COMMIT_TOPK = 0, 1
 
 AMBIG_GAP = 1e-2     # top-2 logit gap below which an argmax is ambiguous
@@ -127,11 +128,13 @@ def key_positions(mode: int, s: int, B: int, S: int, window: int, start: int) ->
       DUAL_PRUNED   : prefix, block, the window [s+B, min(s+B+window, S)) and
                       the trailing position S-1 (once) when the suffix is not
                       empty.
+      PREFIX_SUFFIXQ: prefix, block and suffix, [start, S); the suffix keys
+                      are recomputed by the step itself (its rows are queries)
     """
     end = s + B
     if mode in (MODE_NONE, MODE_PREFIX):
         return np.arange(start, end)
-    if mode == MODE_DUAL:
+    if mode in (MODE_DUAL, MODE_PREFIX_SUFFIXQ):
         return np.arange(start, S)
     if mode == MODE_DUAL_PRUNED:
         wend = min(end + window, S)
@@ -366,7 +369,7 @@ def prefill(cfg: Config, W: Weights, st: State, mirror: bool = True) -> None:
     if cfg.mode == MODE_NONE:
         return
     S = cfg.seq_len
-    end = cfg.prompt_len if cfg.mode == MODE_PREFIX else S
+    end = cfg.prompt_len if cfg.mode in (MODE_PREFIX, MODE_PREFIX_SUFFIXQ) else S
     rows = np.arange(0, end)
     x0 = W.embed(input_ids(cfg, st, 0, end))
     keys = [np.arange(st.starts[bi], end) for bi in range(cfg.batch)]
@@ -409,7 +412,16 @@ def decode_step(cfg: Config, W: Weights, st: State, plants: np.ndarray, s: int,
     Without a cache (MODE_NONE) all positions [start, s+B) are recomputed.
     """
     B, b = cfg.block, cfg.batch
-    if cfg.mode == MODE_NONE:
+    if cfg.mode == MODE_PREFIX_SUFFIXQ:
+        # Fast-dLLM's prefix cache read with the suffix as queries: the block
+        # and every later position run through the layers each step against
+        # [start, S); only the prompt's keys/values come from the cache
+        S = cfg.seq_len
+        rows = np.arange(s, S)
+        x0 = W.embed(input_ids(cfg, st, s, S))
+        keys = [np.arange(st.starts[bi], S) for bi in range(b)]
+        x = forward_rows(cfg, W, x0, rows, keys, st.kcache, st.vcache, st.starts, mirror)[:, :B]
+    elif cfg.mode == MODE_NONE:
         rows = np.arange(0, s + B)
         x0 = W.embed(input_ids(cfg, st, 0, s + B))
         keys = [np.arange(st.starts[bi], s + B) for bi in range(b)]

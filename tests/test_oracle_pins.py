@@ -478,3 +478,55 @@ def test_topk_single_step_commits_the_whole_block():
     w = TINY.replace(commit_mode=wl.COMMIT_TOPK, steps_per_block=1, gen_len=16)
     tr = Case(w).decode()
     assert tr.steps_per_block == [1, 1]
+
+
+# ---------------------------------------------------------------- prefix cache, suffix as queries
+def test_suffix_query_mode_keys_are_the_whole_valid_range():
+    for start in (0, 3):
+        np.testing.assert_array_equal(
+            O.key_positions(O.MODE_PREFIX_SUFFIXQ, 72, 8, 96, 0, start), np.arange(start, 96))
+
+
+def test_suffix_query_step_equals_dual_step_at_one_layer():
+    # with one layer a key/value depends only on its own embedding, so the
+    # suffix keys the step recomputes equal the ones DualCache's prefill cached:
+    # the block rows see identical keys and values
+    w4 = TINY.replace(mode=wl.MODE_PREFIX_SUFFIXQ)
+    w2 = TINY.replace(mode=wl.MODE_DUAL)
+    r = {}
+    for w in (w4, w2):
+        case = Case(w)
+        cfg, W = case.cfg, case.W
+        st = O.new_state(cfg, case.tokens.numpy(), case.masked.numpy().astype(bool),
+                         case.starts.numpy())
+        O.prefill(cfg, W, st)
+        r[w.mode] = O.decode_step(cfg, W, st, case.plants64, w.prompt_len, apply=False)
+    np.testing.assert_allclose(r[4].hidden, r[2].hidden, rtol=0, atol=1e-12)
+    assert np.array_equal(r[4].tok, r[2].tok)
+    np.testing.assert_allclose(r[4].conf, r[2].conf, rtol=0, atol=1e-12)
+
+
+def test_suffix_query_mode_differs_from_dual_with_two_layers():
+    # from the second layer on, the recomputed suffix states attend to the
+    # current block, so the two readings part
+    w4 = TINY.replace(mode=wl.MODE_PREFIX_SUFFIXQ, n_layers=2)
+    w2 = TINY.replace(mode=wl.MODE_DUAL, n_layers=2)
+    h = {}
+    for w in (w4, w2):
+        case = Case(w)
+        cfg, W = case.cfg, case.W
+        st = O.new_state(cfg, case.tokens.numpy(), case.masked.numpy().astype(bool),
+                         case.starts.numpy())
+        O.prefill(cfg, W, st)
+        h[w.mode] = O.decode_step(cfg, W, st, case.plants64, w.prompt_len, apply=False).hidden
+    assert np.abs(h[4] - h[2]).max() > 1e-6
+
+
+def test_suffix_query_decode_invariants():
+    w = TINY.replace(mode=wl.MODE_PREFIX_SUFFIXQ, gen_len=16)
+    tr = Case(w).decode()
+    assert all(1 <= n <= w.block for n in tr.steps_per_block)
+    assert not (tr.tokens[:, w.prompt_len:] < 0).any()
+    for s, r in tr.steps:
+        conf = r.conf[~np.isnan(r.conf)]
+        assert np.all((conf > 0) & (conf <= 1))
