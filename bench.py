@@ -40,6 +40,9 @@ def parse():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--commit", default="threshold", choices=["threshold", "topk"],
                     help="commit rule: conf > tau (default) or a fixed top-k budget per step")
+    ap.add_argument("--cache", default="",
+                    help="override the workload's cache mode (none, prefix, dual, dual_pruned, "
+                         "prefix_suffixq)")
     ap.add_argument("--steps-per-block", type=int, default=0,
                     help="topk: steps a block takes (default block/4)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -95,17 +98,24 @@ def peaks():
 def selected_workload(args):
     from diffusion_decoding_step_b200 import workload as wl
     w = wl.WORKLOADS[args.workload]
+    if args.cache:
+        w = w.replace(mode={v: k for k, v in wl.MODE_NAMES.items()}[args.cache])
     if args.commit == "topk":
         w = w.replace(commit_mode=wl.COMMIT_TOPK,
                       steps_per_block=args.steps_per_block or max(1, w.block // 4))
     return w
 
 
+def _mode_name(mode):
+    from diffusion_decoding_step_b200 import workload as wl
+    return wl.MODE_NAMES[mode]
+
+
 def workload_config(w, data_note):
     return {"workload": w.name, "batch": w.batch, "layers": w.n_layers, "hidden": w.hidden,
             "heads": f"{w.n_q_heads}/{w.n_kv_heads}x{w.head_dim}", "vocab": w.vocab,
             "prompt_len": w.prompt_len, "gen_len": w.gen_len, "block": w.block, "tau": w.tau,
-            "cache": ["none", "prefix", "dual", "dual_pruned"][w.mode],
+            "cache": _mode_name(w.mode),
             "commit": ("threshold" if w.commit_mode == 0
                        else f"topk, {w.steps_per_block} steps per block"),
             "l2": data_note}
@@ -117,7 +127,7 @@ def step_key_counts(w, s):
     end = s + w.block
     out = []
     for st in starts:
-        if w.mode == 2:                       # DualCache: the whole valid range
+        if w.mode in (2, 4):                  # DualCache / suffix as queries: whole range
             n = w.seq_len - st
         elif w.mode == 3:                     # pruned suffix window + trailing position
             wend = min(end + w.window, w.seq_len)
@@ -139,7 +149,8 @@ def step_algorithmic_bytes(w, s):
     K/V rows it writes and the activations between kernels, then the LM-head
     weights.  Logits are never stored, so they are not counted."""
     d, D, Hq, Hkv = w.hidden, w.head_dim, w.n_q_heads, w.n_kv_heads
-    rows = w.batch * ((s + w.block) if w.mode == 0 else w.block)
+    rows = w.batch * ((s + w.block) if w.mode == 0
+                      else (w.seq_len - s) if w.mode == 4 else w.block)
     per_layer = (w.qkv_rows * d * 2 + d * Hq * D * 2            # W_qkv, W_o
                  + sum(step_key_counts(w, s)) * Hkv * D * 2 * 2  # K, V read
                  + rows * (Hq + 2 * Hkv) * D * 2                 # q, k, v written

@@ -71,7 +71,7 @@ dllm_status check_cfg(const dllm_config* c, Shape* s) {
       c->n_kv_heads < 1 || c->head_dim < 1 || c->vocab < 2 || c->prompt_len < 0 ||
       c->gen_len < 1 || c->block < 1)
     return DLLM_ERR_INVALID;
-  if (c->mode < DLLM_CACHE_NONE || c->mode > DLLM_CACHE_DUAL_PRUNED) return DLLM_ERR_INVALID;
+  if (c->mode < DLLM_CACHE_NONE || c->mode > DLLM_CACHE_PREFIX_SUFFIXQ) return DLLM_ERR_INVALID;
   if (c->weight_format != DLLM_W_BF16 && c->weight_format != DLLM_W_F32_SPLIT)
     return DLLM_ERR_INVALID;
   if (c->n_q_heads % c->n_kv_heads) return DLLM_ERR_INVALID;
@@ -200,7 +200,8 @@ int key_tiles_bound(const Shape& s, int blk, int seg_end) {
   if (seg_end > 0) return cdiv(seg_end, kKeyTile);
   const int end = blk + s.B;
   switch (s.mode) {
-    case DLLM_CACHE_DUAL: return cdiv(s.S, kKeyTile);
+    case DLLM_CACHE_DUAL:
+    case DLLM_CACHE_PREFIX_SUFFIXQ: return cdiv(s.S, kKeyTile);
     case DLLM_CACHE_DUAL_PRUNED: {
       const int wend = std::min(end + s.W, s.S);
       return cdiv(wend, kKeyTile) + ((end < s.S && s.S - 1 >= wend) ? 1 : 0);
@@ -221,6 +222,9 @@ std::vector<int> row_counts(const Shape& s) {
   std::vector<int> r;
   if (s.mode == DLLM_CACHE_NONE) {
     for (int blk = s.P; blk < s.S; blk += s.B) r.push_back(blk + s.B);
+  } else if (s.mode == DLLM_CACHE_PREFIX_SUFFIXQ) {
+    r.push_back(s.G);  // the first block's step: block and whole suffix
+    r.push_back(std::max(s.P, 1));
   } else {
     r.push_back(s.B);
     r.push_back(s.mode == DLLM_CACHE_PREFIX ? std::max(s.P, 1) : s.S);
@@ -654,9 +658,11 @@ dllm_status check_block(const Shape& s, int blk) {
 dllm_status step(const Ctx& c, const dllm_weights* w, const dllm_state* st, int blk) {
   const Shape& s = c.s;
   if (!st->plants || !aligned16(st->plants)) return DLLM_ERR_INVALID;
-  const int row0 = s.mode == DLLM_CACHE_NONE ? 0 : blk;
-  const int n_rows = s.mode == DLLM_CACHE_NONE ? blk + s.B : s.B;
-  DLLM_TRY(run_forward(c, w, st, row0, n_rows, blk, s.mode == DLLM_CACHE_NONE ? blk + s.B : 0,
+  const bool none = s.mode == DLLM_CACHE_NONE;
+  const bool sufq = s.mode == DLLM_CACHE_PREFIX_SUFFIXQ;
+  const int row0 = none ? 0 : blk;
+  const int n_rows = none ? blk + s.B : sufq ? s.S - blk : s.B;
+  DLLM_TRY(run_forward(c, w, st, row0, n_rows, blk, none ? blk + s.B : sufq ? s.S : 0,
                        true));
   DLLM_TRY(run_final_norm(c, c.at<float>(c.l.x), row0, n_rows, blk, st->masked, st->plants,
                           c.at<void>(c.l.h), true));
@@ -948,7 +954,8 @@ dllm_status dllm_prefill(const dllm_config* cfg, const dllm_weights* w, const dl
   DLLM_TRY(make_ctx(cfg, ws, ws_bytes, stream, &c));
   DLLM_TRY(check_state(c.s, w, st));
   if (c.s.mode == DLLM_CACHE_NONE) return DLLM_OK;
-  const int end = c.s.mode == DLLM_CACHE_PREFIX ? c.s.P : c.s.S;
+  const int end =
+      (c.s.mode == DLLM_CACHE_PREFIX || c.s.mode == DLLM_CACHE_PREFIX_SUFFIXQ) ? c.s.P : c.s.S;
   if (end < 1) return DLLM_OK;
   const GraphKey key = make_key(cfg, w, st, ws, ws_bytes, kGraphPrefill, 0);
   return run_graph(c, key,

@@ -90,7 +90,7 @@ __device__ __forceinline__ void seq_segments(const AttnParams& p, int b, int* sg
   int l0, s1 = 0, l1 = 0;
   if (p.seg_end > 0) {
     l0 = p.seg_end - st;
-  } else if (p.mode == 2) {  // DUAL
+  } else if (p.mode == 2 || p.mode == 4) {  // DUAL, PREFIX_SUFFIXQ
     l0 = p.S - st;
   } else if (p.mode == 3) {  // DUAL_PRUNED
     const int wend = min(end + p.window, p.S);

@@ -62,7 +62,7 @@ __global__ void __launch_bounds__(256) embed_kernel(const EmbedParams p) {
     const int end = p.blk_start + p.blk_len;
     if (p.seg_end > 0) {
       l0 = p.seg_end - st;
-    } else if (p.mode == 2) {           // DUAL
+    } else if (p.mode == 2 || p.mode == 4) {  // DUAL, PREFIX_SUFFIXQ
       l0 = p.S - st;
     } else if (p.mode == 3) {           // DUAL_PRUNED
       const int wend = min(end + p.window, p.S);

@@ -59,12 +59,17 @@ typedef enum {
  *   NONE        [st, s+B), every position recomputed each step (no cache)
  *   PREFIX      [st, s+B), prefix keys/values from the cache
  *   DUAL        [st, S),   prefix and suffix from the cache
- *   DUAL_PRUNED [st, min(s+B+window, S)) plus S-1 when the suffix is not empty */
+ *   DUAL_PRUNED [st, min(s+B+window, S)) plus S-1 when the suffix is not empty
+ *   PREFIX_SUFFIXQ [st, S), prefix from the cache; the block and every later
+ *               position run through the layers as queries each step (their
+ *               keys/values are recomputed), only the block reaches the LM
+ *               head.  The prefill covers the prompt, as for PREFIX. */
 typedef enum {
   DLLM_CACHE_NONE = 0,
   DLLM_CACHE_PREFIX = 1,
   DLLM_CACHE_DUAL = 2,
-  DLLM_CACHE_DUAL_PRUNED = 3
+  DLLM_CACHE_DUAL_PRUNED = 3,
+  DLLM_CACHE_PREFIX_SUFFIXQ = 4
 } dllm_cache_mode;
 
 /* Weight storage.  BF16: bf16 weights, K extent = the input width.

@@ -206,3 +206,23 @@ def test_decode_block_topk_takes_the_step_budget():
     torch.cuda.synchronize()
     assert steps == [w.steps_per_block] * (w.gen_len // w.block)
     assert not dec.masked.any()
+
+
+
+# ---------------------------------------------------------------- prefix cache, suffix as queries
+SUFQ = {
+    "tiny_suffixq": TINY.replace(mode=wl.MODE_PREFIX_SUFFIXQ),
+    "dream_mid_suffixq": MID["dream_mid_prefix"].replace(mode=wl.MODE_PREFIX_SUFFIXQ),
+}
+
+
+@pytest.mark.parametrize("name", list(SUFQ))
+def test_lockstep_decode_suffix_queries(name):
+    """Every step runs the block and the whole suffix through the layers
+    (GQA and RoPE in the mid-size case), in lockstep with the oracle."""
+    case = Case(SUFQ[name])
+    dec = make_decoder(case)
+    rep = lockstep(dec, case)
+    assert rep.steps >= (case.w.gen_len // case.w.block)
+    assert rep.flagged_mismatch <= max(2, rep.rows // 50)
+    assert not dec.masked.any()
