@@ -222,6 +222,15 @@ def topk_ambiguity(conf, masked, k):
     return amb
 
 
+def capped(cfg, step_in_block: int) -> bool:
+    """Threshold rule with a step cap (steps_per_block > 0): the Fast-dLLM
+    README's evaluation knobs bound the sampler's steps (diffusion_steps) next
+    to the threshold; plainest reading: the step that reaches the cap commits
+    every row still masked, so a block never takes more steps than that."""
+    return (cfg.commit_mode == COMMIT_THRESHOLD and cfg.steps_per_block > 0
+            and step_in_block + 1 >= cfg.steps_per_block)
+
+
 def ambiguity_flags(conf, gap, masked, tau):
     """Rows whose outcome a correct implementation may decide either way.
 
@@ -402,7 +411,7 @@ class StepResult:
 
 
 def decode_step(cfg: Config, W: Weights, st: State, plants: np.ndarray, s: int,
-                mirror: bool = True, apply: bool = True) -> StepResult:
+                mirror: bool = True, apply: bool = True, step_in_block: int = 0) -> StepResult:
     """One denoising step of the block at [s, s+B).
 
     The block rows run through every layer (their keys/values overwrite the
@@ -452,6 +461,9 @@ def decode_step(cfg: Config, W: Weights, st: State, plants: np.ndarray, s: int,
                 commit[bi] = topk_commit(cm, m, k)
                 amb_tok[bi] = m & (gap[bi] < AMBIG_GAP)
                 amb_commit[bi] = topk_ambiguity(cm, m, k)
+            elif capped(cfg, step_in_block):
+                commit[bi] = m.copy()   # the step budget is spent: every masked row commits
+                amb_tok[bi] = m & (gap[bi] < AMBIG_GAP)
             else:
                 commit[bi] = threshold_commit(cm, m, cfg.tau)
                 amb_tok[bi], amb_commit[bi] = ambiguity_flags(cm, gap[bi], m, cfg.tau)
@@ -501,7 +513,7 @@ def decode(cfg: Config, W: Weights, tokens, masked, starts, plants,
         while st.masked[:, s:s + B].any():
             if max_steps is not None and n >= max_steps:
                 break
-            r = decode_step(cfg, W, st, plants, s, mirror)
+            r = decode_step(cfg, W, st, plants, s, mirror, step_in_block=n)
             trace.append((s, r))
             n += 1
         steps_per_block.append(n)

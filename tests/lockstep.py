@@ -37,10 +37,11 @@ def state_from_gpu(dec, layers=None) -> O.State:
                    starts=dec.seq_start.cpu().numpy().astype(np.int64))
 
 
-def compare_step(dec, case, s: int, rep: Report, check_kv: bool = True) -> None:
+def compare_step(dec, case, s: int, rep: Report, check_kv: bool = True,
+                 step_in_block: int = 0) -> None:
     cfg, W = case.cfg, case.W
     st = state_from_gpu(dec)
-    r = O.decode_step(cfg, W, st, case.plants64, s, apply=False)
+    r = O.decode_step(cfg, W, st, case.plants64, s, apply=False, step_in_block=step_in_block)
     dec.step(s)
     torch.cuda.synchronize()
     assert dec.device_status() == 0
@@ -123,7 +124,7 @@ def lockstep(dec, case, max_blocks: int | None = None, max_steps: int | None = N
         while dec.masked[:, s:s + cfg.block].any():
             if max_steps is not None and n >= max_steps:
                 break
-            compare_step(dec, case, s, rep)
+            compare_step(dec, case, s, rep, step_in_block=n)
             n += 1
             assert n <= cfg.block
         compare_refresh(dec, case, s)

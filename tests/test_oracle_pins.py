@@ -530,3 +530,32 @@ def test_suffix_query_decode_invariants():
     for s, r in tr.steps:
         conf = r.conf[~np.isnan(r.conf)]
         assert np.all((conf > 0) & (conf <= 1))
+
+
+# ---------------------------------------------------------------- step cap on the threshold rule
+def test_step_cap_of_one_commits_each_block_in_one_step():
+    w = TINY.replace(steps_per_block=1, gen_len=16)
+    tr = Case(w).decode()
+    assert tr.steps_per_block == [1, 1]
+    for _, r in tr.steps:
+        assert r.commit.sum() == w.block
+
+
+def test_step_cap_at_block_size_changes_nothing():
+    w = TINY.replace(gen_len=16)
+    t0 = Case(w).decode()
+    t1 = Case(w.replace(steps_per_block=w.block)).decode()
+    assert np.array_equal(t0.tokens, t1.tokens)
+    assert t0.steps_per_block == t1.steps_per_block
+
+
+def test_step_cap_of_two_finishes_every_block_by_its_second_step():
+    w = TINY.replace(steps_per_block=2, gen_len=16)
+    tr = Case(w).decode()
+    assert all(n <= 2 for n in tr.steps_per_block)
+    for s, r in tr.steps:
+        m = ~np.isnan(r.conf[0])
+        if r.commit[0][m].all() and m.sum() > 1:
+            break
+    else:
+        raise AssertionError("no step committed a whole multi-row remainder")
