@@ -44,7 +44,8 @@ def parse():
                     help="override the workload's cache mode (none, prefix, dual, dual_pruned, "
                          "prefix_suffixq)")
     ap.add_argument("--steps-per-block", type=int, default=0,
-                    help="topk: steps a block takes (default block/4)")
+                    help="topk: steps a block takes (default block/4); threshold: a per-block "
+                         "step cap (default none)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", action="store_true",
@@ -103,6 +104,8 @@ def selected_workload(args):
     if args.commit == "topk":
         w = w.replace(commit_mode=wl.COMMIT_TOPK,
                       steps_per_block=args.steps_per_block or max(1, w.block // 4))
+    elif args.steps_per_block > 0:  # threshold rule with a per-block step cap
+        w = w.replace(steps_per_block=args.steps_per_block)
     return w
 
 
@@ -116,8 +119,9 @@ def workload_config(w, data_note):
             "heads": f"{w.n_q_heads}/{w.n_kv_heads}x{w.head_dim}", "vocab": w.vocab,
             "prompt_len": w.prompt_len, "gen_len": w.gen_len, "block": w.block, "tau": w.tau,
             "cache": _mode_name(w.mode),
-            "commit": ("threshold" if w.commit_mode == 0
-                       else f"topk, {w.steps_per_block} steps per block"),
+            "commit": (("threshold" + (f", cap {w.steps_per_block} steps per block"
+                                        if w.steps_per_block > 0 else ""))
+                       if w.commit_mode == 0 else f"topk, {w.steps_per_block} steps per block"),
             "l2": data_note}
 
 

@@ -104,7 +104,7 @@ dllm_status check_cfg(const dllm_config* c, Shape* s) {
   s->mode = c->mode;
   s->wfmt = c->weight_format;
   s->commit_mode = c->commit_mode;
-  s->spb = c->commit_mode == DLLM_COMMIT_TOPK ? c->steps_per_block : 0;
+  s->spb = c->steps_per_block > 0 ? c->steps_per_block : 0;
   s->qkv_rows = qkv;
   const int f = c->weight_format == DLLM_W_F32_SPLIT ? 2 : 1;
   s->Kw = f * c->hidden;
@@ -212,7 +212,7 @@ int key_tiles_bound(const Shape& s, int blk, int seg_end) {
 
 // ------------------------------------------------------------------ workspace
 struct Layout {
-  size_t status, x, xb, sumsq, q, attn, h, stats, conf, tok, gap, commit,
+  size_t status, stepc, x, xb, sumsq, q, attn, h, stats, conf, tok, gap, commit,
       remaining, segs, rope, total;
   int rmax, lm_slots;
 };
@@ -247,6 +247,7 @@ Layout layout(const Shape& s) {
   const GemmPlan gl = plan_lmhead(s.V, s.b * s.B, s.Kw);
   l.lm_slots = gl.grid / gl.n_tiles;
   l.status = take(256);
+  l.stepc = take((size_t)s.b * 2 * 4);  // per sequence: steps in the block, block start
   l.x = take((size_t)l.rmax * s.d * 4);
   l.xb = take((size_t)l.rmax * s.d * 2);
   l.sumsq = take((size_t)l.rmax * (s.d / 128) * 4);
@@ -636,6 +637,7 @@ dllm_status run_commit(const Ctx& c, const dllm_state* stt, int blk_start, bool 
   p.do_commit = 1;
   p.topk = s.commit_mode == DLLM_COMMIT_TOPK;
   p.steps_per_block = s.spb;
+  p.step_ctr = c.at<int>(c.l.stepc);
   return cuda_status(launch_commit(p, pdl, c.st));
 }
 

@@ -158,7 +158,8 @@ struct CommitParams {
   int* remaining;
   int do_commit;
   int topk;             // fixed-budget rule instead of the threshold
-  int steps_per_block;  // topk: steps a block takes
+  int steps_per_block;  // topk: steps a block takes; threshold: step cap (0 = none)
+  int* step_ctr;        // [b][2] steps taken in the current block, its start (null: no cap)
 };
 cudaError_t launch_commit(const CommitParams& p, bool pdl, cudaStream_t s);
 

@@ -283,8 +283,25 @@ __global__ void __launch_bounds__(1024) commit_kernel(const CommitParams p) {
     k0 = m0 && r0 < k;
     k1 = m1 && r1 < k;
   } else {
-    k0 = m0 && (c0 > p.tau || (any_masked && bi == i0));
-    k1 = m1 && (c1 > p.tau || (any_masked && bi == i1));
+    // step cap: the step that reaches it commits every row still masked.
+    // The counter restarts whenever the block start changes or the block is
+    // untouched (every row masked).
+    bool force = false;
+    if (p.steps_per_block > 0 && p.step_ctr != nullptr) {
+      const int nm =
+          __popc(__ballot_sync(0xffffffffu, m0)) + __popc(__ballot_sync(0xffffffffu, m1));
+      int n = 0;
+      if (lane == 0) {
+        int* ctr = p.step_ctr + 2 * b;
+        n = (ctr[1] != p.blk_start || nm == p.B) ? 0 : ctr[0];
+        ctr[0] = n + 1;
+        ctr[1] = p.blk_start;
+      }
+      n = __shfl_sync(0xffffffffu, n, 0);
+      force = n + 1 >= p.steps_per_block;
+    }
+    k0 = m0 && (force || c0 > p.tau || (any_masked && bi == i0));
+    k1 = m1 && (force || c1 > p.tau || (any_masked && bi == i1));
   }
   if (k0) {
     p.tokens[base + i0] = s_tok[i0];

@@ -99,7 +99,10 @@ typedef struct {
   int32_t mode;          /* dllm_cache_mode */
   int32_t weight_format; /* dllm_weight_format */
   int32_t commit_mode;   /* dllm_commit_mode */
-  int32_t steps_per_block; /* TOPK: 1 <= steps_per_block <= block; ignored otherwise */
+  int32_t steps_per_block; /* TOPK: 1 <= steps_per_block <= block.  THRESHOLD: a step cap
+                            * per block when > 0 (the step that reaches it commits every
+                            * row still masked; counted per sequence in the workspace by
+                            * dllm_decode_step / dllm_decode_block), none when <= 0 */
 } dllm_config;
 
 /* Kw = hidden (BF16) or 2*hidden (F32_SPLIT); Ko = Hq*D or 2*Hq*D. */

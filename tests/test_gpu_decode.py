@@ -226,3 +226,35 @@ def test_lockstep_decode_suffix_queries(name):
     assert rep.steps >= (case.w.gen_len // case.w.block)
     assert rep.flagged_mismatch <= max(2, rep.rows // 50)
     assert not dec.masked.any()
+
+
+# ---------------------------------------------------------------- step cap
+CAPPED = {
+    "tiny_prefix_cap2": TINY.replace(steps_per_block=2),
+    "llada_mid_dual_cap3": MID["llada_mid_dual"].replace(steps_per_block=3),
+}
+
+
+@pytest.mark.parametrize("name", list(CAPPED))
+def test_lockstep_decode_step_cap(name):
+    """Threshold rule with a per-block step cap, in lockstep with the oracle:
+    the capping step commits every row still masked."""
+    w = CAPPED[name]
+    case = Case(w)
+    dec = make_decoder(case)
+    rep = lockstep(dec, case)
+    assert rep.steps <= (w.gen_len // w.block) * w.steps_per_block
+    assert rep.flagged_mismatch <= max(2, rep.rows // 50)
+    assert not dec.masked.any()
+
+
+def test_decode_block_respects_the_step_cap_across_generations():
+    w = CAPPED["llada_mid_dual_cap3"]
+    case = Case(w)
+    dec = make_decoder(case)
+    for _ in range(2):   # the per-sequence step counters restart with every block
+        dec.reset()
+        steps = dec.generate()
+        torch.cuda.synchronize()
+        assert all(1 <= n <= w.steps_per_block for n in steps)
+        assert not dec.masked.any()
