@@ -40,6 +40,9 @@ def parse():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--commit", default="threshold", choices=["threshold", "topk"],
                     help="commit rule: conf > tau (default) or a fixed top-k budget per step")
+    ap.add_argument("--blocks", default="lockstep", choices=["lockstep", "per-sequence"],
+                    help="batches: blocks advance together (default) or each sequence at its "
+                         "own block (dllm_decode_all)")
     ap.add_argument("--cache", default="",
                     help="override the workload's cache mode (none, prefix, dual, dual_pruned, "
                          "prefix_suffixq)")
@@ -330,13 +333,20 @@ def run_ours(args, rank, world, local_rank):
     dec = Decoder(w, weights, tokens, masked, starts, plants, device=str(dev))
     stream = dec.stream
 
-    def generation():
-        dec.reset()
+    per_seq = args.blocks == "per-sequence"
+
+    def decode_all_blocks():
+        if per_seq:  # prefill included
+            return dec.generate_per_sequence()
         dec.prefill()
         n = 0
         for s in range(w.prompt_len, w.seq_len, w.block):
             n += dec.decode_block(s)
         return n
+
+    def generation():
+        dec.reset()
+        return decode_all_blocks()
 
     def barrier():
         if world > 1:
@@ -372,8 +382,11 @@ def run_ours(args, rank, world, local_rank):
     p0.record(stream)
     dec.prefill()
     p1.record(stream)
-    for s_ in range(w.prompt_len, w.seq_len, w.block):
-        dec.decode_block(s_)
+    if per_seq:
+        dec.decode_all()
+    else:
+        for s_ in range(w.prompt_len, w.seq_len, w.block):
+            dec.decode_block(s_)
     p2.record(stream)
     torch.cuda.synchronize(dev)
     prefill_ms = p0.elapsed_time(p1)
@@ -446,9 +459,7 @@ def run_ours(args, rank, world, local_rank):
         dec.tokens.copy_(h_tokens, non_blocking=True)
         dec.masked.copy_(h_masked, non_blocking=True)
         dec.plants.copy_(h_plants, non_blocking=True)
-        dec.prefill()
-        for s_ in range(w.prompt_len, w.seq_len, w.block):
-            dec.decode_block(s_)
+        decode_all_blocks()
         h_out.copy_(dec.tokens, non_blocking=True)
 
     e2e_generation()
@@ -505,6 +516,7 @@ def run_ours(args, rank, world, local_rank):
             "gpu_launches": int(launches),
             "clocks": clk,
         }
+        line["config"]["blocks"] = args.blocks
         print(json.dumps(line), flush=True)
 
 

@@ -69,6 +69,7 @@ SIGNATURES = {
     "dllm_kv_cache_refresh": (C.c_int, [_CFG, _W, _ST, _I, _P, C.c_size_t, _P]),
     "dllm_decode_block": (C.c_int, [_CFG, _W, _ST, _I, _I, C.POINTER(C.c_int32), _P,
                                     C.c_size_t, _P]),
+    "dllm_decode_all": (C.c_int, [_CFG, _W, _ST, C.POINTER(C.c_int32), _P, C.c_size_t, _P]),
     "dllm_step_outputs": (C.c_int, [_CFG, _P, C.c_size_t, C.POINTER(C.c_void_p),
                                     C.POINTER(C.c_void_p), C.POINTER(C.c_void_p),
                                     C.POINTER(C.c_void_p)]),

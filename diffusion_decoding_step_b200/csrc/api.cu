@@ -212,7 +212,7 @@ int key_tiles_bound(const Shape& s, int blk, int seg_end) {
 
 // ------------------------------------------------------------------ workspace
 struct Layout {
-  size_t status, stepc, x, xb, sumsq, q, attn, h, stats, conf, tok, gap, commit,
+  size_t status, stepc, seqblk, seqdone, x, xb, sumsq, q, attn, h, stats, conf, tok, gap, commit,
       remaining, segs, rope, total;
   int rmax, lm_slots;
 };
@@ -248,6 +248,8 @@ Layout layout(const Shape& s) {
   l.lm_slots = gl.grid / gl.n_tiles;
   l.status = take(256);
   l.stepc = take((size_t)s.b * 2 * 4);  // per sequence: steps in the block, block start
+  l.seqblk = take((size_t)s.b * 4);     // per sequence: current block (dllm_decode_all)
+  l.seqdone = take((size_t)s.b * 4);    // per sequence: every block done
   l.x = take((size_t)l.rmax * s.d * 4);
   l.xb = take((size_t)l.rmax * s.d * 2);
   l.sumsq = take((size_t)l.rmax * (s.d / 128) * 4);
@@ -272,6 +274,9 @@ struct Ctx {
   Layout l;
   uint8_t* ws;
   cudaStream_t st;
+  // per-sequence block starts in the workspace (dllm_decode_all), or null:
+  // every sequence is at the block the call names
+  int* seq_blk = nullptr;
   template <class T>
   T* at(size_t off) const {
     return reinterpret_cast<T*>(ws + off);
@@ -370,6 +375,7 @@ dllm_status run_qkv(const Ctx& c, const void* wqkv, int layer, const void* xb,
   p.kb_per_split = g.kbps;
   p.units = g.units;
   p.layer = layer;
+  p.seq_blk = c.seq_blk;
   p.status = c.at<int>(c.l.status);
   p.n_rows = n_rows;
   p.row0 = row0;
@@ -467,6 +473,7 @@ dllm_status run_attn(const Ctx& c, int layer, int n_rows, const void* q, const v
   p.seq_start = keys.seq_start;
   p.dep_lo = keys.dep_lo;
   p.dep_hi = keys.dep_hi;
+  p.seq_blk = c.seq_blk;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.status = c.at<int>(c.l.status);
   p.scale_log2 = 1.4426950408889634f / sqrtf((float)s.D);
@@ -490,6 +497,7 @@ dllm_status run_embed(const Ctx& c, const dllm_weights* w, const dllm_state* stt
   e.mask_id = s.mask_id;
   e.npart = s.d / 128;
   e.status = c.at<int>(c.l.status);
+  e.seq_blk = c.seq_blk;
   e.tokens = stt->tokens;
   e.masked = stt->masked;
   e.embed = w->embed;
@@ -526,7 +534,9 @@ dllm_status run_forward(const Ctx& c, const dllm_weights* w, const dllm_state* s
                         int n_rows, int blk_start, int seg_end, bool lm_next) {
   const Shape& s = c.s;
   DLLM_TRY(run_embed(c, w, stt, row0, n_rows, blk_start, seg_end, true));
-  const int ntb = key_tiles_bound(s, blk_start, seg_end);
+  int ntb = key_tiles_bound(s, blk_start, seg_end);
+  if (c.seq_blk)  // each sequence at its own block: plan for the widest key set
+    for (int blk = s.P; blk < s.S; blk += s.B) ntb = std::max(ntb, key_tiles_bound(s, blk, seg_end));
   const long long qkv_bytes = (long long)s.qkv_rows * s.Kw * 2;
   const long long wo_bytes = (long long)s.d * s.Ko * 2;
   const auto* wqkv = static_cast<const uint8_t*>(w->wqkv);
@@ -586,6 +596,7 @@ dllm_status run_final_norm(const Ctx& c, const float* x, int row0, int n_rows, i
   f.masked = masked;
   f.plants = static_cast<const __nv_bfloat16*>(plants);
   f.h = static_cast<__nv_bfloat16*>(h);
+  f.seq_blk = c.seq_blk;
   return cuda_status(launch_final_norm(f, pdl, c.st));
 }
 
@@ -638,6 +649,8 @@ dllm_status run_commit(const Ctx& c, const dllm_state* stt, int blk_start, bool 
   p.topk = s.commit_mode == DLLM_COMMIT_TOPK;
   p.steps_per_block = s.spb;
   p.step_ctr = c.at<int>(c.l.stepc);
+  p.seq_blk = c.seq_blk;
+  p.seq_done = c.seq_blk ? c.at<int>(c.l.seqdone) : nullptr;
   return cuda_status(launch_commit(p, pdl, c.st));
 }
 
@@ -756,7 +769,7 @@ dllm_status run_graph(const Ctx& c, const GraphKey& key, F&& body) {
   return cuda_status(cudaGraphLaunch(exec, c.st));
 }
 
-enum GraphKind { kGraphStep = 1, kGraphRefresh = 2, kGraphPrefill = 3 };
+enum GraphKind { kGraphStep = 1, kGraphRefresh = 2, kGraphPrefill = 3, kGraphSeqPass = 4 };
 
 dllm_status step_graph(const Ctx& c, const dllm_config* cfg, const dllm_weights* w,
                        const dllm_state* st, void* ws, size_t ws_bytes, int blk) {
@@ -1015,6 +1028,48 @@ dllm_status dllm_decode_block(const dllm_config* cfg, const dllm_weights* w, con
   }
   if (steps_taken) *steps_taken = n;
   return refresh_graph(c, cfg, w, st, ws, ws_bytes, block_start);
+}
+
+dllm_status dllm_decode_all(const dllm_config* cfg, const dllm_weights* w, const dllm_state* st,
+                            int32_t* passes, void* ws, size_t ws_bytes, dllm_stream stream) {
+  NvtxRange nv("dllm_decode_all");
+  Ctx c;
+  DLLM_TRY(make_ctx(cfg, ws, ws_bytes, stream, &c));
+  DLLM_TRY(check_state(c.s, w, st));
+  if (c.s.mode == DLLM_CACHE_NONE || c.s.mode == DLLM_CACHE_PREFIX_SUFFIXQ)
+    return DLLM_ERR_UNSUPPORTED;
+  if (!st->plants || !aligned16(st->plants)) return DLLM_ERR_INVALID;
+  const Shape& s = c.s;
+  // every sequence starts at the first generated block
+  std::vector<int> init(s.b, s.P);
+  if (cudaMemcpyAsync(c.at<int>(c.l.seqblk), init.data(), sizeof(int) * s.b,
+                      cudaMemcpyHostToDevice, c.st) != cudaSuccess ||
+      cudaMemsetAsync(c.at<int>(c.l.seqdone), 0, sizeof(int) * s.b, c.st) != cudaSuccess ||
+      cudaMemsetAsync(c.at<int>(c.l.stepc), 0, sizeof(int) * 2 * s.b, c.st) != cudaSuccess)
+    return DLLM_ERR_CUDA;
+  Ctx cs = c;
+  cs.seq_blk = c.at<int>(c.l.seqblk);
+  const GraphKey key = make_key(cfg, w, st, ws, ws_bytes, kGraphSeqPass, 0);
+  // a block takes at most B steps and one refresh pass
+  const int max_passes = (s.G / s.B) * (s.B + 1) + 1;
+  std::vector<int> rem(s.b + 1);
+  int n = 0;
+  for (; n < max_passes;) {
+    DLLM_TRY(run_graph(cs, key, [&](const Ctx& cc) { return step(cc, w, st, s.P); }));
+    ++n;
+    if (cudaMemcpyAsync(rem.data(), c.at<int>(c.l.remaining), sizeof(int) * s.b,
+                        cudaMemcpyDeviceToHost, c.st) != cudaSuccess ||
+        cudaMemcpyAsync(rem.data() + s.b, c.at<int>(c.l.status), sizeof(int),
+                        cudaMemcpyDeviceToHost, c.st) != cudaSuccess)
+      return DLLM_ERR_CUDA;
+    DLLM_TRY(wait_stream(c.st, kHostDeadlineS));
+    if (rem[s.b] != 0) return DLLM_ERR_TIMEOUT;
+    int left = 0;
+    for (int i = 0; i < s.b; ++i) left += rem[i];
+    if (left == 0) break;
+  }
+  if (passes) *passes = n;
+  return n < max_passes ? DLLM_OK : DLLM_ERR_INVALID;
 }
 
 dllm_status dllm_selftest_wait_timeout(int32_t* status, int32_t limit_us, dllm_stream stream) {

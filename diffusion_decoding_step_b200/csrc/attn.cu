@@ -86,7 +86,7 @@ __device__ __forceinline__ void seq_segments(const AttnParams& p, int b, int* sg
     return;
   }
   const int st = p.seq_start[b];
-  const int end = p.blk_start + p.blk_len;
+  const int end = (p.seq_blk ? p.seq_blk[b] : p.blk_start) + p.blk_len;
   int l0, s1 = 0, l1 = 0;
   if (p.seg_end > 0) {
     l0 = p.seg_end - st;
@@ -224,13 +224,16 @@ __global__ void __launch_bounds__(128, 1)
   };
 
   unsigned pre = 0;  // stages requested before the dependency wait
+  // key positions the preceding kernel writes: this sequence's query rows
+  const int dep_lo = p.seq_blk ? p.seq_blk[b] : p.dep_lo;
+  const int dep_hi = p.seq_blk ? p.seq_blk[b] + p.n_rows : p.dep_hi;
   if (t == 0 && p.segs == nullptr) {
     int first, n;
     chunk_range(first, n);
     for (int j = 0; j < min(n, ST); ++j) {
       int start, nv;
       tile_of(sg, first + j, start, nv);
-      if (start + kKeys <= p.dep_lo || start >= p.dep_hi) {
+      if (start + kKeys <= dep_lo || start >= dep_hi) {
         issue_kv(j, start);
         pre |= 1u << j;
       }

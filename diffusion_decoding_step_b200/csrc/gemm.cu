@@ -136,7 +136,7 @@ __device__ __forceinline__ void epi_prepare(const GemmParams& p, int n, int et, 
         if (xrow < p.R) {
           const int b = xrow / p.n_rows;
           const int ii = xrow - b * p.n_rows;
-          const int pos = p.row0 + ii;
+          const int pos = (p.seq_blk ? p.seq_blk[b] : p.row0) + ii;
           if (p.rope_tab != nullptr) r = pos - p.seq_start[b];
           qo = b * p.Hq * p.n_rows + ii;                       // in units of D
           ko = (p.layer * p.batch + b) * p.Hkv * p.S + pos;    // in units of D

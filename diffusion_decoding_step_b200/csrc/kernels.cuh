@@ -60,6 +60,7 @@ struct GemmParams {
   LmStat* stats;
   int stat_slots;
   int recv_in_ring;  // split K: partials go into the weight ring (grid > SM count)
+  const int* seq_blk;  // QKV: per-sequence first row position, or null: row0
   L2Prefetch pf;
 };
 
@@ -76,6 +77,7 @@ struct AttnParams {
   int dep_lo, dep_hi;  // key positions the preceding kernel writes (load after the wait)
   __nv_bfloat16* out;  // [b*n_rows][Hq*D]
   int* status;
+  const int* seq_blk;  // per-sequence block starts (query rows and dep range), or null
   float scale_log2;    // log2(e) / sqrt(D)
   L2Prefetch pf;
 };
@@ -129,6 +131,7 @@ struct EmbedParams {
   int* segs;
   const int* seq_start;
   int mode, window, seg_end;  // seg_end: end of the key range for prefill/none
+  const int* seq_blk;  // per-sequence block starts (rows start there), or null: row0 / blk_start
 };
 cudaError_t launch_embed(const EmbedParams& p, bool pdl, cudaStream_t s);
 
@@ -140,6 +143,7 @@ struct FinalNormParams {
   const uint8_t* masked;
   const __nv_bfloat16* plants;
   __nv_bfloat16* h;
+  const int* seq_blk;  // per-sequence block starts, or null: blk_start (= row0)
 };
 cudaError_t launch_final_norm(const FinalNormParams& p, bool pdl, cudaStream_t s);
 
@@ -160,6 +164,11 @@ struct CommitParams {
   int topk;             // fixed-budget rule instead of the threshold
   int steps_per_block;  // topk: steps a block takes; threshold: step cap (0 = none)
   int* step_ctr;        // [b][2] steps taken in the current block, its start (null: no cap)
+  // per-sequence blocks (null: blk_start for every sequence): a pass that
+  // finds no masked row in a sequence's block was that block's refresh, and
+  // the sequence moves on to its next block (or is done after the last)
+  int* seq_blk;
+  int* seq_done;
 };
 cudaError_t launch_commit(const CommitParams& p, bool pdl, cudaStream_t s);
 

@@ -55,11 +55,11 @@ __global__ void __launch_bounds__(256) embed_kernel(const EmbedParams p) {
   grid_dep_launch();
   const int row = blockIdx.x;
   const int b = row / p.n_rows;
-  const int pos = p.row0 + (row - b * p.n_rows);
+  const int pos = (p.seq_blk ? p.seq_blk[b] : p.row0) + (row - b * p.n_rows);
   for (int bb = threadIdx.x; row == 0 && p.segs != nullptr && bb < p.batch; bb += blockDim.x) {
     const int st = p.seq_start[bb];
     int s0 = st, l0 = 0, s1 = 0, l1 = 0;
-    const int end = p.blk_start + p.blk_len;
+    const int end = (p.seq_blk ? p.seq_blk[bb] : p.blk_start) + p.blk_len;
     if (p.seg_end > 0) {
       l0 = p.seg_end - st;
     } else if (p.mode == 2 || p.mode == 4) {  // DUAL, PREFIX_SUFFIXQ
@@ -126,8 +126,9 @@ __global__ void __launch_bounds__(256) final_norm_kernel(const FinalNormParams p
   grid_dep_wait();
   grid_dep_launch();
   const int b = blockIdx.x / p.B, i = blockIdx.x - b * p.B;
-  const int pos = p.blk_start + i;
-  const float* xr = p.x + ((size_t)b * p.n_rows + (pos - p.row0)) * p.d;
+  const int blk = p.seq_blk ? p.seq_blk[b] : p.blk_start;
+  const int pos = blk + i;
+  const float* xr = p.x + ((size_t)b * p.n_rows + (pos - (p.seq_blk ? blk : p.row0))) * p.d;
   float sq = 0.f;
   for (int k = threadIdx.x * 4; k < p.d; k += blockDim.x * 4) {
     const float4 f = *reinterpret_cast<const float4*>(xr + k);
@@ -236,7 +237,8 @@ __global__ void __launch_bounds__(1024) commit_kernel(const CommitParams p) {
   if (!p.do_commit || warp != 0) return;
   // two rows per lane (B <= 64)
   const int i0 = lane, i1 = lane + 32;
-  const size_t base = (size_t)b * p.S + p.blk_start;
+  const int blk = p.seq_blk ? p.seq_blk[b] : p.blk_start;
+  const size_t base = (size_t)b * p.S + blk;
   const bool m0 = i0 < p.B && p.masked[base + i0];
   const bool m1 = i1 < p.B && p.masked[base + i1];
   const float c0 = m0 ? s_conf[i0] : -1.f;
@@ -293,9 +295,9 @@ __global__ void __launch_bounds__(1024) commit_kernel(const CommitParams p) {
       int n = 0;
       if (lane == 0) {
         int* ctr = p.step_ctr + 2 * b;
-        n = (ctr[1] != p.blk_start || nm == p.B) ? 0 : ctr[0];
+        n = (ctr[1] != blk || nm == p.B) ? 0 : ctr[0];
         ctr[0] = n + 1;
-        ctr[1] = p.blk_start;
+        ctr[1] = blk;
       }
       n = __shfl_sync(0xffffffffu, n, 0);
       force = n + 1 >= p.steps_per_block;
@@ -317,6 +319,20 @@ __global__ void __launch_bounds__(1024) commit_kernel(const CommitParams p) {
   }
   const unsigned left = __popc(__ballot_sync(0xffffffffu, m0 && !k0)) +
                         __popc(__ballot_sync(0xffffffffu, m1 && !k1));
+  if (p.seq_blk != nullptr) {
+    // per-sequence blocks: a block without masked rows was refreshed by this
+    // pass; move on.  remaining = 1 while the sequence has work left.
+    const bool any_start = __any_sync(0xffffffffu, m0 || m1);
+    if (lane == 0) {
+      int done = p.seq_done[b];
+      if (!done && !any_start) {
+        if (blk + p.B >= p.S) p.seq_done[b] = done = 1;
+        else p.seq_blk[b] = blk + p.B;
+      }
+      if (p.remaining) p.remaining[b] = done ? 0 : 1;
+    }
+    return;
+  }
   if (lane == 0 && p.remaining) p.remaining[b] = (int)left;
 }
 

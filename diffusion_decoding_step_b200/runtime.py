@@ -119,6 +119,21 @@ class Decoder:
             steps.append(self.decode_block(s))
         return steps
 
+    def generate_per_sequence(self) -> int:
+        """Prefill, then every sequence decoded at its own block position
+        (dllm_decode_all); returns the number of passes."""
+        self.prefill()
+        return self.decode_all()
+
+    def decode_all(self) -> int:
+        """Every sequence decoded at its own block position, after a prefill;
+        returns the number of passes."""
+        n = C.c_int32(0)
+        abi.check(abi.dllm_decode_all(self.cfg_p, C.byref(self.weights_c), C.byref(self.state_c),
+                                      C.byref(n), _ptr(self.ws), self.ws_bytes, self._sh),
+                  "decode_all")
+        return int(n.value)
+
     def step_outputs(self):
         """(conf, tok, gap, commit) of the last step, each [b][B], as views."""
         ptrs = [C.c_void_p() for _ in range(4)]

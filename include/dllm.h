@@ -245,6 +245,19 @@ dllm_status dllm_decode_block(const dllm_config* cfg, const dllm_weights* w,
                               int32_t* steps_taken, void* ws, size_t ws_bytes,
                               dllm_stream stream);
 
+/* Decode every block of every sequence, each sequence at its own block
+ * (after dllm_prefill).  A pass runs one step for every sequence at its
+ * current block; a pass that finds no masked row in a sequence's block is
+ * that block's refresh (the rows, all committed, rewrite their keys/values
+ * against the step's key set) and the sequence moves to its next block.  A
+ * finished sequence's passes recompute its last block (no state change).
+ * Each sequence's tokens equal those of dllm_decode_block run block by block
+ * with the batch in lockstep: sequences never interact.  Blocks the calling
+ * host thread until done; *passes (host, may be NULL) gets the pass count.
+ * NONE and PREFIX_SUFFIXQ caches return DLLM_ERR_UNSUPPORTED. */
+dllm_status dllm_decode_all(const dllm_config* cfg, const dllm_weights* w, const dllm_state* st,
+                            int32_t* passes, void* ws, size_t ws_bytes, dllm_stream stream);
+
 /* Device pointers (into ws) of the last step's outputs, each [b][B]. */
 dllm_status dllm_step_outputs(const dllm_config* cfg, void* ws, size_t ws_bytes, float** conf,
                               int32_t** tok, float** gap, uint8_t** commit);

@@ -1,4 +1,6 @@
 """Step-level and whole-decode parity of the CUDA path with the oracle (B200 only)."""
+import ctypes as C
+
 import numpy as np
 import pytest
 import torch
@@ -258,3 +260,49 @@ def test_decode_block_respects_the_step_cap_across_generations():
         torch.cuda.synchronize()
         assert all(1 <= n <= w.steps_per_block for n in steps)
         assert not dec.masked.any()
+
+
+# ---------------------------------------------------------------- per-sequence blocks
+PER_SEQ = {
+    "batch_mid_dual": MID["batch_mid_dual"],
+    "qwen_mid_pruned": MID["qwen_mid_pruned"],
+    "tiny_prefix": TINY,
+    "batch_mid_dual_topk": MID["batch_mid_dual"].replace(commit_mode=wl.COMMIT_TOPK,
+                                                         steps_per_block=4),
+    "batch_mid_dual_cap": MID["batch_mid_dual"].replace(steps_per_block=3),
+}
+
+
+@pytest.mark.parametrize("name", list(PER_SEQ))
+def test_per_sequence_blocks_reproduce_lockstep_tokens(name):
+    """Sequences never interact, so decoding each at its own block must give
+    bit-identical tokens to the batch moving block by block in lockstep (whose
+    parity with the oracle the lockstep tests establish)."""
+    w = PER_SEQ[name]
+    case = Case(w)
+    dec = make_decoder(case)
+    steps = dec.generate()
+    torch.cuda.synchronize()
+    want = dec.tokens.cpu().numpy().copy()
+    assert not dec.masked.any()
+    dec.reset()
+    passes = dec.generate_per_sequence()
+    torch.cuda.synchronize()
+    assert dec.device_status() == 0
+    assert not dec.masked.any()
+    assert np.array_equal(dec.tokens.cpu().numpy(), want)
+    # a sequence takes its blocks' steps plus one refresh pass per block; the
+    # batch finishes with the slowest sequence, never later than lockstep
+    assert passes <= sum(steps) + len(steps)
+
+
+def test_per_sequence_blocks_reject_unsupported_caches():
+    abi = ensure_lib()
+    for w in (TINY.replace(mode=wl.MODE_NONE), TINY.replace(mode=wl.MODE_PREFIX_SUFFIXQ)):
+        case = Case(w)
+        dec = make_decoder(case)
+        n = C.c_int32(0)
+        st = abi.dllm_decode_all(dec.cfg_p, C.byref(dec.weights_c), C.byref(dec.state_c),
+                                 C.byref(n), C.c_void_p(dec.ws.data_ptr()), dec.ws_bytes,
+                                 dec._sh)
+        assert st == abi.DLLM_ERR_UNSUPPORTED
