@@ -41,7 +41,8 @@ class dllm_weights(C.Structure):
 
 class dllm_state(C.Structure):
     _fields_ = [("tokens", C.c_void_p), ("masked", C.c_void_p), ("seq_start", C.c_void_p),
-                ("k_cache", C.c_void_p), ("v_cache", C.c_void_p), ("plants", C.c_void_p)]
+                ("k_cache", C.c_void_p), ("v_cache", C.c_void_p), ("plants", C.c_void_p),
+                ("tau", C.c_void_p)]
 
 
 _P = C.c_void_p

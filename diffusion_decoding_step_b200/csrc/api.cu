@@ -649,6 +649,7 @@ dllm_status run_commit(const Ctx& c, const dllm_state* stt, int blk_start, bool 
   p.topk = s.commit_mode == DLLM_COMMIT_TOPK;
   p.steps_per_block = s.spb;
   p.step_ctr = c.at<int>(c.l.stepc);
+  p.tau_seq = stt->tau;
   p.seq_blk = c.seq_blk;
   p.seq_done = c.seq_blk ? c.at<int>(c.l.seqdone) : nullptr;
   return cuda_status(launch_commit(p, pdl, c.st));

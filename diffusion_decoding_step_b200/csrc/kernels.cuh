@@ -169,6 +169,7 @@ struct CommitParams {
   // the sequence moves on to its next block (or is done after the last)
   int* seq_blk;
   int* seq_done;
+  const float* tau_seq;  // [b] per-sequence threshold, or null: tau
 };
 cudaError_t launch_commit(const CommitParams& p, bool pdl, cudaStream_t s);
 

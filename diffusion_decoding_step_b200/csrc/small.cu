@@ -302,8 +302,9 @@ __global__ void __launch_bounds__(1024) commit_kernel(const CommitParams p) {
       n = __shfl_sync(0xffffffffu, n, 0);
       force = n + 1 >= p.steps_per_block;
     }
-    k0 = m0 && (force || c0 > p.tau || (any_masked && bi == i0));
-    k1 = m1 && (force || c1 > p.tau || (any_masked && bi == i1));
+    const float tau = p.tau_seq ? p.tau_seq[b] : p.tau;
+    k0 = m0 && (force || c0 > tau || (any_masked && bi == i0));
+    k1 = m1 && (force || c1 > tau || (any_masked && bi == i1));
   }
   if (k0) {
     p.tokens[base + i0] = s_tok[i0];

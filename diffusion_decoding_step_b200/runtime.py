@@ -67,6 +67,7 @@ class Decoder:
         self.v_cache = torch.zeros(cache_shape, dtype=torch.bfloat16, device=dev)
         self.state_c = abi.dllm_state(_ptr(self.tokens), _ptr(self.masked), _ptr(self.seq_start),
                                       _ptr(self.k_cache), _ptr(self.v_cache), _ptr(self.plants))
+        self.tau_seq = None
         self.ws_bytes = workspace_bytes(w)
         self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device=dev)
         abi.check(abi.dllm_workspace_init(C.byref(self.cfg), _ptr(self.ws), self.ws_bytes, sh),
@@ -88,6 +89,17 @@ class Decoder:
     def reset(self):
         self.tokens.copy_(self.tokens0)
         self.masked.copy_(self.masked0)
+
+    def set_tau(self, tau) -> None:
+        """Per-sequence thresholds (a list of b floats), or None for the
+        configuration's single tau.  The steps read them from device memory."""
+        if tau is None:
+            self.tau_seq = None
+            self.state_c.tau = None
+        else:
+            self.tau_seq = torch.tensor(list(tau), dtype=torch.float32, device=self.device)
+            assert self.tau_seq.numel() == self.w.batch
+            self.state_c.tau = _ptr(self.tau_seq)
 
     def prefill(self):
         abi.check(abi.dllm_prefill(self.cfg_p, C.byref(self.weights_c), C.byref(self.state_c),

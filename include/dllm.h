@@ -120,6 +120,8 @@ typedef struct {
   void* k_cache;            /* bf16 [L][b][Hkv][S][D]; must hold finite values */
   void* v_cache;            /* bf16 [L][b][Hkv][S][D] */
   const void* plants;       /* bf16 [b][G][hidden] planted LM-head offsets of generated rows */
+  const float* tau;         /* [b] per-sequence commit threshold (device), read by every step,
+                             * so a policy may change it between steps; NULL: cfg->tau */
 } dllm_state;
 
 /* Bytes of workspace a configuration needs (host call, no GPU work). */

@@ -131,18 +131,22 @@ def lockstep(dec, case, max_blocks: int | None = None, max_steps: int | None = N
     return rep
 
 
-def compare_step_sampled(dec, case, s: int, seqs, rep: Report) -> None:
+def compare_step_sampled(dec, case, s: int, seqs, rep: Report, taus=None,
+                         step_in_block: int = 0) -> None:
     """One GPU step of the whole batch, checked on the sequences `seqs` only:
     the oracle recomputes each of them alone from its GPU state (sequences of
-    a batch are independent, which the oracle's own pins establish)."""
-    cfg1 = dataclasses.replace(case.cfg, batch=1)
+    a batch are independent, which the oracle's own pins establish).  taus:
+    per-sequence thresholds, when the GPU runs with them."""
     refs = {}
     for bi in seqs:
+        cfg1 = dataclasses.replace(case.cfg, batch=1,
+                                   **({} if taus is None else {"tau": float(taus[bi])}))
         st = O.State(tokens=dec.tokens[bi:bi + 1].cpu().numpy().astype(np.int64),
                      masked=dec.masked[bi:bi + 1].cpu().numpy().astype(bool),
                      kcache=f64(dec.k_cache[:, bi:bi + 1]), vcache=f64(dec.v_cache[:, bi:bi + 1]),
                      starts=dec.seq_start[bi:bi + 1].cpu().numpy().astype(np.int64))
-        refs[bi] = O.decode_step(cfg1, case.W, st, case.plants64[bi:bi + 1], s, apply=False)
+        refs[bi] = O.decode_step(cfg1, case.W, st, case.plants64[bi:bi + 1], s, apply=False,
+                                 step_in_block=step_in_block)
         del st
     dec.step(s)
     torch.cuda.synchronize()
@@ -150,6 +154,9 @@ def compare_step_sampled(dec, case, s: int, seqs, rep: Report) -> None:
     conf, tok, gap, commit = (t.cpu().numpy() for t in dec.step_outputs())
     for bi, r in refs.items():
         m = ~np.isnan(r.conf[0])
+        if not m.any():  # this sequence's block is already done
+            assert not commit[bi].any()
+            continue
         rep.rows += int(m.sum())
         err = np.abs(conf[bi][m] - r.conf[0][m])
         rep.max_conf_err = max(rep.max_conf_err, float(err.max()))

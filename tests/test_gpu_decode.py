@@ -306,3 +306,48 @@ def test_per_sequence_blocks_reject_unsupported_caches():
                                  C.byref(n), C.c_void_p(dec.ws.data_ptr()), dec.ws_bytes,
                                  dec._sh)
         assert st == abi.DLLM_ERR_UNSUPPORTED
+
+
+# ---------------------------------------------------------------- per-sequence thresholds
+def test_per_sequence_tau_in_lockstep_with_the_oracle():
+    """Each sequence commits against its own threshold, read from device
+    memory every step (here fixed per sequence; a policy may change them)."""
+    from tests.lockstep import Report, compare_step_sampled
+    w = MID["batch_mid_dual"]
+    taus = [0.5, 0.9, 1.5]
+    case = Case(w)
+    dec = make_decoder(case)
+    dec.set_tau(taus)
+    dec.prefill()
+    rep = Report()
+    for s in range(w.prompt_len, w.seq_len, w.block):
+        n = 0
+        while dec.masked[:, s:s + w.block].any():
+            compare_step_sampled(dec, case, s, list(range(w.batch)), rep, taus=taus,
+                                 step_in_block=n)
+            n += 1
+            assert n <= w.block
+        dec.refresh(s)
+    torch.cuda.synchronize()
+    assert dec.device_status() == 0 and not dec.masked.any()
+    assert rep.flagged_mismatch <= max(2, rep.rows // 50)
+
+
+def test_tau_array_changes_between_steps():
+    """The graphs read the thresholds from device memory: changing them
+    between steps takes effect without rebuilding anything."""
+    w = MID["batch_mid_dual"]
+    case = Case(w)
+    dec = make_decoder(case)
+    dec.set_tau([2.0] * w.batch)          # one commit per sequence per step
+    dec.prefill()
+    s = w.prompt_len
+    dec.step(s)
+    c1 = dec.step_outputs()[3].cpu().numpy().sum(1)
+    dec.tau_seq.fill_(-1.0)               # now every masked row clears it
+    dec.step(s)
+    torch.cuda.synchronize()
+    c2 = dec.step_outputs()[3].cpu().numpy().sum(1)
+    assert (c1 <= 1).all()
+    assert (dec.masked[:, s:s + w.block].cpu().numpy() == 0).all()
+    assert (c2 >= 1).all()
