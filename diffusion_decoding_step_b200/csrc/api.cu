@@ -121,8 +121,9 @@ struct GemmPlan {
 };
 
 // Split K only for decode tiles (NT <= 64): the splits of a tile run as one
-// cluster whose partials meet in rank 0's stage buffers, which hold
-// (splits - 1) partials of 128 x NT fp32.
+// cluster (at most 4 CTAs for NT 32, 3 for NT 64) whose ranks exchange their
+// fp32 partials through distributed shared memory.  The cost model counts
+// k-blocks per CTA, one per unit, and one for a split's reduction.
 GemmPlan plan_gemm(int M, int R, int K, bool allow_split) {
   GemmPlan g;
   g.nt = R <= 32 ? 32 : R <= 64 ? 64 : R <= 128 ? 128 : 256;
@@ -132,7 +133,6 @@ GemmPlan plan_gemm(int M, int R, int K, bool allow_split) {
   const int kbt = K / 64;
   int best_s = 1, best_kbps = kbt;
   double best_cost = 1e30;
-  // rank 0's stage region: 3 x (16 KB + NT*128 B) -> 60 KB (NT 32), 72 KB (NT 64)
   const int cluster_max = g.nt == 32 ? 4 : g.nt == 64 ? 3 : 1;
   const int max_s = allow_split ? std::min(cluster_max, kbt) : 1;
   for (int s = 1; s <= max_s; ++s) {
@@ -167,11 +167,17 @@ GemmPlan plan_gemm_splits(int M, int R, int K, int sp) {
   return g;
 }
 
+// The LM head streams whole vocabulary tiles on persistent CTAs.  Its grid
+// is the fewest CTAs (at most one per SM, a multiple of the row tiles) that
+// keep the tiles per CTA at their minimum, so no last round runs on a few
+// SMs alone: 1188 tiles take 132 CTAs x 9 rather than 148 CTAs with 4 of
+// them streaming a ninth tile after the others are done.
 GemmPlan plan_lmhead(int V, int R, int K) {
   GemmPlan g = plan_gemm(V, R, K, false);
-  int grid = std::min(g.units, kNumSMs);
-  grid = std::max(g.n_tiles, grid / g.n_tiles * g.n_tiles);
-  g.grid = grid;
+  const int rounds = cdiv(g.units, kNumSMs);
+  int grid = cdiv(cdiv(g.units, rounds), g.n_tiles) * g.n_tiles;
+  if (grid > kNumSMs) grid = kNumSMs / g.n_tiles * g.n_tiles;
+  g.grid = std::max(g.n_tiles, grid);
   return g;
 }
 
@@ -347,19 +353,26 @@ dllm_status wait_stream(cudaStream_t st, double deadline_s) {
 constexpr double kHostDeadlineS = 60.0;
 
 // ------------------------------------------------------------------ launches
+// Q/K/V projection plan for R activation rows.  More split CTAs than SMs
+// start partly late (beside the O-projection still running); two splits on a
+// deeper ring measured faster than three.
+GemmPlan plan_qkv(const Shape& s, int R, int* epi) {
+  GemmPlan g = plan_gemm(s.qkv_rows, R, s.Kw, true);
+  *epi = EPI_QKV;
+  if (g.nt <= 64 && g.splits > 2 && g.grid > kNumSMs) {
+    g = plan_gemm_splits(s.qkv_rows, R, s.Kw, 2);
+    *epi = EPI_QKV_DEEP;
+  }
+  return g;
+}
+
 dllm_status run_qkv(const Ctx& c, const void* wqkv, int layer, const void* xb,
                     const float* sumsq, int row0, int n_rows, const int* seq_start, void* q_out,
                     void* kc, void* vc, bool pdl, const L2Prefetch& pf = L2Prefetch{}) {
   const Shape& s = c.s;
   const int R = s.b * n_rows;
-  GemmPlan g = plan_gemm(s.qkv_rows, R, s.Kw, true);
-  // More split CTAs than SMs start partly late (beside the O-projection
-  // still running); two splits on a deeper ring measured faster than three.
-  int epi = EPI_QKV;
-  if (g.nt <= 64 && g.splits > 2 && g.grid > kNumSMs) {
-    g = plan_gemm_splits(s.qkv_rows, R, s.Kw, 2);
-    epi = EPI_QKV_DEEP;
-  }
+  int epi;
+  const GemmPlan g = plan_qkv(s, R, &epi);
   CUtensorMap wm, xm;
   if (!make_map(&wm, wqkv, s.Kw, s.qkv_rows, s.L, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map(&xm, xb, s.d, R, 1, 64, g.nt, CU_TENSOR_MAP_SWIZZLE_128B))

@@ -94,13 +94,16 @@ __device__ __forceinline__ LmStat lm_shfl_xor(const LmStat& a, int mask) {
 
 // Sum over the 128 lanes of each of the chunk's 16 columns staged as
 // stage[col][lane]: 8 threads per column, 16 lanes each, then a shuffle
-// tree.  Returns the column sum in the thread with (et & 7) == 0.
+// tree.  Returns the column sum in the thread with (et & 7) == 0.  Each
+// thread starts its 16 lanes at a rotation that puts the warp's 32 threads
+// (4 columns x 8 subs) on 32 distinct banks at every step.
 __device__ __forceinline__ float column_sum16(const float* stage, int et) {
   const int col = et >> 3, sub = et & 7;
   const float* cv = stage + col * 128 + sub * 16;
+  const int rot = 4 * (col & 3) + (sub >> 1);
   float s = 0.f;
 #pragma unroll
-  for (int q = 0; q < 16; ++q) s += cv[q];
+  for (int q = 0; q < 16; ++q) s += cv[(q + rot) & 15];
 #pragma unroll
   for (int mask = 1; mask < 8; mask <<= 1) s += __shfl_xor_sync(0xffffffffu, s, mask);
   return s;
@@ -275,8 +278,16 @@ __device__ __forceinline__ void epi_chunk(const GemmParams& p, int m, int n, int
   }
 }
 
+// CTAs per SM the register budget is sized for.  The O-projection runs one
+// CTA per SM (its ring and receive buffer), so its NT = 32 variant may take
+// the registers of two; the Q/K/V projection runs two or three per SM.
 template <int NT, int EPI>
-__global__ void __launch_bounds__(192, NT <= 32 ? 3 : NT <= 64 ? 2 : 1)
+constexpr int gemm_min_blocks() {
+  return (EPI == EPI_OPROJ && NT <= 32) ? 2 : NT <= 32 ? 3 : NT <= 64 ? 2 : 1;
+}
+
+template <int NT, int EPI>
+__global__ void __launch_bounds__(192, gemm_min_blocks<NT, EPI>())
     gemm_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap xmap,
                 const GemmParams p) {
   using C = GemmCfg<NT, EPI>;
@@ -565,9 +576,12 @@ __global__ void __launch_bounds__(192, NT <= 32 ? 3 : NT <= 64 ? 2 : 1)
                         part[q * 16 + 4 * j + 2], part[q * 16 + 4 * j + 3], rbar);
         }
       }
+      // The closing cluster barrier only keeps every CTA alive until the
+      // partials sent to it have landed; the partials themselves are ordered
+      // by red_bar, so the arrivals need no release.
       if (epi && rank < NT / 16) {
         const bool got = mbar_wait_cluster(red_bar, 0, p.status);
-        cluster_arrive();
+        cluster_arrive_relaxed();
         if (got && !flags[0]) {
           int m, n, tile, kb0, kb1;
           decode_unit(p, blockIdx.x, m, n, tile, kb0, kb1);
@@ -607,7 +621,7 @@ __global__ void __launch_bounds__(192, NT <= 32 ? 3 : NT <= 64 ? 2 : 1)
           }
         }
       } else {
-        cluster_arrive();
+        cluster_arrive_relaxed();
       }
       cluster_wait();
     }
