@@ -16,10 +16,11 @@
 //              CTA's vocabulary tiles; logits never leave the SM
 // When (weight tiles x row tiles) would leave SMs idle, K is split: the
 // splits of a tile run as one thread-block cluster, one unit per CTA.  The
-// tile's 16-column chunks are dealt round robin to the ranks; each rank sends
-// its fp32 partials of the chunks it does not own to their owners with
-// st.async (completing on the owner's mbarrier), and every owner adds the
-// partials in rank order and runs the epilogue of its chunks.  The result
+// tile's 16-column chunks are dealt round robin to the ranks; each rank stages
+// its fp32 partials of the chunks it does not own in its idle ring and sends
+// each to its owner with one bulk copy (completing on the owner's mbarrier),
+// and every owner adds the partials in rank order and runs the epilogue of
+// its chunks.  The result
 // does not depend on timing and no partial goes through global memory.
 #include <float.h>
 #include <limits.h>
@@ -59,6 +60,11 @@ struct GemmCfg {
                                       (2 * kStages + 4) * 8 + 64;
   static constexpr size_t kSmem = kSmemBase + kRecvBytes;
   static_assert(kSmem <= 227 * 1024, "GEMM shared memory");
+  // split-K staging of the chunks a rank sends, after the receive buffer when
+  // that sits in the ring
+  static_assert(NT > 64 || EPI == EPI_LMHEAD ||
+                    kRecvBytes + (NT / 16) * 128 * 16 * 4 <= kStages * (kWBytes + kXBytes),
+                "split-K staging must fit in the ring");
 };
 
 __device__ __forceinline__ void decode_unit(const GemmParams& p, int u, int& m, int& n, int& tile,
@@ -544,7 +550,7 @@ __global__ void __launch_bounds__(192, gemm_min_blocks<NT, EPI>())
       // The splits of a tile form one cluster (one unit per CTA).  The tile's
       // 16-column chunks are dealt round robin to the ranks; every rank sends
       // its partial of each chunk it does not own to the owner's receive
-      // buffer with st.async (the bytes complete on the owner's red_bar), and
+      // buffer with a bulk copy (the bytes complete on the owner's red_bar), and
       // each owner adds the partials of its chunks in rank order and runs
       // their epilogue.  The final cluster barrier keeps every CTA alive
       // until the transfers into it have landed.
@@ -561,19 +567,35 @@ __global__ void __launch_bounds__(192, gemm_min_blocks<NT, EPI>())
       const int own = (NT / 16 + sp - 1) / sp;  // chunk slots per owner
       const int sw = (wl >> 1) & 3;              // float4 j of a lane sits at j ^ sw
       if (epi) {
+        // Each chunk this rank does not own is staged in the (idle) ring in
+        // the owner's layout, then sent with one bulk copy.
+        float* stg = reinterpret_cast<float*>(w_st + (p.recv_in_ring ? C::kRecvBytes : 0));
+        int k = 0;
 #pragma unroll
         for (int q = 0; q < NT / 16; ++q) {
-          const int owner = q % sp;
-          if (owner == rank) continue;
-          const int slot = rank < owner ? rank : rank - 1;
-          const uint32_t base =
-              smem_u32(recv + ((size_t)(slot * own + q / sp) * 128 + wl) * 16);
-          const uint32_t rbar = map_to_rank(smem_u32(red_bar), (uint32_t)owner);
+          if (q % sp == rank) continue;
+          float4* row = reinterpret_cast<float4*>(stg + ((size_t)k * 128 + wl) * 16);
 #pragma unroll
           for (int j = 0; j < 4; ++j)
-            st_async_v4(map_to_rank(base + ((j ^ sw) << 4), (uint32_t)owner),
-                        part[q * 16 + 4 * j], part[q * 16 + 4 * j + 1],
-                        part[q * 16 + 4 * j + 2], part[q * 16 + 4 * j + 3], rbar);
+            row[j ^ sw] = make_float4(part[q * 16 + 4 * j], part[q * 16 + 4 * j + 1],
+                                      part[q * 16 + 4 * j + 2], part[q * 16 + 4 * j + 3]);
+          ++k;
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (et == 0) {
+          k = 0;
+#pragma unroll
+          for (int q = 0; q < NT / 16; ++q) {
+            const int owner = q % sp;
+            if (owner == rank) continue;
+            const int slot = rank < owner ? rank : rank - 1;
+            const uint32_t dst = map_to_rank(
+                smem_u32(recv + (size_t)(slot * own + q / sp) * 128 * 16), (uint32_t)owner);
+            bulk_copy_to_cluster(dst, smem_u32(stg + (size_t)k * 128 * 16), 128 * 16 * 4,
+                                 map_to_rank(smem_u32(red_bar), (uint32_t)owner));
+            ++k;
+          }
         }
       }
       // The closing cluster barrier only keeps every CTA alive until the

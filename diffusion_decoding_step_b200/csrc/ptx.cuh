@@ -231,22 +231,6 @@ DLLM_DEV void cluster_arrive_relaxed() {
 }
 DLLM_DEV void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
 DLLM_DEV void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
-// 16-byte store into another CTA's shared memory that completes its bytes
-// on that CTA's mbarrier (both addresses from map_to_rank).
-DLLM_DEV void st_async_v4(uint32_t addr, float a, float b, float c, float d, uint32_t bar) {
-  asm volatile(
-      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::
-          "r"(addr),
-      "f"(a), "f"(b), "f"(c), "f"(d), "r"(bar)
-      : "memory");
-}
-DLLM_DEV void st_async_v2(uint32_t addr, float a, float b, uint32_t bar) {
-  asm volatile(
-      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(
-          addr),
-      "f"(a), "f"(b), "r"(bar)
-      : "memory");
-}
 // Bounded wait on a local mbarrier whose bytes come from other CTAs.
 DLLM_DEV bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, int* status) {
   const unsigned long long t0 = global_ns();
@@ -265,6 +249,14 @@ DLLM_DEV bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, int* status) {
       return false;
     }
   }
+}
+// Bulk copy of `bytes` from this CTA's shared memory into another CTA's
+// (dst and mbar from map_to_rank); the bytes complete on that CTA's mbarrier.
+DLLM_DEV void bulk_copy_to_cluster(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t mbar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(dst), "r"(src), "r"(bytes), "r"(mbar)
+      : "memory");
 }
 // Address of the same shared-memory offset in CTA `rank` of this cluster.
 DLLM_DEV uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
