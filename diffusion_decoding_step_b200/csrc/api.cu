@@ -190,11 +190,16 @@ AttnPlan plan_attn(const Shape& s, int n_rows, int ntile_bound) {
   const int g = s.Hq / s.Hkv;
   a.row_tiles = cdiv(g * n_rows, 128);
   const int base = s.b * s.Hkv * a.row_tiles;
-  // at most 6 key chunks per row tile: the chunks form one cluster and merge on chip
-  int chunks = std::max(1, std::min({ntile_bound, cdiv(kNumSMs, base), 6}));
+  // Key chunks per row tile: the chunks form one cluster and merge on chip.
+  // At most 8 for head_dim 128 and 6 for head_dim 32 (the merge buffer must
+  // fit in the K/V/P region).  Seven head_dim-128 chunks would not fit either,
+  // so they run as eight, the last one without keys.
+  const int cap = s.D == 128 ? 8 : 6;
+  int chunks = std::max(1, std::min({ntile_bound, cdiv(kNumSMs, base), cap}));
   if (base >= kNumSMs) chunks = 1;
   a.tpc = cdiv(ntile_bound, chunks);
   a.chunks = cdiv(ntile_bound, a.tpc);
+  if (a.chunks == 7) a.chunks = 8;
   return a;
 }
 

@@ -32,7 +32,7 @@
 namespace dllm {
 
 constexpr int kKeys = 128;     // keys per tile
-constexpr int kMaxMerge = 6;   // key chunks (cluster size) per row tile
+constexpr int kMaxMerge = 8;   // key chunks (cluster size) per row tile
 
 // 2^x with the SFU instruction (relative error ~2^-22; P is rounded to bf16).
 DLLM_DEV float fast_exp2(float x) {
@@ -70,6 +70,7 @@ static_assert(merge_bytes<128>(2) <= AttnCfg<128, 1>::kRegion &&
                   merge_bytes<128>(4) <= AttnCfg<128, 1>::kRegion &&
                   merge_bytes<128>(5) <= AttnCfg<128, 1>::kRegion &&
                   merge_bytes<128>(6) <= AttnCfg<128, 1>::kRegion &&
+                  merge_bytes<128>(8) <= AttnCfg<128, 1>::kRegion &&
                   merge_bytes<32>(2) <= AttnCfg<32, 1>::kRegion &&
                   merge_bytes<32>(3) <= AttnCfg<32, 1>::kRegion &&
                   merge_bytes<32>(4) <= AttnCfg<32, 1>::kRegion &&
@@ -511,6 +512,7 @@ template <int D, int ST>
 static cudaError_t launch_attn_t(const CUtensorMap& qmap, const CUtensorMap& kmap,
                                  const CUtensorMap& vmap, const AttnParams& p, bool pdl,
                                  cudaStream_t s) {
+  using C_ = AttnCfg<D, ST>;
   auto kern = attn_kernel<D, ST>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.batch * p.Hkv * p.row_tiles * p.chunks);
@@ -524,6 +526,8 @@ static cudaError_t launch_attn_t(const CUtensorMap& qmap, const CUtensorMap& kma
     attr[na].val.programmaticStreamSerializationAllowed = 1;
     ++na;
   }
+  if (p.chunks > kMaxMerge || (p.chunks > 1 && merge_bytes<D>(p.chunks) > C_::kRegion))
+    return cudaErrorInvalidValue;  // the merge buffer would not fit
   if (p.chunks > 1) {  // the chunks of a row tile merge through distributed shared memory
     attr[na].id = cudaLaunchAttributeClusterDimension;
     attr[na].val.clusterDim.x = p.chunks;

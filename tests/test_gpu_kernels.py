@@ -285,6 +285,8 @@ ATTN_CASES = [  # (Hq, Hkv, D, batch, n_rows, S, segs per sequence, layer)
     (28, 4, 128, 1, 32, 640, [[(0, 544), (639, 1)]], 0),   # 6 key chunks
     (28, 4, 128, 1, 32, 1024, [[(5, 539), (0, 0)]], 1),    # 5 chunks of 2 tiles
     (8, 8, 32, 1, 16, 640, [[(0, 600), (0, 0)]], 0),       # head_dim 32, 6 chunks
+    (28, 4, 128, 1, 32, 896, [[(0, 880), (895, 1)]], 0),   # 8 key chunks
+    (28, 4, 128, 1, 32, 768, [[(3, 700), (0, 0)]], 1),     # 7 tiles: 8 chunks, the last empty
 ]
 
 
