@@ -18,6 +18,8 @@ DLLM_CACHE_NONE, DLLM_CACHE_PREFIX, DLLM_CACHE_DUAL, DLLM_CACHE_DUAL_PRUNED = 0,
 DLLM_W_BF16, DLLM_W_F32_SPLIT = 0, 1
 DLLM_COMMIT_THRESHOLD, DLLM_COMMIT_TOPK = 0, 1
 DLLM_DEVICE_TIMEOUT = 1  # status-word bit of a device wait that gave up
+DLLM_DEVICE_BAD_TOKEN = 2  # a token id outside [0, V) reached the embedding gather
+DLLM_DEVICE_INDEX = 4  # DLLM_DEBUG build: a row position from device memory was out of range
 
 
 class DllmError(RuntimeError):

@@ -9,6 +9,9 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libdllm.so")
+# The same sources with DLLM_DEBUG: row positions read from device memory are
+# range-checked in the kernels (an error bit instead of an access).
+LIB_DEBUG = os.path.join(HERE, "libdllm_debug.so")
 SOURCES = ["api.cu", "gemm.cu", "attn.cu", "small.cu"]
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
          "-Xcompiler", "-fPIC", "-shared", "--expt-relaxed-constexpr"]
@@ -21,30 +24,34 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def stale() -> bool:
-    if not os.path.exists(LIB):
+def stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = [os.path.join(CSRC, f) for f in os.listdir(CSRC)]
     deps.append(os.path.join(HERE, "..", "include", "dllm.h"))
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile every CUDA source into libdllm.so next to this file."""
-    if not force and not stale():
-        return LIB
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    """Compile every CUDA source into libdllm.so next to this file (with
+    debug=True: libdllm_debug.so, the DLLM_DEBUG build)."""
+    lib = LIB_DEBUG if debug else LIB
+    if not force and not stale(lib):
+        return lib
     cmd = [nvcc(), *FLAGS]
+    if debug:
+        cmd += ["-DDLLM_DEBUG"]
     if verbose:
         cmd += ["-Xptxas", "-v"]
     cmd += [os.path.join(CSRC, f) for f in SOURCES]
-    tmp = LIB + ".tmp"
+    tmp = lib + ".tmp"
     cmd += ["-o", tmp]
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose="-v" in sys.argv)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv,
+                debug="--debug" in sys.argv))

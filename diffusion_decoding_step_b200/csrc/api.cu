@@ -615,6 +615,7 @@ dllm_status run_final_norm(const Ctx& c, const float* x, int row0, int n_rows, i
   f.plants = static_cast<const __nv_bfloat16*>(plants);
   f.h = static_cast<__nv_bfloat16*>(h);
   f.seq_blk = c.seq_blk;
+  f.status = c.at<int>(c.l.status);
   return cuda_status(launch_final_norm(f, pdl, c.st));
 }
 
@@ -670,6 +671,7 @@ dllm_status run_commit(const Ctx& c, const dllm_state* stt, int blk_start, bool 
   p.tau_seq = stt->tau;
   p.seq_blk = c.seq_blk;
   p.seq_done = c.seq_blk ? c.at<int>(c.l.seqdone) : nullptr;
+  p.status = c.at<int>(c.l.status);
   return cuda_status(launch_commit(p, pdl, c.st));
 }
 

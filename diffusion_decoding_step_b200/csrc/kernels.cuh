@@ -144,6 +144,7 @@ struct FinalNormParams {
   const __nv_bfloat16* plants;
   __nv_bfloat16* h;
   const int* seq_blk;  // per-sequence block starts, or null: blk_start (= row0)
+  int* status;         // device status word, or null
 };
 cudaError_t launch_final_norm(const FinalNormParams& p, bool pdl, cudaStream_t s);
 
@@ -170,6 +171,7 @@ struct CommitParams {
   int* seq_blk;
   int* seq_done;
   const float* tau_seq;  // [b] per-sequence threshold, or null: tau
+  int* status;           // device status word, or null
 };
 cudaError_t launch_commit(const CommitParams& p, bool pdl, cudaStream_t s);
 

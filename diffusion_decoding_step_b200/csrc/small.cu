@@ -32,6 +32,30 @@ static cudaError_t launch_simple(K kern, dim3 grid, dim3 block, bool pdl, cudaSt
   return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
+// ------------------------------------------------------------------ debug checks
+// A DLLM_DEBUG build checks the row positions that come from device memory
+// before they address a buffer.  An out-of-range position sets kErrIndex in
+// the status word, and the CTA skips the access.  The per-sequence block
+// starts of dllm_decode_all are written only by the commit kernel, which
+// checks both what it reads and what it writes, so the projection and
+// attention kernels that read them later get checked values.  Other builds
+// compile the checks away.
+constexpr int kErrIndex = 4;  // status bit beside kErrTimeout and kErrBadArg
+#ifdef DLLM_DEBUG
+constexpr bool kDebugChecks = true;
+#else
+constexpr bool kDebugChecks = false;
+#endif
+// lo <= v < hi, or (DLLM_DEBUG builds only) false with kErrIndex recorded.
+__device__ __forceinline__ bool dbg_in_range(int v, int lo, int hi, int* status) {
+  if constexpr (kDebugChecks) {
+    const bool ok = v >= lo && v < hi;
+    if (!ok && status != nullptr) atomicOr(status, kErrIndex);
+    return ok;
+  }
+  return true;
+}
+
 // ------------------------------------------------------------------ embed
 // Sum of a value over the CTA (blockDim.x a multiple of 32, <= 1024).
 __device__ __forceinline__ float block_sum(float v, float* red) {
@@ -80,6 +104,7 @@ __global__ void __launch_bounds__(256) embed_kernel(const EmbedParams p) {
     o[2] = s1;
     o[3] = l1;
   }
+  if (!dbg_in_range(pos, 0, p.S, p.status)) return;  // uniform over the CTA
   int tok = p.masked[(size_t)b * p.S + pos] ? p.mask_id : p.tokens[(size_t)b * p.S + pos];
   if (tok < 0 || tok >= p.vocab) {  // never read outside the embedding table
     if (threadIdx.x == 0 && p.status) atomicOr(p.status, kErrBadArg);
@@ -128,6 +153,7 @@ __global__ void __launch_bounds__(256) final_norm_kernel(const FinalNormParams p
   const int b = blockIdx.x / p.B, i = blockIdx.x - b * p.B;
   const int blk = p.seq_blk ? p.seq_blk[b] : p.blk_start;
   const int pos = blk + i;
+  if (!dbg_in_range(pos, p.P, p.S, p.status)) return;  // uniform over the CTA
   const float* xr = p.x + ((size_t)b * p.n_rows + (pos - (p.seq_blk ? blk : p.row0))) * p.d;
   float sq = 0.f;
   for (int k = threadIdx.x * 4; k < p.d; k += blockDim.x * 4) {
@@ -238,6 +264,7 @@ __global__ void __launch_bounds__(1024) commit_kernel(const CommitParams p) {
   // two rows per lane (B <= 64)
   const int i0 = lane, i1 = lane + 32;
   const int blk = p.seq_blk ? p.seq_blk[b] : p.blk_start;
+  if (!dbg_in_range(blk, 0, p.S - p.B + 1, p.status)) return;  // uniform over the warp
   const size_t base = (size_t)b * p.S + blk;
   const bool m0 = i0 < p.B && p.masked[base + i0];
   const bool m1 = i1 < p.B && p.masked[base + i1];
@@ -328,7 +355,7 @@ __global__ void __launch_bounds__(1024) commit_kernel(const CommitParams p) {
       int done = p.seq_done[b];
       if (!done && !any_start) {
         if (blk + p.B >= p.S) p.seq_done[b] = done = 1;
-        else p.seq_blk[b] = blk + p.B;
+        else if (dbg_in_range(blk + p.B, 0, p.S - p.B + 1, p.status)) p.seq_blk[b] = blk + p.B;
       }
       if (p.remaining) p.remaining[b] = done ? 0 : 1;
     }

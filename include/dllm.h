@@ -264,7 +264,18 @@ dllm_status dllm_decode_all(const dllm_config* cfg, const dllm_weights* w, const
 dllm_status dllm_step_outputs(const dllm_config* cfg, void* ws, size_t ws_bytes, float** conf,
                               int32_t** tok, float** gap, uint8_t** commit);
 
-/* Copy the workspace's device status word to *code (host); synchronises stream. */
+/* Copy the workspace's device status word to *code (host); synchronises stream.
+ * The word is 0, or an OR of:
+ *  - DLLM_DEVICE_TIMEOUT (1): a bounded device wait gave up (see
+ *    dllm_selftest_wait_timeout); the kernel skipped the rest of its work.
+ *  - DLLM_DEVICE_BAD_TOKEN (2): a token id outside [0, V) reached the
+ *    embedding gather; row 0 of the table was read instead.
+ *  - DLLM_DEVICE_INDEX (4): only in the DLLM_DEBUG build (libdllm_debug.so,
+ *    built by build.py --debug).  A row position read from device memory (a
+ *    per-sequence block start) was outside the sequence, and the access was
+ *    skipped.  The other builds do not check these positions. */
+#define DLLM_DEVICE_BAD_TOKEN 2
+#define DLLM_DEVICE_INDEX 4
 dllm_status dllm_device_status(void* ws, int32_t* code, dllm_stream stream);
 
 /* Number of kernels this library has launched in this process (kernels run

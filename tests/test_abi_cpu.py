@@ -41,6 +41,23 @@ def test_library_exports_every_declared_symbol(lib):
         assert name in abi.SIGNATURES, f"binding lacks {name}"
 
 
+def test_debug_build_exports_every_declared_symbol():
+    """The DLLM_DEBUG build (range checks of device-side row positions) is the
+    same library: it builds and exports the whole ABI."""
+    dbg = C.CDLL(build.build(debug=True))
+    for name in header_functions():
+        assert hasattr(dbg, name), name
+
+
+def test_status_bits_match_the_header():
+    text = open(os.path.join(ROOT, "include", "dllm.h")).read()
+    bits = dict(re.findall(r"#define (DLLM_DEVICE_[A-Z_]+) (\d+)", text))
+    assert set(bits) == {"DLLM_DEVICE_TIMEOUT", "DLLM_DEVICE_BAD_TOKEN", "DLLM_DEVICE_INDEX"}
+    for name, value in bits.items():
+        assert getattr(abi, name) == int(value), name
+    assert len({int(v) for v in bits.values()}) == len(bits)  # distinct bits
+
+
 @pytest.mark.parametrize("name", list(wl.WORKLOADS))
 def test_workspace_size_for_every_workload(lib, name):
     n = C.c_size_t(0)
