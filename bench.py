@@ -85,7 +85,7 @@ def run_profile(args):
         dec.step(w.prompt_len)
     torch.cuda.synchronize()
     n2 = abi.dllm_launch_count()
-    assert dec.device_status() == 0
+    check_clean(dec)
     print(f"profile {w.name} layers={w.n_layers}: launches before warm-up {n0}, "
           f"warm-up {n1 - n0}, timed {n2 - n1} ({(n2 - n1) // max(1, args.steps)} per step)")
 
@@ -177,6 +177,16 @@ def gemm_source_sha1():
         with open(os.path.join(ROOT, "diffusion_decoding_step_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
+
+
+def check_clean(dec, finished=False):
+    """Raise when a device wait gave up or a bad index was seen, or (finished)
+    when a generation left positions masked."""
+    code = dec.device_status()
+    if code != 0:
+        raise RuntimeError(f"device status word {code:#x} after the run")
+    if finished and bool(dec.masked.any()):
+        raise RuntimeError("the generation left masked positions")
 
 
 def max_over_ranks(value, world, device=None):
@@ -371,8 +381,7 @@ def run_ours(args, rank, world, local_rank):
     ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     tokens_total = world * w.batch * w.gen_len * args.steps
     value = tokens_total / (ms / 1000.0)
-    assert dec.device_status() == 0
-    assert not bool(dec.masked.any())
+    check_clean(dec, finished=True)
 
     # prefill share, decode-only rate and per-step latency (separate measurement)
     p0 = torch.cuda.Event(enable_timing=True)

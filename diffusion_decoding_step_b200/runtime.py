@@ -97,8 +97,10 @@ class Decoder:
             self.tau_seq = None
             self.state_c.tau = None
         else:
-            self.tau_seq = torch.tensor(list(tau), dtype=torch.float32, device=self.device)
-            assert self.tau_seq.numel() == self.w.batch
+            vals = [float(t) for t in tau]
+            if len(vals) != self.w.batch:
+                raise ValueError(f"set_tau: {len(vals)} thresholds for {self.w.batch} sequences")
+            self.tau_seq = torch.tensor(vals, dtype=torch.float32, device=self.device)
             self.state_c.tau = _ptr(self.tau_seq)
 
     def prefill(self):

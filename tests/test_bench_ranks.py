@@ -70,3 +70,24 @@ def test_single_rank_is_identity():
     sys.path.insert(0, ROOT)
     import bench
     assert bench.max_over_ranks(3.25, 1) == 3.25
+
+
+class _FakeDecoder:
+    def __init__(self, code, masked):
+        import torch
+        self.code = code
+        self.masked = torch.tensor(masked, dtype=torch.uint8)
+
+    def device_status(self):
+        return self.code
+
+
+def test_clean_run_check():
+    sys.path.insert(0, ROOT)
+    import bench
+    bench.check_clean(_FakeDecoder(0, [0, 0]), finished=True)
+    bench.check_clean(_FakeDecoder(0, [1, 0]))            # mid-run: masked rows are fine
+    with pytest.raises(RuntimeError, match="status word"):
+        bench.check_clean(_FakeDecoder(4, [0, 0]))
+    with pytest.raises(RuntimeError, match="masked"):
+        bench.check_clean(_FakeDecoder(0, [0, 1]), finished=True)
