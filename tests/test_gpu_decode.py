@@ -351,3 +351,4 @@ def test_tau_array_changes_between_steps():
     assert (c1 <= 1).all()
     assert (dec.masked[:, s:s + w.block].cpu().numpy() == 0).all()
     assert (c2 >= 1).all()
+
