@@ -10,6 +10,8 @@
 
 #include <nvtx3/nvToolsExt.h>
 
+#include <float.h>
+
 #include <chrono>
 #include <thread>
 
@@ -83,7 +85,15 @@ dllm_status check_cfg(const dllm_config* c, Shape* s) {
   if (c->commit_mode == DLLM_COMMIT_TOPK &&
       (c->steps_per_block < 1 || c->steps_per_block > c->block))
     return DLLM_ERR_INVALID;
-  if (!(c->tau == c->tau) || c->rope_theta < 0.f) return DLLM_ERR_INVALID;
+  if (!(c->tau == c->tau)) return DLLM_ERR_INVALID;
+  if (!(c->rope_theta >= 0.f && c->rope_theta <= FLT_MAX)) return DLLM_ERR_INVALID;  // NaN, inf
+  // Positions are int32 on the device, and cache and query rows are addressed
+  // with 32-bit offsets in units of head_dim.
+  const long long seq = (long long)c->prompt_len + c->gen_len;
+  if (seq > (1ll << 24)) return DLLM_ERR_UNSUPPORTED;
+  if ((long long)c->n_layers * c->batch * c->n_kv_heads * seq >= (1ll << 31) ||
+      (long long)c->batch * seq * c->n_q_heads >= (1ll << 31))
+    return DLLM_ERR_UNSUPPORTED;
   if (c->head_dim != 32 && c->head_dim != 128) return DLLM_ERR_UNSUPPORTED;
   const int qkv = (c->n_q_heads + 2 * c->n_kv_heads) * c->head_dim;
   if (c->hidden % 128 || (c->n_q_heads * c->head_dim) % 128 || qkv % 128 || c->vocab % 128)

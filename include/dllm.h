@@ -30,7 +30,10 @@
  *    b = batch, L = layers, d = hidden, Hq/Hkv = query/kv heads, D = head_dim,
  *    V = vocab, P = prompt_len, G = gen_len, B = block, S = P + G.
  *  - Supported: D in {32, 128}; d, Hq*D and (Hq+2Hkv)*D multiples of 128;
- *    V a multiple of 128; Hq a multiple of Hkv; B <= 64; b <= 1024.
+ *    V a multiple of 128; Hq a multiple of Hkv; B <= 64; b <= 1024;
+ *    S <= 2^24; L*b*Hkv*S < 2^31 and b*S*Hq < 2^31 (the device addresses cache
+ *    and query rows with 32-bit offsets in units of D).  rope_theta must be
+ *    finite and >= 0 (0: no RoPE); tau must not be NaN.
  *  - Device-side waits are bounded (about 2 s); a wait that gives up sets a bit
  *    in the workspace status word, read with dllm_device_status.
  */

@@ -81,6 +81,19 @@ def test_rejects_bad_configs(lib):
     assert _status(base.replace(vocab=1000, mask_id=5)) == abi.DLLM_ERR_UNSUPPORTED
     assert _status(base.replace(mask_id=2000)) == abi.DLLM_ERR_INVALID
     assert abi.dllm_workspace_size(None, None) == abi.DLLM_ERR_INVALID
+    # rope_theta and tau
+    assert _status(base.replace(rope_theta=float("nan"))) == abi.DLLM_ERR_INVALID
+    assert _status(base.replace(rope_theta=float("inf"))) == abi.DLLM_ERR_INVALID
+    assert _status(base.replace(rope_theta=-1.0)) == abi.DLLM_ERR_INVALID
+    assert _status(base.replace(tau=float("nan"))) == abi.DLLM_ERR_INVALID
+    assert _status(base.replace(tau=float("inf"))) == abi.DLLM_OK   # forced commits only
+    # sizes whose positions or 32-bit row offsets would overflow
+    assert _status(base.replace(prompt_len=2 ** 31 - 64)) == abi.DLLM_ERR_UNSUPPORTED
+    assert _status(base.replace(prompt_len=2 ** 24)) == abi.DLLM_ERR_UNSUPPORTED
+    llada = wl.WORKLOADS["llada8b_dual"]
+    assert _status(llada.replace(batch=1024, prompt_len=65536 - 256)) \
+        == abi.DLLM_ERR_UNSUPPORTED                                      # L*b*Hkv*S >= 2^31
+    assert _status(llada.replace(batch=1024, prompt_len=1024)) == abi.DLLM_OK
 
 
 def test_commit_mode_validation(lib):
