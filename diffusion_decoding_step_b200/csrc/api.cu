@@ -329,7 +329,7 @@ dllm_status make_ctx(const dllm_config* cfg, void* ws, size_t ws_bytes, dllm_str
   if (reinterpret_cast<uintptr_t>(ws) % 256) return DLLM_ERR_INVALID;
   c->ws = static_cast<uint8_t*>(ws);
   c->st = reinterpret_cast<cudaStream_t>(stream);
-  return prepare_device();
+  return DLLM_OK;  // validation only: nothing here touches the device
 }
 
 dllm_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DLLM_OK : DLLM_ERR_CUDA; }
@@ -696,8 +696,14 @@ dllm_status check_state(const Shape& s, const dllm_weights* w, const dllm_state*
   return DLLM_OK;
 }
 
+// [start, start + len) inside [0, limit), in 64-bit so that no int32
+// argument can wrap the test.
+bool rows_ok(long long start, long long len, long long limit) {
+  return start >= 0 && len >= 1 && start + len <= limit;
+}
+
 dllm_status check_block(const Shape& s, int blk) {
-  if (blk < s.P || blk + s.B > s.S || (blk - s.P) % s.B) return DLLM_ERR_INVALID;
+  if (blk < s.P || !rows_ok(blk, s.B, s.S) || (blk - s.P) % s.B) return DLLM_ERR_INVALID;
   return DLLM_OK;
 }
 
@@ -764,6 +770,7 @@ cudaStream_t capture_stream(int device) {
 
 template <class F>
 dllm_status run_graph(const Ctx& c, const GraphKey& key, F&& body) {
+  DLLM_TRY(prepare_device());  // attribute calls may not run inside the capture below
   std::lock_guard<std::mutex> lock(g_graph_mu);
   for (const GraphEntry& e : g_graphs) {
     if (memcmp(&e.key, &key, sizeof(GraphKey)) == 0) {
@@ -854,7 +861,7 @@ dllm_status dllm_embed_rows(const dllm_config* cfg, const dllm_weights* w, const
   Shape s;
   DLLM_TRY(check_cfg(cfg, &s));
   if (!w || !w->embed || !st || !st->tokens || !st->masked || !x || !xb) return DLLM_ERR_INVALID;
-  if (row0 < 0 || n_rows < 1 || row0 + n_rows > s.S) return DLLM_ERR_INVALID;
+  if (!rows_ok(row0, n_rows, s.S)) return DLLM_ERR_INVALID;
   EmbedParams e{};
   e.batch = s.b;
   e.S = s.S;
@@ -883,7 +890,8 @@ dllm_status dllm_final_norm(const dllm_config* cfg, const float* x, int32_t row0
   DLLM_TRY(check_cfg(cfg, &s));
   if (!x || !masked || !plants || !h) return DLLM_ERR_INVALID;
   DLLM_TRY(check_block(s, block_start));
-  if (row0 < 0 || n_rows < 1 || block_start < row0 || block_start + s.B > row0 + n_rows)
+  if (!rows_ok(row0, n_rows, s.S) || block_start < row0 ||
+      (long long)block_start + s.B > (long long)row0 + n_rows)
     return DLLM_ERR_INVALID;
   Ctx c;
   c.s = s;
@@ -899,8 +907,9 @@ dllm_status dllm_qkv_proj(const dllm_config* cfg, const dllm_weights* w, int32_t
   DLLM_TRY(make_ctx(cfg, ws, ws_bytes, stream, &c));
   if (!w || !w->wqkv || !xb || !seq_start || !q_out || !k_cache || !v_cache)
     return DLLM_ERR_INVALID;
-  if (layer < 0 || layer >= c.s.L || row0 < 0 || n_rows < 1 || row0 + n_rows > c.s.S)
+  if (layer < 0 || layer >= c.s.L || !rows_ok(row0, n_rows, c.s.S))
     return DLLM_ERR_INVALID;
+  DLLM_TRY(prepare_device());
   return run_qkv(c, w->wqkv, layer, xb, row_sumsq, row0, n_rows, seq_start, q_out, k_cache,
                  v_cache, false);
 }
@@ -914,6 +923,7 @@ dllm_status dllm_block_attn(const dllm_config* cfg, int32_t layer, int32_t n_row
   if (layer < 0 || layer >= c.s.L || n_rows < 1 || n_rows > c.s.S) return DLLM_ERR_INVALID;
   const int ntb = cdiv(c.s.S, kKeyTile) + 1;
   const AttnKeys keys{segs, nullptr, 0, 0, 0, c.s.S};
+  DLLM_TRY(prepare_device());
   return run_attn(c, layer, n_rows, q, k_cache, v_cache, keys, out, ntb, false);
 }
 
@@ -923,8 +933,9 @@ dllm_status dllm_o_proj(const dllm_config* cfg, const dllm_weights* w, int32_t l
   Ctx c;
   DLLM_TRY(make_ctx(cfg, ws, ws_bytes, stream, &c));
   if (!w || !w->wo || !attn || !x || !xb) return DLLM_ERR_INVALID;
-  if (layer < 0 || layer >= c.s.L || row0 < 0 || n_rows < 1 || row0 + n_rows > c.s.S)
+  if (layer < 0 || layer >= c.s.L || !rows_ok(row0, n_rows, c.s.S))
     return DLLM_ERR_INVALID;
+  DLLM_TRY(prepare_device());
   return run_oproj(c, w->wo, layer, attn, row0, n_rows, x, xb, row_sumsq, false);
 }
 
@@ -935,6 +946,7 @@ dllm_status dllm_lmhead_confidence(const dllm_config* cfg, const dllm_weights* w
   DLLM_TRY(make_ctx(cfg, ws, ws_bytes, stream, &c));
   if (!w || !w->w_lm || !h || !conf || !tok) return DLLM_ERR_INVALID;
   if (n_rows < 1 || n_rows > c.s.b * c.s.B) return DLLM_ERR_INVALID;
+  DLLM_TRY(prepare_device());
   DLLM_TRY(run_lmhead(c, w->w_lm, h, n_rows, false));
   // reduce the per-CTA statistics (one "sequence" of n_rows rows, no commit)
   const GemmPlan g = plan_lmhead(c.s.V, n_rows, c.s.Kw);

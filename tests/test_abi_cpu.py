@@ -118,6 +118,9 @@ def test_null_pointers_rejected_before_launch(lib):
     assert abi.dllm_workspace_init(C.byref(cfg), None, n.value, None) == abi.DLLM_ERR_INVALID
     assert abi.dllm_threshold_commit(C.byref(cfg), 64, None, None, None, None, None, None,
                                      None) == abi.DLLM_ERR_INVALID
+    import torch
+    if torch.cuda.is_available():   # the checks below pass dummy device pointers
+        return
     # misaligned workspace pointer
     assert abi.dllm_workspace_init(C.byref(cfg), C.c_void_p(0x1008), n.value, None) \
         == abi.DLLM_ERR_INVALID
@@ -129,3 +132,36 @@ def test_null_pointers_rejected_before_launch(lib):
 def test_status_strings(lib):
     assert abi.dllm_status_string(0) == b"ok"
     assert b"workspace" in abi.dllm_status_string(abi.DLLM_ERR_WORKSPACE)
+
+
+def test_range_arguments_cannot_wrap(lib):
+    """Row and block ranges are checked in 64-bit before anything touches the
+    device: int32 arguments near 2^31 that would wrap an int32 sum are
+    rejected.  Every call here must fail validation, so the dummy pointers
+    are never used (no call in this test may pass it)."""
+    import torch
+    if torch.cuda.is_available():   # a regression would launch on the dummy pointers
+        pytest.skip("dummy device pointers: runs only where no GPU is visible")
+    w = wl.WORKLOADS["llada8b_dual"]           # P 256, B 32, S 512
+    cfg = C.byref(make_config(w))
+    n = C.c_size_t(0)
+    assert abi.dllm_workspace_size(cfg, C.byref(n)) == abi.DLLM_OK
+    d = C.c_void_p(1 << 20)                    # aligned, never dereferenced
+    weights = C.byref(abi.dllm_weights(d, d, d, d))
+    state = C.byref(abi.dllm_state(d, d, d, d, d, d, None))
+    big = 2 ** 31 - 32                         # (big - P) % B == 0; big + B wraps
+    bad = abi.DLLM_ERR_INVALID
+    assert abi.dllm_decode_step(cfg, weights, state, big, d, n.value, None) == bad
+    assert abi.dllm_kv_cache_refresh(cfg, weights, state, big, d, n.value, None) == bad
+    steps = C.c_int32(0)
+    assert abi.dllm_decode_block(cfg, weights, state, big, 0, C.byref(steps), d, n.value,
+                                 None) == bad
+    assert abi.dllm_threshold_commit(cfg, big, d, d, d, d, None, None, None) == bad
+    assert abi.dllm_embed_rows(cfg, weights, state, big, 64, d, d, None, None) == bad
+    assert abi.dllm_final_norm(cfg, d, big, 64, 256, d, d, d, None) == bad
+    assert abi.dllm_final_norm(cfg, d, 0, 512, big, d, d, d, None) == bad
+    assert abi.dllm_qkv_proj(cfg, weights, 0, d, None, big, 64, d, d, d, d, d, n.value,
+                             None) == bad
+    assert abi.dllm_o_proj(cfg, weights, 0, d, big, 64, d, d, None, d, n.value, None) == bad
+    assert abi.dllm_qkv_proj(cfg, weights, 0, d, None, 0, 2 ** 31 - 1, d, d, d, d, d, n.value,
+                             None) == bad
