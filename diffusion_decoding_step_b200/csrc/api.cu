@@ -291,10 +291,10 @@ Layout layout(const Shape& s) {
 
 // ------------------------------------------------------------------ context
 struct Ctx {
-  Shape s;
-  Layout l;
-  uint8_t* ws;
-  cudaStream_t st;
+  Shape s{};
+  Layout l{};
+  uint8_t* ws = nullptr;  // null for entry points that take no workspace
+  cudaStream_t st = nullptr;
   // per-sequence block starts in the workspace (dllm_decode_all), or null:
   // every sequence is at the block the call names
   int* seq_blk = nullptr;
@@ -625,7 +625,7 @@ dllm_status run_final_norm(const Ctx& c, const float* x, int row0, int n_rows, i
   f.plants = static_cast<const __nv_bfloat16*>(plants);
   f.h = static_cast<__nv_bfloat16*>(h);
   f.seq_blk = c.seq_blk;
-  f.status = c.at<int>(c.l.status);
+  f.status = c.ws ? c.at<int>(c.l.status) : nullptr;
   return cuda_status(launch_final_norm(f, pdl, c.st));
 }
 
@@ -681,7 +681,7 @@ dllm_status run_commit(const Ctx& c, const dllm_state* stt, int blk_start, bool 
   p.tau_seq = stt->tau;
   p.seq_blk = c.seq_blk;
   p.seq_done = c.seq_blk ? c.at<int>(c.l.seqdone) : nullptr;
-  p.status = c.at<int>(c.l.status);
+  p.status = c.ws ? c.at<int>(c.l.status) : nullptr;
   return cuda_status(launch_commit(p, pdl, c.st));
 }
 
