@@ -4,7 +4,7 @@
  * The method (Fast-dLLM v1): a block of masked positions is denoised in
  * parallel; each step every masked position gets the max-softmax confidence
  * and argmax token of the LM head, and every position whose confidence
- * clears the threshold tau is committed ("Fast-dLLM: Four Acceleration Tracks
+ * exceeds the threshold tau is committed ("Fast-dLLM: Four Acceleration Tracks
  * for Diffusion Language Models...", section "The v1 Mechanism: KV Cache Plus
  * Confidence-Threshold Parallel Decoding").  A key/value cache holds the
  * attention state of settled positions (same section; Fast-dLLM README,

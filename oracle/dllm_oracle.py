@@ -10,7 +10,7 @@ What it computes (sources, by page title and section):
   v1 decodes with "KV Cache + Parallel Decoding" on Dream/LLaDA backbones.
 * "Fast-dLLM: Four Acceleration Tracks ...", section "The v1 Mechanism":
   every masked position of the block is evaluated in parallel, the ones whose
-  confidence clears the threshold are committed, a committed token is never
+  confidence exceeds the threshold are committed, a committed token is never
   revised, and a key/value cache keeps the attention state of settled
   positions so that it is not recomputed.
 * Same page, section "Fast-dLLM v1 Versus a Standard Diffusion Sampler":
@@ -22,11 +22,11 @@ What it computes (sources, by page title and section):
   the trailing position.
 
 The pages give no formulas.  Where they are silent this module takes the
-plainest reading, and every such reading is listed in the design notes:
+plainest reading that the rest supports:
 textbook scaled-dot-product softmax attention with scale 1/sqrt(D) and
 contiguous GQA groups; rotate-half rotary embedding; confidence = the largest
 softmax probability over the whole vocabulary; argmax ties go to the lowest
-id; "clears the threshold" is strict ``conf > tau``; at least the single most
+id; the threshold test is strict ``conf > tau``; at least the single most
 confident masked row commits each step (lowest position on ties); the key set
 per cache mode is given by :func:`key_positions`.
 
