@@ -12,7 +12,7 @@ LIB = os.path.join(HERE, "libdllm.so")
 # The same sources with DLLM_DEBUG: row positions read from device memory are
 # range-checked in the kernels (an error bit instead of an access).
 LIB_DEBUG = os.path.join(HERE, "libdllm_debug.so")
-SOURCES = ["api.cu", "gemm.cu", "attn.cu", "small.cu"]
+SOURCES = ["api.cu", "gemm.cu", "attn.cu", "small.cu", "stack.cu"]
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
          "-Xcompiler", "-fPIC", "-shared", "--expt-relaxed-constexpr"]
 

@@ -231,11 +231,91 @@ int key_tiles_bound(const Shape& s, int blk, int seg_end) {
   }
 }
 
+// ------------------------------------------------------------------ layer stack
+// Plan of the persistent layer-stack kernel (csrc/stack.cu) for a step or a
+// refresh of n_rows rows per sequence at block blk.  Shape conditions only;
+// whether the kernel is used at run time also depends on the device and on
+// dllm_set_layer_stack.
+struct StackPlan {
+  bool ok = false;
+  int nt = 0, grid = 0, qt = 0, ot = 0, qkbt = 0, okbt = 0, qn = 0, on = 0, qmaxc = 0, omaxc = 0;
+  int rt = 0, chunks = 0, tpc = 0, units = 0, fs = 0;
+};
+constexpr int kStackMinSeg = 2;  // k-blocks a CTA's share holds at least
+
+// 64-key attention tiles of the widest sequence (sequence start 0).
+int stack_key_tiles(const Shape& s, int blk) {
+  const int end = blk + s.B;
+  if (s.mode == DLLM_CACHE_DUAL) return cdiv(s.S, 64);
+  if (s.mode == DLLM_CACHE_DUAL_PRUNED) {
+    const int wend = std::min(end + s.W, s.S);
+    return cdiv(wend, 64) + ((end < s.S && s.S - 1 >= wend) ? 1 : 0);
+  }
+  return cdiv(end, 64);
+}
+
+// Largest number of contributors (CTA shares) of one tile.
+int stack_maxc(int tiles, int kbt, int n) {
+  const long long T = (long long)tiles * kbt;
+  int mx = 0;
+  for (int t = 0; t < tiles; ++t) {
+    const int ca = stack_owner((long long)t * kbt, n, T);
+    const int cb = stack_owner((long long)t * kbt + kbt - 1, n, T);
+    mx = std::max(mx, cb - ca + 1);
+  }
+  return mx;
+}
+
+StackPlan plan_stack(const Shape& s, int n_rows, int blk, int grid) {
+  StackPlan P;
+  if (grid < 1 || s.D != 128 || s.wfmt != DLLM_W_BF16) return P;
+  if (s.mode != DLLM_CACHE_PREFIX && s.mode != DLLM_CACHE_DUAL && s.mode != DLLM_CACHE_DUAL_PRUNED)
+    return P;
+  const int R = s.b * n_rows;
+  if (R < 1 || R > 64) return P;
+  P.nt = R <= 32 ? 32 : 64;
+  P.grid = grid;
+  P.qt = s.qkv_rows / 128;
+  P.ot = s.d / 128;
+  P.qkbt = s.Kw / 64;
+  P.okbt = s.Ko / 64;
+  P.qn = std::min(grid, std::max(1, P.qt * P.qkbt / kStackMinSeg));
+  P.on = std::min(grid, std::max(1, P.ot * P.okbt / kStackMinSeg));
+  StackSeg tmp[kStackMaxSeg];
+  for (int c = 0; c < P.qn; ++c)
+    if (stack_segments(c, P.qt, P.qkbt, P.qn, tmp, kStackMaxSeg) < 0) return P;
+  for (int c = 0; c < P.on; ++c)
+    if (stack_segments(c, P.ot, P.okbt, P.on, tmp, kStackMaxSeg) < 0) return P;
+  P.qmaxc = stack_maxc(P.qt, P.qkbt, P.qn);
+  P.omaxc = stack_maxc(P.ot, P.okbt, P.on);
+  const int g = s.Hq / s.Hkv;
+  P.rt = cdiv(g * n_rows, 128);
+  // key chunks of a row tile: a power of two (each finishes D/chunks columns
+  // of the merge) that keeps at most two 64-key tiles per chunk, fewer when
+  // the units would outnumber the CTAs (one unit per CTA and layer)
+  const int nt64 = stack_key_tiles(s, blk);
+  int chunks = 1;
+  while (chunks < 16 && cdiv(nt64, chunks) > 2) chunks *= 2;
+  while (chunks > 1 && s.b * s.Hkv * P.rt * chunks > grid) chunks /= 2;
+  P.chunks = chunks;
+  P.tpc = cdiv(nt64, chunks);
+  P.units = s.b * s.Hkv * P.rt * chunks;
+  if (P.units > grid) return P;
+  // counters of one layer, each on its own 128-byte line (32 ints)
+  P.fs = 32 * (2 * P.qt + 2 * P.ot + s.b * s.Hkv * P.rt + s.Hkv);
+  P.ok = true;
+  return P;
+}
+
 // ------------------------------------------------------------------ workspace
 struct Layout {
   size_t status, stepc, seqblk, seqdone, x, xb, sumsq, q, attn, h, stats, conf, tok, gap, commit,
       remaining, segs, rope, total;
   int rmax, lm_slots;
+  // layer-stack kernel: flags, split-K partials, attention chunk partials
+  size_t stk_flags, stk_qpart, stk_opart, stk_apart, stk_aml;
+  long long stk_nflags;  // ints of flags reserved (0: the shape never uses the kernel)
+  int stk_chunks;        // key chunks the attention partials are sized for
 };
 
 // Row counts (per sequence) a configuration uses: decode steps and prefill.
@@ -285,6 +365,23 @@ Layout layout(const Shape& s) {
   l.remaining = take((size_t)s.b * 4);
   l.segs = take((size_t)s.b * 16);
   l.rope = take(s.theta > 0.f ? (size_t)s.S * (s.D / 2) * 8 : 256);
+  // the layer-stack kernel runs steps and refreshes of b*B rows; its scratch
+  // is sized for the widest key set over the blocks
+  StackPlan sp{};
+  for (int blk = s.P; blk < s.S; blk += s.B) {
+    const StackPlan q = plan_stack(s, s.B, blk, kNumSMs);
+    if (q.ok && (!sp.ok || q.chunks > sp.chunks)) sp = q;
+  }
+  if (sp.ok) {
+    l.stk_nflags = (long long)s.L * sp.fs + 32;  // then the abort word
+    l.stk_chunks = sp.chunks;
+    l.stk_flags = take((size_t)l.stk_nflags * 4);
+    l.stk_qpart = take((size_t)sp.qt * sp.qmaxc * sp.nt * 128 * 4);
+    l.stk_opart = take((size_t)sp.ot * sp.omaxc * sp.nt * 128 * 4);
+    const size_t slots = (size_t)s.b * s.Hkv * sp.rt * sp.chunks;
+    l.stk_apart = take(slots * 128 * 128 * 4);
+    l.stk_aml = take(slots * 128 * 8);
+  }
   l.total = off;
   return l;
 }
@@ -304,6 +401,14 @@ struct Ctx {
   }
 };
 
+// Process-wide switches of the layer-stack kernel (dllm_set_layer_stack).
+struct StackTune {
+  bool enable = false;  // measured slower than the per-projection kernels (see the header)
+  int lookahead = 16;   // weight k-blocks prefetched into L2 beyond the ring
+};
+StackTune g_stack_tune;
+bool g_stack_dev_ok[64] = {};
+
 // One-time per-device setup that must not run inside a graph capture:
 // kernel shared-memory attributes and the tensor-map encoder entry point.
 dllm_status prepare_device() {
@@ -313,10 +418,27 @@ dllm_status prepare_device() {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DLLM_ERR_CUDA;
   std::lock_guard<std::mutex> lock(mu);
   if (done[dev]) return DLLM_OK;
-  if (!encode_fn() || gemm_prepare() != cudaSuccess || attn_prepare() != cudaSuccess)
+  if (!encode_fn() || gemm_prepare() != cudaSuccess || attn_prepare() != cudaSuccess ||
+      stack_prepare() != cudaSuccess)
     return DLLM_ERR_CUDA;
+  // The layer-stack kernel's CTAs wait on one another, so all of them must be
+  // resident at once: one CTA on each of kNumSMs SMs.
+  int sms = 0, per_sm32 = 0, per_sm64 = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      stack_occupancy(32, &per_sm32) != cudaSuccess || stack_occupancy(64, &per_sm64) != cudaSuccess)
+    return DLLM_ERR_CUDA;
+  g_stack_dev_ok[dev] = sms >= kNumSMs && per_sm32 >= 1 && per_sm64 >= 1;
   done[dev] = true;
   return DLLM_OK;
+}
+
+// The layer-stack kernel runs on the current device (prepared above) and is
+// switched on (dllm_set_layer_stack).
+bool stack_usable() {
+  int dev = 0;
+  if (!g_stack_tune.enable || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+    return false;
+  return g_stack_dev_ok[dev];
 }
 
 dllm_status make_ctx(const dllm_config* cfg, void* ws, size_t ws_bytes, dllm_stream stream,
@@ -510,7 +632,8 @@ dllm_status run_attn(const Ctx& c, int layer, int n_rows, const void* q, const v
 }
 
 dllm_status run_embed(const Ctx& c, const dllm_weights* w, const dllm_state* stt, int row0,
-                      int n_rows, int blk_start, int seg_end, bool pdl) {
+                      int n_rows, int blk_start, int seg_end, bool pdl, int* zero = nullptr,
+                      long long nzero = 0) {
   const Shape& s = c.s;
   EmbedParams e{};
   e.batch = s.b;
@@ -537,6 +660,8 @@ dllm_status run_embed(const Ctx& c, const dllm_weights* w, const dllm_state* stt
   e.mode = s.mode;
   e.window = s.W;
   e.seg_end = seg_end;
+  e.zero = zero;
+  e.nzero = (int)nzero;
   return cuda_status(launch_embed(e, pdl, c.st));
 }
 
@@ -556,11 +681,122 @@ PrefetchTune g_pf_tune;
 
 long long round16(long long v) { return v < 0 ? 0 : v & ~15ll; }
 
+// All L layers of n_rows rows per sequence at row0 (the block) in one
+// launch of the layer-stack kernel.  The embedding kernel before it clears
+// the kernel's flags.
+dllm_status run_stack(const Ctx& c, const dllm_weights* w, const dllm_state* stt, int row0,
+                      int n_rows, int blk_start, const StackPlan& P) {
+  const Shape& s = c.s;
+  const int R = s.b * n_rows;
+  const int g = s.Hq / s.Hkv;
+  void* xb = c.at<void>(c.l.xb);
+  void* q = c.at<void>(c.l.q);
+  void* attn = c.at<void>(c.l.attn);
+  const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
+  CUtensorMap m[7];
+  if (!make_map(&m[0], w->wqkv, s.Kw, s.qkv_rows, s.L, 64, 128, sw) ||
+      !make_map(&m[1], w->wo, s.Ko, s.d, s.L, 64, 128, sw) ||
+      !make_map(&m[2], xb, s.d, R, 1, 64, P.nt, sw) ||
+      !make_map(&m[3], attn, s.Hq * s.D, R, 1, 64, P.nt, sw) ||
+      !make_map(&m[4], q, s.D, (uint64_t)g * n_rows, (uint64_t)s.b * s.Hkv, 64, 128, sw) ||
+      !make_map(&m[5], stt->k_cache, s.D, s.S, (uint64_t)s.L * s.b * s.Hkv, 64, 64, sw) ||
+      !make_map(&m[6], stt->v_cache, s.D, s.S, (uint64_t)s.L * s.b * s.Hkv, 64, 64, sw))
+    return DLLM_ERR_CUDA;
+  StackParams p{};
+  p.L = s.L;
+  p.R = R;
+  p.n_rows = n_rows;
+  p.batch = s.b;
+  p.Hq = s.Hq;
+  p.Hkv = s.Hkv;
+  p.S = s.S;
+  p.d = s.d;
+  p.g = g;
+  p.qt = P.qt;
+  p.ot = P.ot;
+  p.qkbt = P.qkbt;
+  p.okbt = P.okbt;
+  p.qn = P.qn;
+  p.on = P.on;
+  p.qmaxc = P.qmaxc;
+  p.omaxc = P.omaxc;
+  p.rt = P.rt;
+  p.chunks = P.chunks;
+  p.tpc = P.tpc;
+  p.units = P.units;
+  p.mode = s.mode;
+  p.blk_start = blk_start;
+  p.blk_len = s.B;
+  p.window = s.W;
+  p.seg_end = 0;
+  p.dep_lo = row0;
+  p.dep_hi = row0 + n_rows;
+  p.lookahead = g_stack_tune.lookahead;
+  p.seq_start = stt->seq_start;
+  p.q = static_cast<__nv_bfloat16*>(q);
+  p.attn = static_cast<__nv_bfloat16*>(attn);
+  p.qpart = c.at<float>(c.l.stk_qpart);
+  p.opart = c.at<float>(c.l.stk_opart);
+  p.apart = c.at<float>(c.l.stk_apart);
+  p.aml = c.at<float2>(c.l.stk_aml);
+  p.flags = c.at<int>(c.l.stk_flags);
+  p.fs = P.fs;
+  p.status = c.at<int>(c.l.status);
+  p.scale_log2 = 1.4426950408889634f / sqrtf((float)s.D);
+  // epilogue of the Q/K/V projection: RMS scale, RoPE, q and the cache rows
+  GemmParams& gq = p.gq;
+  gq.M = s.qkv_rows;
+  gq.R = R;
+  gq.K = s.Kw;
+  gq.layer = 0;
+  gq.status = p.status;
+  gq.n_rows = n_rows;
+  gq.row0 = row0;
+  gq.seq_start = stt->seq_start;
+  gq.Hq = s.Hq;
+  gq.Hkv = s.Hkv;
+  gq.D = s.D;
+  gq.S = s.S;
+  gq.batch = s.b;
+  gq.rope_tab = s.theta > 0.f ? c.at<float2>(c.l.rope) : nullptr;
+  gq.q_out = p.q;
+  gq.k_cache = static_cast<__nv_bfloat16*>(stt->k_cache);
+  gq.v_cache = static_cast<__nv_bfloat16*>(stt->v_cache);
+  gq.sumsq_in = c.at<float>(c.l.sumsq);
+  gq.npart = s.d / 128;
+  gq.d_norm = s.d;
+  gq.rms_eps = kRmsEps;
+  // epilogue of the O-projection: residual, its bf16 copy, sums of squares
+  GemmParams& go = p.go;
+  go.M = s.d;
+  go.R = R;
+  go.K = s.Ko;
+  go.status = p.status;
+  go.n_rows = n_rows;
+  go.row0 = row0;
+  go.x = c.at<float>(c.l.x);
+  go.xb = static_cast<__nv_bfloat16*>(xb);
+  go.d_model = s.d;
+  go.sumsq_out = c.at<float>(c.l.sumsq);
+  go.npart = s.d / 128;
+  go.d_norm = s.d;
+  return cuda_status(launch_stack(P.nt, m, p, P.grid, true, c.st));
+}
+
 // Embed + L pre-norm layers for n_rows rows per sequence at row0.  lm_next:
 // the LM head follows the last layer.
 dllm_status run_forward(const Ctx& c, const dllm_weights* w, const dllm_state* stt, int row0,
                         int n_rows, int blk_start, int seg_end, bool lm_next) {
   const Shape& s = c.s;
+  if (c.seq_blk == nullptr && seg_end == 0 && row0 == blk_start && c.l.stk_nflags > 0 &&
+      stack_usable()) {
+    const StackPlan P = plan_stack(s, n_rows, blk_start, kNumSMs);
+    if (P.ok && (long long)s.L * P.fs + 32 <= c.l.stk_nflags && P.chunks <= c.l.stk_chunks) {
+      DLLM_TRY(run_embed(c, w, stt, row0, n_rows, blk_start, seg_end, true,
+                         c.at<int>(c.l.stk_flags), (long long)s.L * P.fs + 32));
+      return run_stack(c, w, stt, row0, n_rows, blk_start, P);
+    }
+  }
   DLLM_TRY(run_embed(c, w, stt, row0, n_rows, blk_start, seg_end, true));
   int ntb = key_tiles_bound(s, blk_start, seg_end);
   if (c.seq_blk)  // each sequence at its own block: plan for the widest key set
@@ -1129,6 +1365,65 @@ dllm_status dllm_set_l2_prefetch(int64_t attn_next_bytes, int64_t oproj_next_byt
   g_pf_tune.oproj_next = oproj_next_bytes;
   g_pf_tune.attn_wo = attn_prefetch_wo != 0;
   dllm_graph_cache_clear();  // cached graphs hold the old prefetch ranges
+  return DLLM_OK;
+}
+
+dllm_status dllm_set_layer_stack(int32_t enable, int32_t l2_lookahead) {
+  if (l2_lookahead < 0 || l2_lookahead > 4096) return DLLM_ERR_INVALID;
+  g_stack_tune.enable = enable != 0;
+  g_stack_tune.lookahead = l2_lookahead;
+  dllm_graph_cache_clear();
+  return DLLM_OK;
+}
+
+dllm_status dllm_layer_stack_plan(const dllm_config* cfg, int32_t block_start, int32_t* info) {
+  Shape s;
+  DLLM_TRY(check_cfg(cfg, &s));
+  if (!info) return DLLM_ERR_INVALID;
+  DLLM_TRY(check_block(s, block_start));
+  const StackPlan P = plan_stack(s, s.B, block_start, kNumSMs);
+  for (int i = 0; i < 8; ++i) info[i] = 0;
+  if (!P.ok) return DLLM_OK;
+  info[0] = 1;
+  info[1] = P.nt;
+  info[2] = P.qn;
+  info[3] = P.on;
+  info[4] = P.chunks;
+  info[5] = P.tpc;
+  info[6] = P.units;
+  // every k-block of every tile belongs to exactly one segment, and the
+  // segments of a tile are numbered 0..nc-1 in k order
+  bool good = true;
+  for (int ph = 0; ph < 2 && good; ++ph) {
+    const int tiles = ph ? P.ot : P.qt, kbt = ph ? P.okbt : P.qkbt, n = ph ? P.on : P.qn;
+    const int maxc = ph ? P.omaxc : P.qmaxc;
+    std::vector<int> owner((size_t)tiles * kbt, -1), nc(tiles, -1), next(tiles, 0);
+    for (int c = 0; c < n && good; ++c) {
+      StackSeg sg[kStackMaxSeg];
+      const int k = stack_segments(c, tiles, kbt, n, sg, kStackMaxSeg);
+      if (k < 1) good = false;
+      for (int i = 0; i < k && good; ++i) {
+        const StackSeg& g = sg[i];
+        if (g.tile < 0 || g.tile >= tiles || g.kb0 < 0 || g.kb1 > kbt || g.kb0 >= g.kb1 ||
+            g.nc < 1 || g.nc > maxc || g.ci != next[g.tile] || (nc[g.tile] >= 0 && nc[g.tile] != g.nc))
+          good = false;
+        if (!good) break;
+        nc[g.tile] = g.nc;
+        ++next[g.tile];
+        for (int kb = g.kb0; kb < g.kb1; ++kb) {
+          int& o = owner[(size_t)g.tile * kbt + kb];
+          if (o >= 0) good = false;
+          o = c;
+        }
+      }
+    }
+    for (int t = 0; t < tiles && good; ++t) {
+      if (next[t] != nc[t]) good = false;
+      for (int kb = 0; kb < kbt; ++kb)
+        if (owner[(size_t)t * kbt + kb] < 0) good = false;
+    }
+  }
+  info[7] = good ? 1 : 0;
   return DLLM_OK;
 }
 

@@ -106,12 +106,90 @@ __device__ __forceinline__ void l2_prefetch_share(const L2Prefetch& pf, int cta,
 }
 #endif
 
+// ---------------------------------------------------------------- layer stack
+// The persistent layer-stack kernel runs every layer of a step (or of a
+// refresh) in one launch, one CTA per SM.  Each GEMM phase (Q/K/V, O-proj)
+// flattens its (weight tile, 64-wide k-block) space and gives each of `n`
+// CTAs one contiguous, equal share (stream-K); a share that crosses a tile
+// boundary is cut into one segment per tile.  The segments of a tile are its
+// contributors, numbered in k order.
+struct StackSeg {
+  int tile, kb0, kb1, ci, nc;  // tile, k-block range, contributor index, contributors
+};
+constexpr int kStackMaxSeg = 4;  // segments per CTA and phase
+
+__host__ __device__ inline long long stack_lo(int c, int n, long long T) {
+  return (long long)c * T / n;
+}
+// The CTA whose share holds k-block kb (0 <= kb < T).
+__host__ __device__ inline int stack_owner(long long kb, int n, long long T) {
+  return (int)(((kb + 1) * n + T - 1) / T) - 1;
+}
+// Segments of CTA c; returns their count, or -1 if more than maxs are needed.
+__host__ __device__ inline int stack_segments(int c, int tiles, int kbt, int n, StackSeg* out,
+                                              int maxs) {
+  if (c >= n) return 0;
+  const long long T = (long long)tiles * kbt;
+  long long a = stack_lo(c, n, T);
+  const long long e = stack_lo(c + 1, n, T);
+  int k = 0;
+  while (a < e) {
+    if (k == maxs) return -1;
+    const int t = (int)(a / kbt);
+    const long long tb = (long long)t * kbt;
+    const long long b = e < tb + kbt ? e : tb + kbt;
+    const int ca = stack_owner(tb, n, T);
+    const int cb = stack_owner(tb + kbt - 1, n, T);
+    out[k].tile = t;
+    out[k].kb0 = (int)(a - tb);
+    out[k].kb1 = (int)(b - tb);
+    out[k].ci = c - ca;
+    out[k].nc = cb - ca + 1;
+    ++k;
+    a = b;
+  }
+  return k;
+}
+
+struct StackParams {
+  int L, R, n_rows, batch, Hq, Hkv, S, d, g;
+  int qt, ot;      // weight tiles of the Q/K/V and O-projection GEMMs
+  int qkbt, okbt;  // k-blocks (64 wide) per tile
+  int qn, on;      // CTAs sharing each phase
+  int qmaxc, omaxc;  // contributor slots per tile in the partial buffers
+  // attention: row tiles and key chunks per (sequence, kv head), 64-key
+  // tiles per chunk, units per layer
+  int rt, chunks, tpc, units;
+  int mode, blk_start, blk_len, window, seg_end, dep_lo, dep_hi;
+  int lookahead;   // weight k-blocks prefetched into L2 beyond the ring
+  const int* seq_start;
+  __nv_bfloat16* q;     // [b][Hq][n_rows][D]
+  __nv_bfloat16* attn;  // [b*n_rows][Hq*D]
+  float* qpart;         // [qt][qmaxc][NT][128] fp32 split-K partials
+  float* opart;         // [ot][omaxc][NT][128]
+  float* apart;         // [b*Hkv*rt][chunks][D][128] unnormalised attention outputs
+  float2* aml;          // [b*Hkv*rt][chunks][128] (running max in log2 units, sum)
+  int* flags;           // fs ints per layer, then the abort word
+  int fs;
+  int* status;
+  float scale_log2;
+  GemmParams gq, go;    // epilogue parameters of the two projections
+};
+
 // Launch helpers (return cudaError_t of the launch).
 cudaError_t launch_gemm(int epi, int nt, const CUtensorMap& wmap, const CUtensorMap& xmap,
                         const GemmParams& p, int grid, bool pdl, cudaStream_t s);
 cudaError_t gemm_prepare();
 cudaError_t attn_prepare();
 cudaError_t launch_wait_timeout(int* status, long long limit_ns, cudaStream_t s);
+
+// Layer-stack kernel (csrc/stack.cu): maps for W_qkv, W_o, xb, the attention
+// output, q, and the K/V caches (64-key boxes).
+cudaError_t stack_prepare();
+size_t stack_smem_bytes(int nt);
+cudaError_t stack_occupancy(int nt, int* blocks_per_sm);
+cudaError_t launch_stack(int nt, const CUtensorMap* maps, const StackParams& p, int grid,
+                         bool pdl, cudaStream_t s);
 
 cudaError_t launch_attn(int head_dim, const CUtensorMap& qmap, const CUtensorMap& kmap,
                         const CUtensorMap& vmap, const AttnParams& p, bool pdl,
@@ -132,6 +210,9 @@ struct EmbedParams {
   const int* seq_start;
   int mode, window, seg_end;  // seg_end: end of the key range for prefill/none
   const int* seq_blk;  // per-sequence block starts (rows start there), or null: row0 / blk_start
+  // optional: ints cleared before the next kernel (the layer-stack kernel's flags)
+  int* zero;
+  int nzero;
 };
 cudaError_t launch_embed(const EmbedParams& p, bool pdl, cudaStream_t s);
 

@@ -78,6 +78,8 @@ __global__ void __launch_bounds__(256) embed_kernel(const EmbedParams p) {
   grid_dep_wait();
   grid_dep_launch();
   const int row = blockIdx.x;
+  for (int i = row * blockDim.x + threadIdx.x; i < p.nzero; i += gridDim.x * blockDim.x)
+    p.zero[i] = 0;
   const int b = row / p.n_rows;
   const int pos = (p.seq_blk ? p.seq_blk[b] : p.row0) + (row - b * p.n_rows);
   for (int bb = threadIdx.x; row == 0 && p.segs != nullptr && bb < p.batch; bb += blockDim.x) {

@@ -303,6 +303,29 @@ void dllm_graph_cache_clear(void);
 dllm_status dllm_set_l2_prefetch(int64_t attn_next_bytes, int64_t oproj_next_bytes,
                                  int32_t attn_prefetch_wo);
 
+/* Persistent layer-stack kernel (a scheduling choice with no counterpart on
+ * the pages; results follow the same definitions).  Off by default: on the
+ * 8B-shaped workloads it measured 1.8-2x slower than the per-projection
+ * kernels, because each hand-off between CTAs through global memory costs
+ * more than a kernel boundary.  When switched on,
+ * a decode step or a block refresh whose b*B rows fit 64 activation rows,
+ * with head_dim 128, bf16 weights and a PREFIX, DUAL or DUAL_PRUNED cache,
+ * runs all L layers in one launch with one CTA per SM (the device must have
+ * at least 148 SMs; otherwise, and for every other shape, the per-projection
+ * kernels run).  l2_lookahead: weight k-blocks (16 KB each) per CTA that the
+ * kernel prefetches into L2 ahead of its shared-memory ring (0..4096,
+ * default 16).  Process-wide; clears the graph cache.  enable = 0 restores
+ * the default. */
+dllm_status dllm_set_layer_stack(int32_t enable, int32_t l2_lookahead);
+
+/* Host query (no GPU work): the layer-stack plan of a step of the block at
+ * block_start.  info (host, 8 ints): [0] 1 if the shape qualifies, [1]
+ * activation tile width, [2]/[3] CTAs sharing the Q/K/V / O-projection
+ * weights, [4] key chunks per attention row tile, [5] 64-key tiles per chunk,
+ * [6] attention units per layer, [7] 1 if every weight k-block of every
+ * tile belongs to exactly one CTA share (a self-check of the partition). */
+dllm_status dllm_layer_stack_plan(const dllm_config* cfg, int32_t block_start, int32_t* info);
+
 /* Failure-detection self-test (no counterpart on the pages).  Launches one
  * CTA whose bounded device wait has nothing to wait for: after limit_us
  * microseconds (clamped to [1, 2000000]) it gives up and ORs

@@ -165,3 +165,32 @@ def test_range_arguments_cannot_wrap(lib):
     assert abi.dllm_o_proj(cfg, weights, 0, d, big, 64, d, d, None, d, n.value, None) == bad
     assert abi.dllm_qkv_proj(cfg, weights, 0, d, None, 0, 2 ** 31 - 1, d, d, d, d, d, n.value,
                              None) == bad
+
+
+def test_layer_stack_plan_partitions_every_weight_block():
+    """Host plan of the persistent layer-stack kernel: for the workload shapes
+    it serves and for ragged mid-size ones, every 64-wide k-block of every
+    weight tile belongs to exactly one CTA share, and the attention units fit
+    one per CTA.  Shapes outside its scope report that they do not qualify."""
+    from diffusion_decoding_step_b200 import workload as wl
+    from diffusion_decoding_step_b200.runtime import make_config
+    shapes = [wl.WORKLOADS["llada8b_dual"], wl.WORKLOADS["dream7b_prefix"]]
+    for hidden, hq, hkv in ((512, 4, 4), (896, 7, 1), (1280, 10, 2), (3584, 28, 4),
+                            (4096, 32, 8), (384, 3, 1), (8192, 64, 8)):
+        shapes.append(wl.Workload("s", batch=1, n_layers=2, hidden=hidden, n_q_heads=hq,
+                                  n_kv_heads=hkv, head_dim=128, vocab=8192, prompt_len=96,
+                                  gen_len=64, block=32, mode=wl.MODE_DUAL))
+    for w in shapes:
+        cfg = make_config(w)
+        for blk in range(w.prompt_len, w.seq_len, w.block):
+            info = (C.c_int32 * 8)()
+            assert abi.dllm_layer_stack_plan(C.byref(cfg), blk, info) == abi.DLLM_OK
+            assert info[0] == 1, (w.hidden, blk)
+            assert info[7] == 1, (w.hidden, blk)
+            assert 1 <= info[2] <= 148 and 1 <= info[3] <= 148
+            assert info[6] <= 148 and info[4] in (1, 2, 4, 8, 16)
+    for name in ("tiny", "llada8b_dual_b16", "qwen7b_long_pruned"):
+        w = wl.WORKLOADS[name]
+        info = (C.c_int32 * 8)()
+        assert abi.dllm_layer_stack_plan(C.byref(make_config(w)), w.prompt_len, info) == abi.DLLM_OK
+        assert info[0] == 0

@@ -54,6 +54,26 @@ def test_lockstep_decode(name):
     assert not dec.masked.any()
 
 
+@pytest.mark.parametrize("name", ["llada_mid_dual", "dream_mid_prefix", "qwen_mid_pruned"])
+def test_lockstep_decode_layer_stack(name):
+    """The persistent layer-stack kernel (one launch for all layers of a step
+    or refresh; off by default) in lockstep with the oracle."""
+    from diffusion_decoding_step_b200 import abi
+    case = Case(MID[name])
+    dec = make_decoder(case)
+    info = (C.c_int32 * 8)()
+    abi.check(abi.dllm_layer_stack_plan(dec.cfg_p, case.w.prompt_len, info), "plan")
+    assert info[0] == 1 and info[7] == 1
+    abi.check(abi.dllm_set_layer_stack(1, 16), "layer stack on")
+    try:
+        rep = lockstep(dec, case)
+    finally:
+        abi.check(abi.dllm_set_layer_stack(0, 16), "layer stack off")
+    assert rep.steps >= (case.w.gen_len // case.w.block)
+    assert rep.flagged_mismatch <= max(2, rep.rows // 50)
+    assert not dec.masked.any()
+
+
 def test_tiny_free_running_decode_matches_oracle():
     case = Case(TINY)
     tr = case.decode()
