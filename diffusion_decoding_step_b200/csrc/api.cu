@@ -1469,22 +1469,33 @@ constexpr int kNoAllocMaxSlots = 160;  // persistent LM-head CTAs per row tile (
 }
 static __device__ __align__(256) dllm::LmStat
     g_noalloc_stats[DLLM_NOALLOC_MAX_ROWS * kNoAllocMaxSlots];
+// Status word of the call in flight: a bounded device wait that gives up sets
+// a bit here, and the reduce kernel then marks every row of the call invalid.
+static __device__ __align__(256) int g_noalloc_status;
 
 namespace {
-// Device address of g_noalloc_stats on the current device, looked up once per
-// device (host code may not use the symbol itself as a device address).
-dllm::LmStat* noalloc_scratch() {
+// Device addresses of g_noalloc_stats and g_noalloc_status on the current
+// device, looked up once per device (host code may not use the symbols
+// themselves as device addresses).
+bool noalloc_scratch(dllm::LmStat** stats, int** status) {
   static std::mutex mu;
   static dllm::LmStat* addr[64] = {};
+  static int* st_addr[64] = {};
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
   std::lock_guard<std::mutex> lock(mu);
   if (!addr[dev]) {
     void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_noalloc_stats) != cudaSuccess) return nullptr;
+    void* sp = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_stats) != cudaSuccess ||
+        cudaGetSymbolAddress(&sp, g_noalloc_status) != cudaSuccess)
+      return false;
     addr[dev] = static_cast<dllm::LmStat*>(ptr);
+    st_addr[dev] = static_cast<int*>(sp);
   }
-  return addr[dev];
+  *stats = addr[dev];
+  *status = st_addr[dev];
+  return true;
 }
 }  // namespace
 
@@ -1500,8 +1511,9 @@ dllm_status dllm_lmhead_confidence_noalloc(const dllm_config* cfg, const dllm_we
   const GemmPlan g = plan_lmhead(s.V, n_rows, s.Kw);
   const int slots = g.grid / g.n_tiles;
   if (slots > kNoAllocMaxSlots) return DLLM_ERR_UNSUPPORTED;
-  LmStat* scratch = noalloc_scratch();
-  if (!scratch) return DLLM_ERR_CUDA;
+  LmStat* scratch = nullptr;
+  int* dstatus = nullptr;
+  if (!noalloc_scratch(&scratch, &dstatus)) return DLLM_ERR_CUDA;
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   CUtensorMap wm, xm;
   if (!make_map(&wm, w->w_lm, s.Kw, s.V, 1, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -1518,9 +1530,10 @@ dllm_status dllm_lmhead_confidence_noalloc(const dllm_config* cfg, const dllm_we
   p.kb_per_split = g.kbps;
   p.units = g.units;
   p.layer = 0;
-  p.status = nullptr;
+  p.status = dstatus;
   p.stats = scratch;  // every slot a later read needs is written by this launch
   p.stat_slots = slots;
+  DLLM_TRY(cuda_status(cudaMemsetAsync(dstatus, 0, sizeof(int), st)));
   DLLM_TRY(cuda_status(launch_gemm(EPI_LMHEAD, g.nt, wm, xm, p, g.grid, false, st)));
   for (int r0 = 0; r0 < n_rows; r0 += 64) {  // the reduce kernel takes 64 rows per CTA
     CommitParams q{};
@@ -1534,6 +1547,8 @@ dllm_status dllm_lmhead_confidence_noalloc(const dllm_config* cfg, const dllm_we
     q.tok = tok + r0;
     q.gap = gap ? gap + r0 : nullptr;
     q.do_commit = 0;
+    q.status = dstatus;
+    q.invalid_on_status = 1;
     DLLM_TRY(cuda_status(launch_commit(q, false, st)));
   }
   return DLLM_OK;

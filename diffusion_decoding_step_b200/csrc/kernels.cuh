@@ -253,6 +253,9 @@ struct CommitParams {
   int* seq_done;
   const float* tau_seq;  // [b] per-sequence threshold, or null: tau
   int* status;           // device status word, or null
+  // reduce only: when the status word is nonzero (a wait of the LM head gave
+  // up), write conf = gap = NaN and tok = -1 instead of the merged statistics
+  int invalid_on_status;
 };
 cudaError_t launch_commit(const CommitParams& p, bool pdl, cudaStream_t s);
 

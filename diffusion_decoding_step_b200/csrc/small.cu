@@ -247,12 +247,18 @@ __global__ void __launch_bounds__(1024) commit_kernel(const CommitParams p) {
         st = merge_stat(st, o);
       }
       if (lane == 0) {
-        const float conf = 1.f / st.s;
+        float conf = 1.f / st.s, gap = st.m - st.m2;
+        int tok = st.idx;
+        if (p.invalid_on_status && p.status != nullptr && *p.status != 0) {
+          conf = __int_as_float(0x7fc00000);  // NaN: the statistics are not this call's
+          gap = conf;
+          tok = -1;
+        }
         s_conf[i] = conf;
-        s_tok[i] = st.idx;
+        s_tok[i] = tok;
         p.conf[b * p.B + i] = conf;
-        p.tok[b * p.B + i] = st.idx;
-        if (p.gap) p.gap[b * p.B + i] = st.m - st.m2;
+        p.tok[b * p.B + i] = tok;
+        if (p.gap) p.gap[b * p.B + i] = gap;
       }
     }
   } else {

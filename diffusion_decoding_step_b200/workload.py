@@ -12,8 +12,10 @@ suffix window (Streaming-dLLM README, figure "approximated suffix pruning").
 No benchmark item, prompt or trained weight is used: token ids are uniform
 random and weights are N(0, 0.02^2).
 
-Planted hidden states.  A masked block row's layer-0 input is
-``h = a * W_lm[t] / ||W_lm[t]||^2 + n`` with ``n ~ N(0, (sigma_w sqrt(d))^-2 I)``.
+Planted hidden states.  A masked block row's LM-head input gets the offset
+``h = a * W_lm[t] / ||W_lm[t]||^2 + n`` with ``n ~ N(0, (sigma_w sqrt(d))^-2 I)``
+added to its final normalised hidden state (its layer-0 input is the mask
+token's embedding, like any masked position).
 This puts the target logit at about ``a`` above logits that are N(0, 1), so
 confidences spread from ~1/V to ~1 as ``a`` goes from 0 to its maximum.
 ``t``, ``a`` and ``n`` are drawn once per (sequence, generated position).
@@ -173,7 +175,8 @@ def make_weights(w: Workload, device="cpu", layers: Optional[int] = None) -> Wei
 
 @dataclasses.dataclass
 class Plants:
-    """Planted layer-0 inputs of generated positions.
+    """Planted LM-head input offsets of generated positions (added to the final
+    normalised hidden state of a masked row).
 
     h [b][G][d] bf16 and the draws behind it: target t [b][G] and scale a [b][G].
     """

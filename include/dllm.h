@@ -22,7 +22,8 @@
  *  - All tensor pointers are DEVICE pointers owned by the caller unless a
  *    parameter says "host".  The library allocates no device memory; scratch
  *    comes from the caller's workspace (dllm_workspace_size bytes, prepared
- *    once with dllm_workspace_init).
+ *    once with dllm_workspace_init), except for dllm_lmhead_confidence_noalloc,
+ *    which keeps a fixed scratch array in the library's device image.
  *  - Calls are asynchronous on `stream` unless documented otherwise; nothing
  *    prints, nothing aborts.  Invalid arguments return DLLM_ERR_INVALID or
  *    DLLM_ERR_UNSUPPORTED before anything is launched.
@@ -35,7 +36,9 @@
  *    and query rows with 32-bit offsets in units of D).  rope_theta must be
  *    finite and >= 0 (0: no RoPE); tau must not be NaN.
  *  - Device-side waits are bounded (about 2 s); a wait that gives up sets a bit
- *    in the workspace status word, read with dllm_device_status.
+ *    in the workspace status word, read with dllm_device_status (calls
+ *    without a workspace report it in their outputs; see
+ *    dllm_lmhead_confidence_noalloc).
  */
 #ifndef DLLM_H_
 #define DLLM_H_
@@ -209,7 +212,12 @@ dllm_status dllm_lmhead_confidence(const dllm_config* cfg, const dllm_weights* w
  *  - All calls share the one scratch array, whatever their stream: calls that
  *    overlap on the GPU race and give wrong results.  Each call writes every
  *    scratch entry it reads, so nothing needs clearing between calls.
- *  - conf/tok/gap as in dllm_lmhead_confidence (gap may be NULL). */
+ *  - conf/tok/gap as in dllm_lmhead_confidence (gap may be NULL).  This call
+ *    has no workspace status word: if one of its bounded device waits gives
+ *    up (about 2 s), every row of the call gets conf = gap = NaN and
+ *    tok = -1, so the failure shows in the outputs themselves.  The call
+ *    clears its own device status word first (a cudaMemsetAsync of 4 bytes of
+ *    the library's static memory; nothing is allocated). */
 dllm_status dllm_lmhead_confidence_noalloc(const dllm_config* cfg, const dllm_weights* w,
                                            const void* h, int32_t n_rows, float* conf,
                                            int32_t* tok, float* gap, dllm_stream stream);
