@@ -66,7 +66,7 @@ SIGNATURES = {
     "dllm_final_norm": (C.c_int, [_CFG, _P, _I, _I, _I, _P, _P, _P, _P]),
     "dllm_lmhead_confidence": (C.c_int, [_CFG, _W, _P, _I, _P, _P, _P, _P, C.c_size_t, _P]),
     "dllm_lmhead_confidence_noalloc": (C.c_int, [_CFG, _W, _P, _I, _P, _P, _P, _P]),
-    "dllm_threshold_commit": (C.c_int, [_CFG, _I, _P, _P, _P, _P, _P, _P, _P]),
+    "dllm_threshold_commit": (C.c_int, [_CFG, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "dllm_prefill": (C.c_int, [_CFG, _W, _ST, _P, C.c_size_t, _P]),
     "dllm_decode_step": (C.c_int, [_CFG, _W, _ST, _I, _P, C.c_size_t, _P]),
     "dllm_kv_cache_refresh": (C.c_int, [_CFG, _W, _ST, _I, _P, C.c_size_t, _P]),
@@ -74,6 +74,7 @@ SIGNATURES = {
                                     C.c_size_t, _P]),
     "dllm_decode_all": (C.c_int, [_CFG, _W, _ST, C.POINTER(C.c_int32), _P, C.c_size_t, _P]),
     "dllm_step_outputs": (C.c_int, [_CFG, _P, C.c_size_t, C.POINTER(C.c_void_p),
+                                    C.POINTER(C.c_void_p), C.POINTER(C.c_void_p),
                                     C.POINTER(C.c_void_p), C.POINTER(C.c_void_p),
                                     C.POINTER(C.c_void_p)]),
     "dllm_device_status": (C.c_int, [_P, C.POINTER(C.c_int32), _P]),

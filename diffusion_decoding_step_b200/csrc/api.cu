@@ -310,7 +310,7 @@ StackPlan plan_stack(const Shape& s, int n_rows, int blk, int grid) {
 // ------------------------------------------------------------------ workspace
 struct Layout {
   size_t status, stepc, seqblk, seqdone, x, xb, sumsq, q, attn, h, stats, conf, tok, gap, commit,
-      remaining, segs, rope, total;
+      remaining, blkdone, refresh, segs, rope, total;
   int rmax, lm_slots;
   // layer-stack kernel: flags, split-K partials, attention chunk partials
   size_t stk_flags, stk_qpart, stk_opart, stk_apart, stk_aml;
@@ -363,6 +363,8 @@ Layout layout(const Shape& s) {
   l.gap = take((size_t)s.b * s.B * 4);
   l.commit = take((size_t)s.b * s.B);
   l.remaining = take((size_t)s.b * 4);
+  l.blkdone = take((size_t)s.b * 4);
+  l.refresh = take((size_t)s.b * 4);
   l.segs = take((size_t)s.b * 16);
   l.rope = take(s.theta > 0.f ? (size_t)s.S * (s.D / 2) * 8 : 256);
   // the layer-stack kernel runs steps and refreshes of b*B rows; its scratch
@@ -910,6 +912,8 @@ dllm_status run_commit(const Ctx& c, const dllm_state* stt, int blk_start, bool 
   p.masked = stt->masked;
   p.commit = c.at<uint8_t>(c.l.commit);
   p.remaining = c.at<int>(c.l.remaining);
+  p.block_done = c.at<int>(c.l.blkdone);
+  p.refresh = c.at<int>(c.l.refresh);
   p.do_commit = 1;
   p.topk = s.commit_mode == DLLM_COMMIT_TOPK;
   p.steps_per_block = s.spb;
@@ -1216,7 +1220,8 @@ dllm_status dllm_lmhead_confidence(const dllm_config* cfg, const dllm_weights* w
 
 dllm_status dllm_threshold_commit(const dllm_config* cfg, int32_t block_start, const float* conf,
                                   const int32_t* tok, int32_t* tokens, uint8_t* masked,
-                                  uint8_t* commit, int32_t* remaining, dllm_stream stream) {
+                                  uint8_t* commit, int32_t* remaining, int32_t* block_done,
+                                  int32_t* refresh_list, dllm_stream stream) {
   Shape s;
   DLLM_TRY(check_cfg(cfg, &s));
   if (!conf || !tok || !tokens || !masked) return DLLM_ERR_INVALID;
@@ -1235,6 +1240,8 @@ dllm_status dllm_threshold_commit(const dllm_config* cfg, int32_t block_start, c
   p.masked = masked;
   p.commit = commit;
   p.remaining = remaining;
+  p.block_done = block_done;
+  p.refresh = refresh_list;
   p.do_commit = 1;
   p.topk = s.commit_mode == DLLM_COMMIT_TOPK;
   p.steps_per_block = s.spb;
@@ -1289,21 +1296,22 @@ dllm_status dllm_decode_block(const dllm_config* cfg, const dllm_weights* w, con
   DLLM_TRY(check_block(c.s, block_start));
   if (max_steps < 1) max_steps = c.s.B;
   if (!st->plants || !aligned16(st->plants)) return DLLM_ERR_INVALID;
-  std::vector<int> rem(c.s.b + 1);
+  // steps until the commit step reports the block done in every sequence
+  std::vector<int> done(c.s.b + 1);
   int n = 0;
   for (; n < max_steps;) {
     DLLM_TRY(step_graph(c, cfg, w, st, ws, ws_bytes, block_start));
     ++n;
-    if (cudaMemcpyAsync(rem.data(), c.at<int>(c.l.remaining), sizeof(int) * c.s.b,
+    if (cudaMemcpyAsync(done.data(), c.at<int>(c.l.blkdone), sizeof(int) * c.s.b,
                         cudaMemcpyDeviceToHost, c.st) != cudaSuccess ||
-        cudaMemcpyAsync(rem.data() + c.s.b, c.at<int>(c.l.status), sizeof(int),
+        cudaMemcpyAsync(done.data() + c.s.b, c.at<int>(c.l.status), sizeof(int),
                         cudaMemcpyDeviceToHost, c.st) != cudaSuccess)
       return DLLM_ERR_CUDA;
     DLLM_TRY(wait_stream(c.st, kHostDeadlineS));
-    if (rem[c.s.b] != 0) return DLLM_ERR_TIMEOUT;
-    int left = 0;
-    for (int i = 0; i < c.s.b; ++i) left += rem[i];
-    if (left == 0) break;
+    if (done[c.s.b] != 0) return DLLM_ERR_TIMEOUT;
+    int all = 1;
+    for (int i = 0; i < c.s.b; ++i) all &= done[i] != 0;
+    if (all) break;
   }
   if (steps_taken) *steps_taken = n;
   return refresh_graph(c, cfg, w, st, ws, ws_bytes, block_start);
@@ -1434,13 +1442,16 @@ void dllm_graph_cache_clear(void) {
 }
 
 dllm_status dllm_step_outputs(const dllm_config* cfg, void* ws, size_t ws_bytes, float** conf,
-                              int32_t** tok, float** gap, uint8_t** commit) {
+                              int32_t** tok, float** gap, uint8_t** commit, int32_t** block_done,
+                              int32_t** refresh_list) {
   Ctx c;
   DLLM_TRY(make_ctx(cfg, ws, ws_bytes, nullptr, &c));
   if (conf) *conf = c.at<float>(c.l.conf);
   if (tok) *tok = c.at<int>(c.l.tok);
   if (gap) *gap = c.at<float>(c.l.gap);
   if (commit) *commit = c.at<uint8_t>(c.l.commit);
+  if (block_done) *block_done = c.at<int>(c.l.blkdone);
+  if (refresh_list) *refresh_list = c.at<int>(c.l.refresh);
   return DLLM_OK;
 }
 

@@ -242,6 +242,11 @@ struct CommitParams {
   uint8_t* masked;
   uint8_t* commit;
   int* remaining;
+  // optional: block_done[b] = 1 when no row of the block is left masked;
+  // refresh[b] = the block start this commit finished (its keys/values are to
+  // be recomputed from the committed tokens), else -1
+  int* block_done;
+  int* refresh;
   int do_commit;
   int topk;             // fixed-budget rule instead of the threshold
   int steps_per_block;  // topk: steps a block takes; threshold: step cap (0 = none)

@@ -355,9 +355,16 @@ __global__ void __launch_bounds__(1024) commit_kernel(const CommitParams p) {
   }
   const unsigned left = __popc(__ballot_sync(0xffffffffu, m0 && !k0)) +
                         __popc(__ballot_sync(0xffffffffu, m1 && !k1));
+  if (lane == 0) {
+    // the block's state after this commit: done, and (when this commit
+    // finished it) due for the key/value refresh from its committed tokens
+    if (p.block_done) p.block_done[b] = left == 0 ? 1 : 0;
+    if (p.refresh) p.refresh[b] = (left == 0 && any_masked) ? blk : -1;
+  }
   if (p.seq_blk != nullptr) {
     // per-sequence blocks: a block without masked rows was refreshed by this
-    // pass; move on.  remaining = 1 while the sequence has work left.
+    // pass (the refresh list named it after the previous pass); move on.
+    // remaining = 1 while the sequence has work left.
     const bool any_start = __any_sync(0xffffffffu, m0 || m1);
     if (lane == 0) {
       int done = p.seq_done[b];

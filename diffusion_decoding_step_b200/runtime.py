@@ -148,19 +148,29 @@ class Decoder:
                   "decode_all")
         return int(n.value)
 
-    def step_outputs(self):
-        """(conf, tok, gap, commit) of the last step, each [b][B], as views."""
-        ptrs = [C.c_void_p() for _ in range(4)]
+    def _outputs(self):
+        ptrs = [C.c_void_p() for _ in range(6)]
         abi.check(abi.dllm_step_outputs(self.cfg_p, _ptr(self.ws), self.ws_bytes,
                                         *[C.byref(p) for p in ptrs]), "step_outputs")
-        base = self.ws.data_ptr()
+        return [p.value - self.ws.data_ptr() for p in ptrs]
+
+    def step_outputs(self):
+        """(conf, tok, gap, commit) of the last step, each [b][B], as views."""
         n = self.w.batch * self.w.block
         out = []
-        for p, dt, size in zip(ptrs, (torch.float32, torch.int32, torch.float32, torch.uint8),
-                               (4, 4, 4, 1)):
-            off = p.value - base
+        for off, dt, size in zip(self._outputs()[:4],
+                                 (torch.float32, torch.int32, torch.float32, torch.uint8),
+                                 (4, 4, 4, 1)):
             out.append(self.ws[off:off + n * size].view(dt).view(self.w.batch, self.w.block))
         return tuple(out)
+
+    def block_state(self):
+        """(block_done, refresh_list) of the last step's commit, each [b] int32
+        views: 1 when the sequence's block has no masked row left, and the
+        block start whose keys/values the commit made due for a refresh (-1:
+        none)."""
+        b = self.w.batch
+        return tuple(self.ws[off:off + 4 * b].view(torch.int32) for off in self._outputs()[4:])
 
     def device_status(self) -> int:
         code = C.c_int32(0)

@@ -186,10 +186,11 @@ class Plants:
 
 
 def make_plants(w: Workload, w_lm: torch.Tensor, a_override: Optional[float] = None,
-                noise: bool = True) -> Plants:
-    """Draw the planted hidden states on ``w_lm``'s device."""
+                noise: bool = True, seed: Optional[int] = None) -> Plants:
+    """Draw the planted hidden states on ``w_lm``'s device (seed: another draw
+    of the same distribution; default SEED_PLANTS)."""
     dev = w_lm.device
-    g = _gen(SEED_PLANTS, dev)
+    g = _gen(SEED_PLANTS if seed is None else seed, dev)
     G = w.gen_len
     t = torch.randint(0, w.vocab, (w.batch, G), generator=g, device=dev)
     a = torch.rand((w.batch, G), generator=g, device=dev, dtype=torch.float32) * w.plant_a_max

@@ -130,15 +130,18 @@ typedef struct {
                              * so a policy may change it between steps; NULL: cfg->tau */
 } dllm_state;
 
-/* Bytes of workspace a configuration needs (host call, no GPU work). */
+/* Bytes of workspace a configuration needs (host call, no GPU work).  Library
+ * plumbing, no counterpart on the pages. */
 dllm_status dllm_workspace_size(const dllm_config* cfg, size_t* bytes);
 
 /* Zero the workspace's counters and status word and build the RoPE table.
- * Call once per workspace before any other call that takes it. */
+ * Call once per workspace before any other call that takes it.  Library
+ * plumbing, no counterpart on the pages. */
 dllm_status dllm_workspace_init(const dllm_config* cfg, void* ws, size_t ws_bytes,
                                 dllm_stream stream);
 
-/* fp32 [rows][cols] -> bf16 [rows][2*cols] with hi = bf16(w), lo = bf16(w - hi). */
+/* fp32 [rows][cols] -> bf16 [rows][2*cols] with hi = bf16(w), lo = bf16(w - hi).
+ * Storage of fp32 weights for the GEMM; no counterpart on the pages. */
 dllm_status dllm_split_f32_weights(const float* src, void* dst, int64_t rows, int64_t cols,
                                    dllm_stream stream);
 
@@ -146,7 +149,10 @@ dllm_status dllm_split_f32_weights(const float* src, void* dst, int64_t rows, in
  * [rows][hidden/128] fp32: entry j is the sum of x^2 over columns
  * [128j, 128j+128) (a row's total is the sum of its entries). */
 
-/* Layer-0 input of n_rows rows per sequence starting at position row0:
+/* Step a1.  Layer-0 input of the rows a step evaluates: a masked position is
+ * evaluated as the mask token, a settled one as its token (the masked
+ * positions of the block are evaluated in parallel: "Fast-dLLM: Four Acceleration Tracks ...", section "The v1 Mechanism").
+ * Layer-0 input of n_rows rows per sequence starting at position row0:
  * x[b*n_rows+i] = embed[masked[b][p] ? mask_id : tokens[b][p]], p = row0+i.
  * x fp32 [b*n_rows][hidden]; xb its bf16 copy; row_sumsq (may be NULL) gets
  * each row's sum of squares in entry 0 and zeros elsewhere. */
@@ -154,7 +160,10 @@ dllm_status dllm_embed_rows(const dllm_config* cfg, const dllm_weights* w,
                             const dllm_state* st, int32_t row0, int32_t n_rows, float* x,
                             void* xb, float* row_sumsq, dllm_stream stream);
 
-/* Q/K/V projection of layer `layer` (GEMM on tcgen05, fp32 accumulate) for
+/* Step a2.  The keys/values written here are the cache the v1 mechanism
+ * keeps for settled positions ("Fast-dLLM: Four Acceleration Tracks ...", section "The v1 Mechanism"); RoPE
+ * is the Qwen2.5-shaped workload's rotary embedding.
+ * Q/K/V projection of layer `layer` (GEMM on tcgen05, fp32 accumulate) for
  * n_rows rows per sequence at positions row0..: (W_qkv . xb) / rms(x) with
  * rms from row_sumsq (NULL = no scaling), RoPE at position p-seq_start on q
  * and k, q -> q_out bf16 [b][Hq][n_rows][D], k/v -> the caches at p.
@@ -164,7 +173,13 @@ dllm_status dllm_qkv_proj(const dllm_config* cfg, const dllm_weights* w, int32_t
                           const int32_t* seq_start, void* q_out, void* k_cache, void* v_cache,
                           void* ws, size_t ws_bytes, dllm_stream stream);
 
-/* Non-causal GQA attention of n_rows query rows per sequence (q bf16
+/* Step a3.  Block attention against the cached keys/values ("Fast-dLLM: Four Acceleration Tracks ...", section "The v1 Mechanism"); the
+ * two segments per sequence express the pruned suffix: a window after the
+ * block plus the trailing position (Streaming-dLLM README, figure
+ * "Illustration of approximated suffix pruning").  There is no log-sum-exp
+ * output: no caller of the step needs it, and the key chunks of a row tile
+ * are merged inside the kernel.
+ * Non-causal GQA attention of n_rows query rows per sequence (q bf16
  * [b][Hq][n_rows][D]) against layer `layer` of the caches.  Query head h reads
  * kv head h/(Hq/Hkv).  Keys of sequence i: segs[i][j] = (start, len) for
  * j = 0,1 (device int32 [b][2][2]; len 0 = unused).  Scale 1/sqrt(D).
@@ -174,13 +189,17 @@ dllm_status dllm_block_attn(const dllm_config* cfg, int32_t layer, int32_t n_row
                             const int32_t* segs, void* out, void* ws, size_t ws_bytes,
                             dllm_stream stream);
 
-/* Output projection and residual: x += attn . Wo^T (fp32), xb = bf16(x),
+/* Step a4 (the backbone's attention output projection; the shapes are the
+ * LLaDA-8B / Dream-7B-shaped workloads').
+ * Output projection and residual: x += attn . Wo^T (fp32), xb = bf16(x),
  * row_sumsq (may be NULL) = the new residual's per-slice sums of squares. */
 dllm_status dllm_o_proj(const dllm_config* cfg, const dllm_weights* w, int32_t layer,
                         const void* attn, int32_t row0, int32_t n_rows, float* x, void* xb,
                         float* row_sumsq, void* ws, size_t ws_bytes, dllm_stream stream);
 
-/* LM-head input of the block at block_start: for every sequence b and block
+/* LM-head input (the final norm, and the workloads' planted hidden state of a
+ * masked row; no counterpart on the pages).
+ * LM-head input of the block at block_start: for every sequence b and block
  * row i (position p = block_start+i, x row b*n_rows + p-row0):
  * h[b][i] = bf16(x / rms(x) + (masked[b][p] ? plants[b][p-P] : 0)).
  * x fp32 [b*n_rows][hidden]; h bf16 [b][B][hidden]. */
@@ -188,7 +207,10 @@ dllm_status dllm_final_norm(const dllm_config* cfg, const float* x, int32_t row0
                             int32_t block_start, const uint8_t* masked, const void* plants,
                             void* h, dllm_stream stream);
 
-/* LM head + confidence over the full vocabulary for n_rows rows of h (bf16
+/* Step a5.  The confidence each masked position is committed on ("Fast-dLLM: Four Acceleration Tracks ...", section "The v1 Mechanism").
+ * The rows are given contiguous (the step's caller compacts them); there is
+ * no row-index list.
+ * LM head + confidence over the full vocabulary for n_rows rows of h (bf16
  * [n_rows][hidden]); no logits are written.  conf = max softmax probability,
  * tok = argmax (lowest id on ties), gap = top-1 minus top-2 logit (may be NULL). */
 dllm_status dllm_lmhead_confidence(const dllm_config* cfg, const dllm_weights* w,
@@ -222,47 +244,71 @@ dllm_status dllm_lmhead_confidence_noalloc(const dllm_config* cfg, const dllm_we
                                            const void* h, int32_t n_rows, float* conf,
                                            int32_t* tok, float* gap, dllm_stream stream);
 
-/* Threshold commit of the block at block_start for every sequence: masked
- * rows with conf > tau commit, and the most confident masked row always does
- * (lowest position on ties).  conf/tok [b][B].  Updates tokens and masked;
- * commit (opt, [b][B] u8) marks committed rows; remaining (opt, [b]) gets the
- * number of rows still masked. */
+/* Step a6.  The commit rule of "Fast-dLLM: Four Acceleration Tracks ...", section "The v1 Mechanism":
+ * positions whose confidence clears the threshold are committed and never
+ * revised; a finished block's keys/values are then recomputed (the cache keeps
+ * settled positions).
+ * Commit of the block at block_start for every sequence (cfg->commit_mode;
+ * THRESHOLD: masked rows with conf > tau commit, and the most confident
+ * masked row always does, lowest position on ties).  conf/tok [b][B].
+ * Updates tokens and masked.  Optional outputs (NULL to skip), all device:
+ *  - commit [b][B] u8: 1 for the rows this call committed;
+ *  - remaining [b]: rows of the block still masked;
+ *  - block_done [b]: 1 when no row of the sequence's block is left masked;
+ *  - refresh_list [b]: block_start when this call finished the sequence's
+ *    block (some row was masked before it), so its keys/values are due for
+ *    dllm_kv_cache_refresh; -1 otherwise. */
 dllm_status dllm_threshold_commit(const dllm_config* cfg, int32_t block_start,
                                   const float* conf, const int32_t* tok, int32_t* tokens,
                                   uint8_t* masked, uint8_t* commit, int32_t* remaining,
+                                  int32_t* block_done, int32_t* refresh_list,
                                   dllm_stream stream);
 
-/* Fill the caches before decoding: PREFIX runs the prompt, DUAL and
+/* Step a8.  The cache a step reads from ("Fast-dLLM: Four Acceleration Tracks ...", section "The v1 Mechanism";
+ * Fast-dLLM README, "Quick Start": use_cache).
+ * Fill the caches before decoding: PREFIX runs the prompt, DUAL and
  * DUAL_PRUNED run prompt plus mask tokens (whole sequence); NONE does nothing. */
 dllm_status dllm_prefill(const dllm_config* cfg, const dllm_weights* w, const dllm_state* st,
                          void* ws, size_t ws_bytes, dllm_stream stream);
 
-/* One denoising step of the block at block_start: embed, L layers, LM head,
- * threshold commit.  The step's conf/tok/gap/commit stay in the workspace
- * (dllm_step_outputs). */
+/* Steps a1-a6 as one denoising step ("Fast-dLLM: Four Acceleration Tracks ...", section "The v1 Mechanism").
+ * One denoising step of the block at block_start: embed, L layers, LM head,
+ * commit.  The step's conf/tok/gap/commit, block-done flags and refresh list
+ * stay in the workspace (dllm_step_outputs). */
 dllm_status dllm_decode_step(const dllm_config* cfg, const dllm_weights* w,
                              const dllm_state* st, int32_t block_start, void* ws,
                              size_t ws_bytes, dllm_stream stream);
 
-/* Recompute the keys/values of a finished block from its committed tokens:
+/* Step a7, the cache refresh of a finished block ("Fast-dLLM: Four Acceleration Tracks ...", section "The v1 Mechanism";
+ * same page, section "Fast-dLLM v1 Versus a Standard Diffusion Sampler").
+ * Recompute the keys/values of a finished block from its committed tokens:
  * L layers with input embed[token], same key set as a step, no LM head. */
 dllm_status dllm_kv_cache_refresh(const dllm_config* cfg, const dllm_weights* w,
                                   const dllm_state* st, int32_t block_start, void* ws,
                                   size_t ws_bytes, dllm_stream stream);
 
-/* Decode one block to completion: steps until no row of the block is masked
- * in any sequence (or max_steps), then the cache refresh.  Blocks the calling
- * host thread until the block is done; *steps_taken (host) gets the count. */
+/* A block of the block schedule decoded to completion, then refreshed
+ * ("Fast-dLLM: Four Acceleration Tracks ...", section "The v1 Mechanism"; same page, section "Fast-dLLM v1
+ * Versus a Standard Diffusion Sampler"; Fast-dLLM README, "Quick Start":
+ * --block_size).
+ * Decode one block to completion: steps until the commit step reports the
+ * block done in every sequence (or max_steps), then the cache refresh.  Blocks
+ * the calling host thread until the block is done; *steps_taken (host) gets
+ * the count. */
 dllm_status dllm_decode_block(const dllm_config* cfg, const dllm_weights* w,
                               const dllm_state* st, int32_t block_start, int32_t max_steps,
                               int32_t* steps_taken, void* ws, size_t ws_bytes,
                               dllm_stream stream);
 
-/* Decode every block of every sequence, each sequence at its own block
+/* The block schedule of "Fast-dLLM: Four Acceleration Tracks ...", section "The v1 Mechanism" run per
+ * sequence: each sequence decodes its own blocks left to right.
+ * Decode every block of every sequence, each sequence at its own block
  * (after dllm_prefill).  A pass runs one step for every sequence at its
- * current block; a pass that finds no masked row in a sequence's block is
- * that block's refresh (the rows, all committed, rewrite their keys/values
- * against the step's key set) and the sequence moves to its next block.  A
+ * current block.  The pass after the one whose commit finished a sequence's
+ * block (the commit step's refresh list names that block) finds no masked
+ * row in it and is that block's refresh (the rows, all committed, rewrite
+ * their keys/values against the step's key set); the sequence then moves to
+ * its next block.  A
  * finished sequence's passes recompute its last block (no state change).
  * Each sequence's tokens equal those of dllm_decode_block run block by block
  * with the batch in lockstep: sequences never interact.  Blocks the calling
@@ -271,9 +317,12 @@ dllm_status dllm_decode_block(const dllm_config* cfg, const dllm_weights* w,
 dllm_status dllm_decode_all(const dllm_config* cfg, const dllm_weights* w, const dllm_state* st,
                             int32_t* passes, void* ws, size_t ws_bytes, dllm_stream stream);
 
-/* Device pointers (into ws) of the last step's outputs, each [b][B]. */
+/* Device pointers (into ws) of the last step's outputs: conf, tok, gap and
+ * commit [b][B]; block_done and refresh_list [b], as dllm_threshold_commit
+ * describes them.  Any output pointer may be NULL. */
 dllm_status dllm_step_outputs(const dllm_config* cfg, void* ws, size_t ws_bytes, float** conf,
-                              int32_t** tok, float** gap, uint8_t** commit);
+                              int32_t** tok, float** gap, uint8_t** commit, int32_t** block_done,
+                              int32_t** refresh_list);
 
 /* Copy the workspace's device status word to *code (host); synchronises stream.
  * The word is 0, or an OR of:

@@ -178,6 +178,19 @@ def threshold_commit(conf: np.ndarray, masked: np.ndarray, tau: float) -> np.nda
     return commit
 
 
+def block_state(masked_before: np.ndarray, masked_after: np.ndarray, s: int):
+    """One sequence's block after a commit: (done, refresh).
+
+    done: no row of the block is left masked.  refresh: the block start s when
+    this commit finished the block (some row was masked before it), else -1;
+    a finished block's keys/values are then recomputed from its committed
+    tokens, since the cache keeps the attention state of settled positions
+    ("Fast-dLLM: Four Acceleration Tracks ...", section "The v1 Mechanism").
+    """
+    done = not bool(np.asarray(masked_after).any())
+    return done, (int(s) if done and bool(np.asarray(masked_before).any()) else -1)
+
+
 def topk_budget(block: int, steps_per_block: int, n_masked: int) -> int:
     """Rows a fixed-budget step commits (the low-confidence-remasking sampler).
 

@@ -47,6 +47,7 @@ def compare_step(dec, case, s: int, rep: Report, check_kv: bool = True,
     assert dec.device_status() == 0
     conf, tok, gap, commit = (t.cpu().numpy() for t in dec.step_outputs())
     B = cfg.block
+    check_block_state(dec, st.masked, s, B)
     for bi in range(cfg.batch):
         m = ~np.isnan(r.conf[bi])
         if not m.any():
@@ -79,6 +80,16 @@ def compare_step(dec, case, s: int, rep: Report, check_kv: bool = True,
         got = f64(dec.v_cache[:, :, :, s:s + B])
         assert rel_l2(got, st.vcache[:, :, :, s:s + B]) <= 5e-3
     rep.steps += 1
+
+
+def check_block_state(dec, masked_before, s: int, B: int) -> None:
+    """The commit step's block-done flags and refresh list are exactly the
+    oracle's rule applied to the mask before and after the GPU's own commit."""
+    done, refresh = (t.cpu().numpy() for t in dec.block_state())
+    after = dec.masked.cpu().numpy().astype(bool)
+    for bi in range(dec.w.batch):
+        d_ref, r_ref = O.block_state(masked_before[bi, s:s + B], after[bi, s:s + B], s)
+        assert int(done[bi]) == int(d_ref) and int(refresh[bi]) == r_ref, (s, bi)
 
 
 def compare_refresh(dec, case, s: int) -> None:
@@ -167,3 +178,81 @@ def compare_step_sampled(dec, case, s: int, seqs, rep: Report, taus=None,
         assert not (bad & ~flag).any(), f"seq {bi}: unflagged mismatch rows {np.where(bad & ~flag)[0]}"
         rep.flagged_mismatch += int(bad.sum())
     rep.steps += 1
+
+
+def lockstep_incremental(dec, case, max_blocks=None, log=None) -> Report:
+    """lockstep() for full-size workloads: the oracle's copy of the state is
+    kept on the host and only what a GPU step or refresh writes (the block's
+    cache slots, tokens and mask) is copied back, instead of the whole caches
+    every step.  Prefill, every step and every refresh are compared exactly as
+    lockstep() does; the block's keys/values are compared after each step."""
+    import time
+    rep = Report()
+    cfg, W, B = case.cfg, case.W, case.cfg.block
+    dec.prefill()
+    torch.cuda.synchronize()
+    assert dec.device_status() == 0
+    st = state_from_gpu(dec)
+    end = cfg.prompt_len if cfg.mode == O.MODE_PREFIX else cfg.seq_len
+    ref = O.new_state(cfg, st.tokens, st.masked, st.starts)
+    O.prefill(cfg, W, ref)
+    for bi in range(cfg.batch):
+        a = int(st.starts[bi])
+        for got, want in ((st.kcache, ref.kcache), (st.vcache, ref.vcache)):
+            assert rel_l2(got[:, bi, :, a:end], want[:, bi, :, a:end]) <= 5e-3
+    del ref
+    blocks = list(range(cfg.prompt_len, cfg.seq_len, B))[:max_blocks]
+    t0 = time.time()
+    for s in blocks:
+        n = 0
+        while st.masked[:, s:s + B].any():
+            r = O.decode_step(cfg, W, st, case.plants64, s, apply=False, step_in_block=n)
+            dec.step(s)
+            torch.cuda.synchronize()
+            assert dec.device_status() == 0
+            conf, tok, gap, commit = (t.cpu().numpy() for t in dec.step_outputs())
+            check_block_state(dec, st.masked, s, B)
+            for bi in range(cfg.batch):
+                m = ~np.isnan(r.conf[bi])
+                if not m.any():
+                    assert not commit[bi].any()
+                    continue
+                rep.rows += int(m.sum())
+                err = np.abs(conf[bi][m] - r.conf[bi][m])
+                rep.max_conf_err = max(rep.max_conf_err, float(err.max()))
+                assert err.max() <= CONF_TOL, f"conf error {err.max()} at block {s}"
+                flag = r.amb_tok[bi] | r.amb_commit[bi]
+                rep.flagged += int(flag.sum())
+                bad = (m & (tok[bi] != r.tok[bi])) | (commit[bi].astype(bool) != r.commit[bi])
+                assert not (bad & ~flag).any(), (
+                    f"block {s} seq {bi}: unflagged mismatch rows {np.where(bad & ~flag)[0]}")
+                rep.flagged_mismatch += int(bad.sum())
+            # the oracle wrote its own keys/values of the block rows into st:
+            # compare, then continue from what the GPU wrote
+            got_k = f64(dec.k_cache[:, :, :, s:s + B])
+            got_v = f64(dec.v_cache[:, :, :, s:s + B])
+            kr = rel_l2(got_k, st.kcache[:, :, :, s:s + B])
+            rep.max_kv_rel = max(rep.max_kv_rel, kr)
+            assert kr <= 5e-3
+            assert rel_l2(got_v, st.vcache[:, :, :, s:s + B]) <= 5e-3
+            st.kcache[:, :, :, s:s + B] = got_k
+            st.vcache[:, :, :, s:s + B] = got_v
+            st.tokens = dec.tokens.cpu().numpy().astype(np.int64)
+            st.masked = dec.masked.cpu().numpy().astype(bool)
+            rep.steps += 1
+            n += 1
+            assert n <= B
+        O.refresh_block(cfg, W, st, s)
+        dec.refresh(s)
+        torch.cuda.synchronize()
+        got_k = f64(dec.k_cache[:, :, :, s:s + B])
+        got_v = f64(dec.v_cache[:, :, :, s:s + B])
+        assert rel_l2(got_k, st.kcache[:, :, :, s:s + B]) <= 5e-3
+        assert rel_l2(got_v, st.vcache[:, :, :, s:s + B]) <= 5e-3
+        st.kcache[:, :, :, s:s + B] = got_k
+        st.vcache[:, :, :, s:s + B] = got_v
+        if log:
+            log(f"block {s}: {n} steps, {rep.steps} steps so far, flagged {rep.flagged}, "
+                f"flagged mismatches {rep.flagged_mismatch}, max conf err {rep.max_conf_err:.2e}, "
+                f"max kv rel {rep.max_kv_rel:.2e}, {time.time() - t0:.0f} s")
+    return rep

@@ -29,12 +29,14 @@ def oracle_weights(W: wl.Weights) -> O.Weights:
 class Case:
     """All inputs of one workload on the CPU, plus the oracle's views of them."""
 
-    def __init__(self, w: wl.Workload, device="cpu", a_override=None, noise=True):
+    def __init__(self, w: wl.Workload, device="cpu", a_override=None, noise=True,
+                 plant_seed=None):
         self.w = w
         self.weights = wl.make_weights(w, device=device)
         self.tokens, self.masked = wl.make_tokens(w)
         self.starts = wl.seq_starts(w)
-        self.plants = wl.make_plants(w, self.weights.w_lm, a_override=a_override, noise=noise)
+        self.plants = wl.make_plants(w, self.weights.w_lm, a_override=a_override, noise=noise,
+                                     seed=plant_seed)
         self.cfg = oracle_config(w)
         self.W = oracle_weights(self.weights)
         self.plants64 = to64(self.plants.h)

@@ -117,7 +117,7 @@ def test_null_pointers_rejected_before_launch(lib):
         == abi.DLLM_ERR_INVALID
     assert abi.dllm_workspace_init(C.byref(cfg), None, n.value, None) == abi.DLLM_ERR_INVALID
     assert abi.dllm_threshold_commit(C.byref(cfg), 64, None, None, None, None, None, None,
-                                     None) == abi.DLLM_ERR_INVALID
+                                     None, None, None) == abi.DLLM_ERR_INVALID
     import torch
     if torch.cuda.is_available():   # the checks below pass dummy device pointers
         return
@@ -156,7 +156,7 @@ def test_range_arguments_cannot_wrap(lib):
     steps = C.c_int32(0)
     assert abi.dllm_decode_block(cfg, weights, state, big, 0, C.byref(steps), d, n.value,
                                  None) == bad
-    assert abi.dllm_threshold_commit(cfg, big, d, d, d, d, None, None, None) == bad
+    assert abi.dllm_threshold_commit(cfg, big, d, d, d, d, None, None, None, None, None) == bad
     assert abi.dllm_embed_rows(cfg, weights, state, big, 64, d, d, None, None) == bad
     assert abi.dllm_final_norm(cfg, d, big, 64, 256, d, d, d, None) == bad
     assert abi.dllm_final_norm(cfg, d, 0, 512, big, d, d, d, None) == bad

@@ -346,8 +346,11 @@ def test_threshold_commit_bit_exact(b, B, tau):
     remaining = torch.zeros(b, dtype=torch.int32, device=DEV)
     t_conf = torch.tensor(conf, device=DEV)
     t_tok = torch.tensor(tok, device=DEV)
+    done = torch.full((b,), 7, dtype=torch.int32, device=DEV)
+    refresh = torch.full((b,), 7, dtype=torch.int32, device=DEV)
     abi.check(abi.dllm_threshold_commit(C.byref(cfg), s, ptr(t_conf), ptr(t_tok), ptr(t_tokens),
-                                        ptr(t_masked), ptr(commit), ptr(remaining), stream()),
+                                        ptr(t_masked), ptr(commit), ptr(remaining), ptr(done),
+                                        ptr(refresh), stream()),
               "commit")
     torch.cuda.synchronize()
     for bi in range(b):
@@ -361,6 +364,8 @@ def test_threshold_commit_bit_exact(b, B, tau):
         assert np.array_equal(t_tokens[bi].cpu().numpy(), want_tok)
         assert np.array_equal(t_masked[bi].cpu().numpy(), want_mask)
         assert int(remaining[bi]) == int(m.sum() - c_ref.sum())
+        d_ref, r_ref = O.block_state(m, m & ~c_ref, s)
+        assert int(done[bi]) == int(d_ref) and int(refresh[bi]) == r_ref, f"seq {bi}"
 
 
 @pytest.mark.parametrize("b,B,spb,done", [(1, 8, 3, 0), (1, 32, 5, 14), (16, 32, 8, 0),
@@ -390,8 +395,11 @@ def test_topk_commit_bit_exact(b, B, spb, done):
     remaining = torch.zeros(b, dtype=torch.int32, device=DEV)
     t_conf = torch.tensor(conf, device=DEV)
     t_tok = torch.tensor(tok, device=DEV)
+    done = torch.full((b,), 7, dtype=torch.int32, device=DEV)
+    refresh = torch.full((b,), 7, dtype=torch.int32, device=DEV)
     abi.check(abi.dllm_threshold_commit(C.byref(cfg), s, ptr(t_conf), ptr(t_tok), ptr(t_tokens),
-                                        ptr(t_masked), ptr(commit), ptr(remaining), stream()),
+                                        ptr(t_masked), ptr(commit), ptr(remaining), ptr(done),
+                                        ptr(refresh), stream()),
               "commit")
     torch.cuda.synchronize()
     for bi in range(b):
@@ -403,3 +411,5 @@ def test_topk_commit_bit_exact(b, B, spb, done):
         want_tok[s:s + B][c_ref] = tok[bi][c_ref]
         assert np.array_equal(t_tokens[bi].cpu().numpy(), want_tok)
         assert int(remaining[bi]) == int(m.sum() - c_ref.sum())
+        d_ref, r_ref = O.block_state(m, m & ~c_ref, s)
+        assert int(done[bi]) == int(d_ref) and int(refresh[bi]) == r_ref, f"seq {bi}"

@@ -559,3 +559,28 @@ def test_step_cap_of_two_finishes_every_block_by_its_second_step():
             break
     else:
         raise AssertionError("no step committed a whole multi-row remainder")
+
+
+# ---------------------------------------------------------------- block state
+def test_block_state_done_and_refresh_rule():
+    m = np.array([True, False, True])
+    assert O.block_state(m, np.zeros(3, bool), 96) == (True, 96)      # this commit finished it
+    assert O.block_state(np.zeros(3, bool), np.zeros(3, bool), 96) == (True, -1)  # already done
+    assert O.block_state(m, np.array([False, False, True]), 96) == (False, -1)
+
+
+def test_block_state_over_a_decode_with_tau_above_one():
+    # one commit per step: the block is done, and due for its refresh, at
+    # exactly its B-th step and at no other
+    w = TINY.replace(tau=1.5)
+    case = Case(w)
+    tr = case.decode()
+    B = w.block
+    masked = case.masked.numpy().astype(bool).copy()
+    k = 0
+    for s, r in tr.steps:
+        before = masked[0, s:s + B].copy()
+        masked[0, s:s + B] &= ~r.commit[0]
+        done, refresh = O.block_state(before, masked[0, s:s + B], s)
+        k = k + 1 if k < B else 1
+        assert done == (k == B) and refresh == (s if k == B else -1)
