@@ -38,8 +38,11 @@ def parse():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
-    ap.add_argument("--commit", default="threshold", choices=["threshold", "topk"],
-                    help="commit rule: conf > tau (default) or a fixed top-k budget per step")
+    ap.add_argument("--commit", default="threshold", choices=["threshold", "topk", "early-exit"],
+                    help="commit rule: conf > tau (default), a fixed top-k budget per step, or "
+                         "conf > tau with an early exit for rows whose argmax repeats")
+    ap.add_argument("--exit-tau", type=float, default=0.5,
+                    help="early-exit: confidence bound of rows whose argmax repeats (default 0.5)")
     ap.add_argument("--blocks", default="lockstep", choices=["lockstep", "per-sequence"],
                     help="batches: blocks advance together (default) or each sequence at its "
                          "own block (dllm_decode_all)")
@@ -107,6 +110,9 @@ def selected_workload(args):
     if args.commit == "topk":
         w = w.replace(commit_mode=wl.COMMIT_TOPK,
                       steps_per_block=args.steps_per_block or max(1, w.block // 4))
+    elif args.commit == "early-exit":
+        w = w.replace(commit_mode=wl.COMMIT_EARLY_EXIT, exit_tau=args.exit_tau,
+                      steps_per_block=max(0, args.steps_per_block))
     elif args.steps_per_block > 0:  # threshold rule with a per-block step cap
         w = w.replace(steps_per_block=args.steps_per_block)
     return w
@@ -124,7 +130,8 @@ def workload_config(w, data_note):
             "cache": _mode_name(w.mode),
             "commit": (("threshold" + (f", cap {w.steps_per_block} steps per block"
                                         if w.steps_per_block > 0 else ""))
-                       if w.commit_mode == 0 else f"topk, {w.steps_per_block} steps per block"),
+                       if w.commit_mode == 0 else f"topk, {w.steps_per_block} steps per block"
+                       if w.commit_mode == 1 else f"early exit above {w.exit_tau}"),
             "l2": data_note}
 
 
@@ -264,7 +271,8 @@ def oracle_sample(w, weights, tokens, masked, starts, plants, budget_s=20.0):
                    n_kv_heads=w.n_kv_heads, head_dim=w.head_dim, vocab=w.vocab,
                    prompt_len=w.prompt_len, gen_len=w.gen_len, block=w.block, tau=w.tau,
                    mode=w.mode, window=w.window, rope_theta=w.rope_theta, mask_id=w.mask_id,
-                   commit_mode=w.commit_mode, steps_per_block=w.steps_per_block)
+                   commit_mode=w.commit_mode, steps_per_block=w.steps_per_block,
+                   exit_tau=w.exit_tau)
     W = O.Weights(lambda l: weights.wqkv[l].cpu().double().numpy(),
                   lambda l: weights.wo[l].cpu().double().numpy(),
                   weights.w_lm.cpu().double().numpy())

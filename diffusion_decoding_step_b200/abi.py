@@ -33,7 +33,7 @@ class dllm_config(C.Structure):
                 ("block", C.c_int32), ("window", C.c_int32), ("mask_id", C.c_int32),
                 ("tau", C.c_float), ("rope_theta", C.c_float), ("mode", C.c_int32),
                 ("weight_format", C.c_int32), ("commit_mode", C.c_int32),
-                ("steps_per_block", C.c_int32)]
+                ("steps_per_block", C.c_int32), ("exit_tau", C.c_float)]
 
 
 class dllm_weights(C.Structure):

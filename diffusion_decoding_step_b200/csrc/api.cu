@@ -63,7 +63,7 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_
 struct Shape {
   int b, L, d, Hq, Hkv, D, V, P, G, B, S, W, mode, wfmt, commit_mode, spb;
   int qkv_rows, Kw, Ko;
-  float tau, theta;
+  float tau, theta, exit_tau;
   int mask_id;
 };
 
@@ -80,7 +80,11 @@ dllm_status check_cfg(const dllm_config* c, Shape* s) {
   if (c->gen_len % c->block) return DLLM_ERR_INVALID;
   if (c->mode == DLLM_CACHE_DUAL_PRUNED && c->window < 0) return DLLM_ERR_INVALID;
   if (c->mask_id < 0 || c->mask_id >= c->vocab) return DLLM_ERR_INVALID;
-  if (c->commit_mode != DLLM_COMMIT_THRESHOLD && c->commit_mode != DLLM_COMMIT_TOPK)
+  if (c->commit_mode != DLLM_COMMIT_THRESHOLD && c->commit_mode != DLLM_COMMIT_TOPK &&
+      c->commit_mode != DLLM_COMMIT_EARLY_EXIT)
+    return DLLM_ERR_INVALID;
+  if (c->commit_mode == DLLM_COMMIT_EARLY_EXIT &&
+      !(c->exit_tau >= 0.f && c->exit_tau <= FLT_MAX))  // NaN, inf, negative
     return DLLM_ERR_INVALID;
   if (c->commit_mode == DLLM_COMMIT_TOPK &&
       (c->steps_per_block < 1 || c->steps_per_block > c->block))
@@ -121,6 +125,7 @@ dllm_status check_cfg(const dllm_config* c, Shape* s) {
   s->Ko = f * c->n_q_heads * c->head_dim;
   s->tau = c->tau;
   s->theta = c->rope_theta;
+  s->exit_tau = c->exit_tau;
   s->mask_id = c->mask_id;
   return DLLM_OK;
 }
@@ -309,7 +314,7 @@ StackPlan plan_stack(const Shape& s, int n_rows, int blk, int grid) {
 
 // ------------------------------------------------------------------ workspace
 struct Layout {
-  size_t status, stepc, seqblk, seqdone, x, xb, sumsq, q, attn, h, stats, conf, tok, gap, commit,
+  size_t status, stepc, seqblk, seqdone, exitst, x, xb, sumsq, q, attn, h, stats, conf, tok, gap, commit,
       remaining, blkdone, refresh, segs, rope, total;
   int rmax, lm_slots;
   // layer-stack kernel: flags, split-K partials, attention chunk partials
@@ -351,6 +356,9 @@ Layout layout(const Shape& s) {
   l.stepc = take((size_t)s.b * 2 * 4);  // per sequence: steps in the block, block start
   l.seqblk = take((size_t)s.b * 4);     // per sequence: current block (dllm_decode_all)
   l.seqdone = take((size_t)s.b * 4);    // per sequence: every block done
+  // early exit: per sequence the block start + 1 of the previous step (0:
+  // none), then every row's argmax at that step; zeroed with the counters
+  l.exitst = take((size_t)s.b * (1 + s.B) * 4);
   l.x = take((size_t)l.rmax * s.d * 4);
   l.xb = take((size_t)l.rmax * s.d * 2);
   l.sumsq = take((size_t)l.rmax * (s.d / 128) * 4);
@@ -918,6 +926,8 @@ dllm_status run_commit(const Ctx& c, const dllm_state* stt, int blk_start, bool 
   p.topk = s.commit_mode == DLLM_COMMIT_TOPK;
   p.steps_per_block = s.spb;
   p.step_ctr = c.at<int>(c.l.stepc);
+  p.exit_state = s.commit_mode == DLLM_COMMIT_EARLY_EXIT ? c.at<int>(c.l.exitst) : nullptr;
+  p.exit_tau = s.exit_tau;
   p.tau_seq = stt->tau;
   p.seq_blk = c.seq_blk;
   p.seq_done = c.seq_blk ? c.at<int>(c.l.seqdone) : nullptr;

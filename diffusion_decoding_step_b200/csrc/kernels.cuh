@@ -251,6 +251,10 @@ struct CommitParams {
   int topk;             // fixed-budget rule instead of the threshold
   int steps_per_block;  // topk: steps a block takes; threshold: step cap (0 = none)
   int* step_ctr;        // [b][2] steps taken in the current block, its start (null: no cap)
+  // early exit (null: off): [b] block start + 1 of the previous step (0: none),
+  // then [b][B] each row's argmax at that step (-1: not masked then)
+  int* exit_state;
+  float exit_tau;
   // per-sequence blocks (null: blk_start for every sequence): a pass that
   // finds no masked row in a sequence's block was that block's refresh, and
   // the sequence moves on to its next block (or is done after the last)

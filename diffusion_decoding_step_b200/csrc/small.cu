@@ -338,8 +338,30 @@ __global__ void __launch_bounds__(1024) commit_kernel(const CommitParams p) {
       force = n + 1 >= p.steps_per_block;
     }
     const float tau = p.tau_seq ? p.tau_seq[b] : p.tau;
-    k0 = m0 && (force || c0 > tau || (any_masked && bi == i0));
-    k1 = m1 && (force || c1 > tau || (any_masked && bi == i1));
+    // early exit: a row whose argmax repeats from the previous step of this
+    // block has converged and commits once conf > exit_tau
+    bool e0 = false, e1 = false;
+    if (p.exit_state != nullptr) {
+      int* pb = p.exit_state + b;
+      int* pt = p.exit_state + p.batch + (size_t)b * p.B;
+      // a block with every row masked is at its first step (also after the
+      // caller reset the state), so there is no previous argmax
+      const int nmask =
+          __popc(__ballot_sync(0xffffffffu, m0)) + __popc(__ballot_sync(0xffffffffu, m1));
+      const bool same = *pb == blk + 1 && nmask < p.B;
+      if (i0 < p.B) {
+        e0 = same && m0 && pt[i0] == s_tok[i0] && c0 > p.exit_tau;
+        pt[i0] = m0 ? s_tok[i0] : -1;
+      }
+      if (i1 < p.B) {
+        e1 = same && m1 && pt[i1] == s_tok[i1] && c1 > p.exit_tau;
+        pt[i1] = m1 ? s_tok[i1] : -1;
+      }
+      __syncwarp();
+      if (lane == 0) *pb = blk + 1;
+    }
+    k0 = m0 && (force || c0 > tau || e0 || (any_masked && bi == i0));
+    k1 = m1 && (force || c1 > tau || e1 || (any_masked && bi == i1));
   }
   if (k0) {
     p.tokens[base + i0] = s_tok[i0];

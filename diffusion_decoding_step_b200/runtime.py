@@ -20,7 +20,7 @@ def make_config(w: Workload) -> abi.dllm_config:
         gen_len=w.gen_len, block=w.block, window=w.window, mask_id=w.mask_id, tau=w.tau,
         rope_theta=w.rope_theta, mode=w.mode,
         weight_format=abi.DLLM_W_F32_SPLIT if w.weight_f32 else abi.DLLM_W_BF16,
-        commit_mode=w.commit_mode, steps_per_block=w.steps_per_block)
+        commit_mode=w.commit_mode, steps_per_block=w.steps_per_block, exit_tau=w.exit_tau)
 
 
 def workspace_bytes(w: Workload) -> int:

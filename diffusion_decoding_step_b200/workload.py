@@ -31,7 +31,9 @@ import torch
 
 MODE_NONE, MODE_PREFIX, MODE_DUAL, MODE_DUAL_PRUNED = 0, 1, 2, 3
 MODE_PREFIX_SUFFIXQ = 4    # prefix cache, block and suffix recomputed as queries each step
-COMMIT_THRESHOLD, COMMIT_TOPK = 0, 1  # conf > tau, or a fixed top-k budget per step
+# conf > tau; a fixed top-k budget per step; conf > tau or, for a row whose
+# argmax repeats from the previous step of the block, conf > exit_tau
+COMMIT_THRESHOLD, COMMIT_TOPK, COMMIT_EARLY_EXIT = 0, 1, 2
 MODE_NAMES = {MODE_NONE: "none", MODE_PREFIX: "prefix", MODE_DUAL: "dual",
               MODE_DUAL_PRUNED: "dual_pruned", MODE_PREFIX_SUFFIXQ: "prefix_suffixq"}
 
@@ -63,6 +65,7 @@ class Workload:
     prompt_len_min: Optional[int] = None  # ragged prompts: U[min, prompt_len]
     commit_mode: int = COMMIT_THRESHOLD
     steps_per_block: int = 0   # COMMIT_TOPK: a block is decoded in exactly this many steps
+    exit_tau: float = 1.0      # COMMIT_EARLY_EXIT: confidence bound of rows whose argmax repeats
 
     def __post_init__(self):
         if self.mask_id < 0:

@@ -93,8 +93,22 @@ typedef enum { DLLM_W_BF16 = 0, DLLM_W_F32_SPLIT = 1 } dllm_weight_format;
  *              steps; step j commits floor(B/steps) + [j < B mod steps] of
  *              the most confident masked rows (lower position first on
  *              equal confidence), j being inferred from the rows already
- *              committed.  tau is not used. */
-typedef enum { DLLM_COMMIT_THRESHOLD = 0, DLLM_COMMIT_TOPK = 1 } dllm_commit_mode;
+ *              committed.  tau is not used.
+ *   EARLY_EXIT a dynamic threshold, reading Streaming-dLLM's confidence-aware
+ *              early exit for converged tokens (thelatestinai listing page,
+ *              Streaming-dLLM abstract): a masked row whose argmax equals
+ *              its argmax at the previous step of the same block has
+ *              converged and commits once conf > exit_tau (<= tau); other
+ *              rows as THRESHOLD (conf > tau, plus the most confident masked
+ *              row).  At a block's first step it is THRESHOLD.  The previous
+ *              argmax per row is kept in the workspace by dllm_decode_step /
+ *              dllm_decode_block / dllm_decode_all; dllm_threshold_commit,
+ *              which has no workspace, applies the first-step rule. */
+typedef enum {
+  DLLM_COMMIT_THRESHOLD = 0,
+  DLLM_COMMIT_TOPK = 1,
+  DLLM_COMMIT_EARLY_EXIT = 2
+} dllm_commit_mode;
 
 typedef struct {
   int32_t batch, n_layers, hidden, n_q_heads, n_kv_heads, head_dim, vocab;
@@ -108,7 +122,10 @@ typedef struct {
   int32_t steps_per_block; /* TOPK: 1 <= steps_per_block <= block.  THRESHOLD: a step cap
                             * per block when > 0 (the step that reaches it commits every
                             * row still masked; counted per sequence in the workspace by
-                            * dllm_decode_step / dllm_decode_block), none when <= 0 */
+                            * dllm_decode_step / dllm_decode_block), none when <= 0.
+                            * EARLY_EXIT: the same step cap */
+  float exit_tau;          /* EARLY_EXIT: confidence bound of converged rows, finite, >= 0
+                            * (>= tau: the THRESHOLD rule).  Unused otherwise. */
 } dllm_config;
 
 /* Kw = hidden (BF16) or 2*hidden (F32_SPLIT); Ko = Hq*D or 2*Hq*D. */

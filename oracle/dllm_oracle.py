@@ -54,7 +54,7 @@ import numpy as np
 
 MODE_NONE, MODE_PREFIX, MODE_DUAL, MODE_DUAL_PRUNED = 0, 1, 2, 3
 MODE_PREFIX_SUFFIXQ = 4   # prefix cache; block and suffix recomputed as queries every step
-COMMIT_THRESHOLD, COMMIT_TOPK = 0, 1
+COMMIT_THRESHOLD, COMMIT_TOPK, COMMIT_EARLY_EXIT = 0, 1, 2
 
 AMBIG_GAP = 1e-2     # top-2 logit gap below which an argmax is ambiguous
 AMBIG_CONF = 2e-3    # |conf - tau| (or forced-pick conf difference) band
@@ -235,12 +235,48 @@ def topk_ambiguity(conf, masked, k):
     return amb
 
 
+def early_exit_commit(conf: np.ndarray, tok: np.ndarray, prev_tok: np.ndarray,
+                      masked: np.ndarray, tau: float, exit_tau: float) -> np.ndarray:
+    """Threshold commit with an early exit for converged rows.
+
+    Streaming-dLLM's abstract (listing page, third abstract) names a dynamic,
+    confidence-aware strategy with an early exit that skips the remaining
+    iterations of converged tokens, without a formula.  Reading: a masked row
+    has converged when its argmax equals its argmax at the previous step of
+    the same block (prev_tok; -1 where there is none, as at a block's first
+    step); a converged row commits once its confidence exceeds exit_tau, a
+    bound at or below tau, instead of tau.  Rows with conf > tau commit as in
+    the plain rule, and the most confident masked row always commits (lowest
+    position on ties).  exit_tau >= tau gives the plain threshold rule.
+    Returns a bool [B].
+    """
+    stable = masked & (prev_tok >= 0) & (tok == prev_tok)
+    commit = masked & ((conf > tau) | (stable & (conf > exit_tau)))
+    if masked.any():
+        cand = np.where(masked, conf, -np.inf)
+        commit[int(np.argmax(cand))] = True
+    return commit
+
+
+def early_exit_ambiguity(conf, gap, tok, prev_tok, masked, tau, exit_tau):
+    """Flags of the early-exit rule: the threshold rule's bands, rows whose
+    confidence is within 2e-3 of exit_tau while their argmax repeats, and rows
+    whose argmax itself is ambiguous (top-2 gap < 1e-2) while their confidence
+    could clear exit_tau, since their 'repeats' test may go either way."""
+    amb_tok, amb_commit = ambiguity_flags(conf, gap, masked, tau)
+    has_prev = masked & (prev_tok >= 0)
+    stable = has_prev & (tok == prev_tok)
+    amb_commit = (amb_commit | (stable & (np.abs(conf - exit_tau) < AMBIG_CONF))
+                  | (has_prev & (gap < AMBIG_GAP) & (conf > exit_tau - AMBIG_CONF)))
+    return amb_tok, amb_commit
+
+
 def capped(cfg, step_in_block: int) -> bool:
     """Threshold rule with a step cap (steps_per_block > 0): the Fast-dLLM
     README's evaluation knobs bound the sampler's steps (diffusion_steps) next
     to the threshold; plainest reading: the step that reaches the cap commits
     every row still masked, so a block never takes more steps than that."""
-    return (cfg.commit_mode == COMMIT_THRESHOLD and cfg.steps_per_block > 0
+    return (cfg.commit_mode in (COMMIT_THRESHOLD, COMMIT_EARLY_EXIT) and cfg.steps_per_block > 0
             and step_in_block + 1 >= cfg.steps_per_block)
 
 
@@ -286,6 +322,7 @@ class Config:
     mask_id: int
     commit_mode: int = COMMIT_THRESHOLD
     steps_per_block: int = 0
+    exit_tau: float = 1.0   # COMMIT_EARLY_EXIT: confidence bound of converged rows
 
     @property
     def seq_len(self):
@@ -424,8 +461,12 @@ class StepResult:
 
 
 def decode_step(cfg: Config, W: Weights, st: State, plants: np.ndarray, s: int,
-                mirror: bool = True, apply: bool = True, step_in_block: int = 0) -> StepResult:
+                mirror: bool = True, apply: bool = True, step_in_block: int = 0,
+                prev_tok: Optional[np.ndarray] = None) -> StepResult:
     """One denoising step of the block at [s, s+B).
+
+    prev_tok [b, B]: the argmax of each row at the previous step of this block
+    (-1 where there is none), read by the early-exit rule only.
 
     The block rows run through every layer (their keys/values overwrite the
     cache at [s, s+B)), the LM head scores the masked rows, and the commit
@@ -477,6 +518,12 @@ def decode_step(cfg: Config, W: Weights, st: State, plants: np.ndarray, s: int,
             elif capped(cfg, step_in_block):
                 commit[bi] = m.copy()   # the step budget is spent: every masked row commits
                 amb_tok[bi] = m & (gap[bi] < AMBIG_GAP)
+            elif cfg.commit_mode == COMMIT_EARLY_EXIT:
+                pt = (np.full(B, -1, dtype=np.int64) if prev_tok is None
+                      else np.asarray(prev_tok[bi], dtype=np.int64))
+                commit[bi] = early_exit_commit(cm, tok[bi], pt, m, cfg.tau, cfg.exit_tau)
+                amb_tok[bi], amb_commit[bi] = early_exit_ambiguity(cm, gap[bi], tok[bi], pt, m,
+                                                                   cfg.tau, cfg.exit_tau)
             else:
                 commit[bi] = threshold_commit(cm, m, cfg.tau)
                 amb_tok[bi], amb_commit[bi] = ambiguity_flags(cm, gap[bi], m, cfg.tau)
@@ -523,11 +570,13 @@ def decode(cfg: Config, W: Weights, tokens, masked, starts, plants,
     steps_per_block, trace = [], []
     for s in range(cfg.prompt_len, cfg.seq_len, B):
         n = 0
+        prev = np.full((cfg.batch, B), -1, dtype=np.int64)   # argmax at the previous step
         while st.masked[:, s:s + B].any():
             if max_steps is not None and n >= max_steps:
                 break
-            r = decode_step(cfg, W, st, plants, s, mirror, step_in_block=n)
+            r = decode_step(cfg, W, st, plants, s, mirror, step_in_block=n, prev_tok=prev)
             trace.append((s, r))
+            prev = r.tok.copy()
             n += 1
         steps_per_block.append(n)
         refresh_block(cfg, W, st, s, mirror)

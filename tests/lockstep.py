@@ -38,10 +38,13 @@ def state_from_gpu(dec, layers=None) -> O.State:
 
 
 def compare_step(dec, case, s: int, rep: Report, check_kv: bool = True,
-                 step_in_block: int = 0) -> None:
+                 step_in_block: int = 0, prev_tok=None):
+    """One step compared; returns the GPU's argmax of the rows masked before
+    the step (-1 elsewhere), the previous-step argmax of the early-exit rule."""
     cfg, W = case.cfg, case.W
     st = state_from_gpu(dec)
-    r = O.decode_step(cfg, W, st, case.plants64, s, apply=False, step_in_block=step_in_block)
+    r = O.decode_step(cfg, W, st, case.plants64, s, apply=False, step_in_block=step_in_block,
+                      prev_tok=prev_tok)
     dec.step(s)
     torch.cuda.synchronize()
     assert dec.device_status() == 0
@@ -80,6 +83,7 @@ def compare_step(dec, case, s: int, rep: Report, check_kv: bool = True,
         got = f64(dec.v_cache[:, :, :, s:s + B])
         assert rel_l2(got, st.vcache[:, :, :, s:s + B]) <= 5e-3
     rep.steps += 1
+    return np.where(st.masked[:, s:s + B], tok, -1).astype(np.int64)
 
 
 def check_block_state(dec, masked_before, s: int, B: int) -> None:
@@ -132,10 +136,11 @@ def lockstep(dec, case, max_blocks: int | None = None, max_steps: int | None = N
         blocks = blocks[:max_blocks]
     for s in blocks:
         n = 0
+        prev = None
         while dec.masked[:, s:s + cfg.block].any():
             if max_steps is not None and n >= max_steps:
                 break
-            compare_step(dec, case, s, rep, step_in_block=n)
+            prev = compare_step(dec, case, s, rep, step_in_block=n, prev_tok=prev)
             n += 1
             assert n <= cfg.block
         compare_refresh(dec, case, s)
@@ -205,8 +210,10 @@ def lockstep_incremental(dec, case, max_blocks=None, log=None) -> Report:
     t0 = time.time()
     for s in blocks:
         n = 0
+        prev = None
         while st.masked[:, s:s + B].any():
-            r = O.decode_step(cfg, W, st, case.plants64, s, apply=False, step_in_block=n)
+            r = O.decode_step(cfg, W, st, case.plants64, s, apply=False, step_in_block=n,
+                              prev_tok=prev)
             dec.step(s)
             torch.cuda.synchronize()
             assert dec.device_status() == 0
@@ -237,6 +244,7 @@ def lockstep_incremental(dec, case, max_blocks=None, log=None) -> Report:
             assert rel_l2(got_v, st.vcache[:, :, :, s:s + B]) <= 5e-3
             st.kcache[:, :, :, s:s + B] = got_k
             st.vcache[:, :, :, s:s + B] = got_v
+            prev = np.where(st.masked[:, s:s + B], tok, -1).astype(np.int64)
             st.tokens = dec.tokens.cpu().numpy().astype(np.int64)
             st.masked = dec.masked.cpu().numpy().astype(bool)
             rep.steps += 1

@@ -14,7 +14,7 @@ def oracle_config(w: wl.Workload) -> O.Config:
                     vocab=w.vocab, prompt_len=w.prompt_len, gen_len=w.gen_len,
                     block=w.block, tau=w.tau, mode=w.mode, window=w.window,
                     rope_theta=w.rope_theta, mask_id=w.mask_id, commit_mode=w.commit_mode,
-                    steps_per_block=w.steps_per_block)
+                    steps_per_block=w.steps_per_block, exit_tau=w.exit_tau)
 
 
 def to64(t: torch.Tensor) -> np.ndarray:

@@ -103,7 +103,13 @@ def test_commit_mode_validation(lib):
     assert _status(topk.replace(steps_per_block=base.block)) == abi.DLLM_OK
     assert _status(topk.replace(steps_per_block=0)) == abi.DLLM_ERR_INVALID
     assert _status(topk.replace(steps_per_block=base.block + 1)) == abi.DLLM_ERR_INVALID
-    assert _status(base.replace(commit_mode=2)) == abi.DLLM_ERR_INVALID
+    ex = base.replace(commit_mode=wl.COMMIT_EARLY_EXIT)
+    assert _status(ex.replace(exit_tau=0.5)) == abi.DLLM_OK
+    assert _status(ex.replace(exit_tau=0.0)) == abi.DLLM_OK
+    assert _status(ex.replace(exit_tau=-0.1)) == abi.DLLM_ERR_INVALID
+    assert _status(ex.replace(exit_tau=float("nan"))) == abi.DLLM_ERR_INVALID
+    assert _status(ex.replace(exit_tau=float("inf"))) == abi.DLLM_ERR_INVALID
+    assert _status(base.replace(commit_mode=3)) == abi.DLLM_ERR_INVALID
     # the threshold rule ignores steps_per_block
     assert _status(base.replace(steps_per_block=-3)) == abi.DLLM_OK
 

@@ -124,6 +124,50 @@ def test_tiny_free_running_decode_equals_oracle_bit_exact(mode):
     assert steps == tr.steps_per_block
 
 
+EARLY_EXIT_CASES = {
+    # (workload, plant scale or None for the workload's draw, plant seed)
+    "prefix": (TINY.replace(commit_mode=wl.COMMIT_EARLY_EXIT, exit_tau=0.5), None, 35),
+    "nocache": (TINY.replace(commit_mode=wl.COMMIT_EARLY_EXIT, exit_tau=0.3,
+                             mode=wl.MODE_NONE), None, 35),
+    "converged": (TINY.replace(commit_mode=wl.COMMIT_EARLY_EXIT, exit_tau=0.5), 8.0, None),
+}
+
+
+@pytest.mark.parametrize("name", list(EARLY_EXIT_CASES))
+def test_early_exit_generation_equals_oracle_bit_exact(name):
+    """The early-exit commit rule (converged rows commit above exit_tau) on
+    the GPU, whole generations against a flag-free oracle decode: tokens and
+    steps per block bit for bit.  'converged' plants confidences between
+    exit_tau and tau, where every block takes exactly two steps."""
+    w, a, seed = EARLY_EXIT_CASES[name]
+    case = Case(w, a_override=a, noise=a is None, plant_seed=seed)
+    tr = case.decode()
+    assert state_flags(tr) == 0
+    if name == "converged":
+        assert tr.steps_per_block == [2] * (w.gen_len // w.block)
+    dec = make_decoder(case)
+    steps = dec.generate()
+    torch.cuda.synchronize()
+    assert dec.device_status() == 0
+    assert np.array_equal(dec.tokens.cpu().numpy(), tr.tokens)
+    assert steps == tr.steps_per_block
+    # a second generation from the reset state restarts the rule at the first
+    # block (the saved argmax of an earlier generation is not reused)
+    dec.reset()
+    assert dec.generate() == tr.steps_per_block
+    assert np.array_equal(dec.tokens.cpu().numpy(), tr.tokens)
+
+
+@pytest.mark.parametrize("name", ["llada_mid_dual", "dream_mid_prefix", "qwen_mid_pruned"])
+def test_lockstep_decode_early_exit(name):
+    case = Case(MID[name].replace(commit_mode=wl.COMMIT_EARLY_EXIT, exit_tau=0.5))
+    dec = make_decoder(case)
+    rep = lockstep(dec, case)
+    assert rep.steps >= (case.w.gen_len // case.w.block)
+    assert rep.flagged_mismatch <= max(2, rep.rows // 50)
+    assert not dec.masked.any()
+
+
 def test_tiny_free_running_decode_matches_oracle_up_to_first_flag():
     """The default plant draw flags rows (8 over the generation), so the two
     decodes may part at the first flagged step; every position settled before
@@ -363,6 +407,8 @@ PER_SEQ = {
     "batch_mid_dual_topk": MID["batch_mid_dual"].replace(commit_mode=wl.COMMIT_TOPK,
                                                          steps_per_block=4),
     "batch_mid_dual_cap": MID["batch_mid_dual"].replace(steps_per_block=3),
+    "batch_mid_dual_exit": MID["batch_mid_dual"].replace(commit_mode=wl.COMMIT_EARLY_EXIT,
+                                                         exit_tau=0.5),
 }
 
 

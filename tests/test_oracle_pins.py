@@ -584,3 +584,74 @@ def test_block_state_over_a_decode_with_tau_above_one():
         done, refresh = O.block_state(before, masked[0, s:s + B], s)
         k = k + 1 if k < B else 1
         assert done == (k == B) and refresh == (s if k == B else -1)
+
+
+# ---------------------------------------------------------------- early exit
+def test_early_exit_commit_cases():
+    tau, ex = 0.9, 0.5
+    conf = np.array([0.60, 0.60, 0.95, 0.40, 0.70, 0.55])
+    tok = np.array([3, 4, 5, 6, 7, 8])
+    prev = np.array([3, 9, 1, 6, -1, 8])      # rows 0, 3, 5 repeat; row 4 has no previous
+    masked = np.array([True, True, True, True, True, False])
+    c = O.early_exit_commit(conf, tok, prev, masked, tau, ex)
+    # 0: repeats and clears exit_tau; 1: changed; 2: clears tau; 3: repeats but
+    # below exit_tau; 4: no previous step; 5: not masked
+    assert c.tolist() == [True, False, True, False, False, False]
+    # the most confident masked row commits even when nothing else does
+    c = O.early_exit_commit(np.array([0.3, 0.4]), np.array([1, 2]), np.array([-1, -1]),
+                            np.ones(2, bool), tau, ex)
+    assert c.tolist() == [False, True]
+    # exit_tau at tau: the plain threshold rule
+    for _ in range(50):
+        conf = RNG.uniform(0, 1, 12)
+        tok = RNG.integers(0, 3, 12)
+        prev = RNG.integers(-1, 3, 12)
+        masked = RNG.uniform(size=12) < 0.8
+        masked[0] = True
+        np.testing.assert_array_equal(O.early_exit_commit(conf, tok, prev, masked, tau, tau),
+                                      O.threshold_commit(conf, masked, tau))
+
+
+def test_early_exit_finishes_converged_blocks_in_two_steps():
+    # planted confidences between exit_tau and tau, argmax fixed by the plant:
+    # the threshold rule commits one forced row per step (B steps per block);
+    # with the early exit every other row has repeated its argmax by the
+    # second step and commits there
+    base = TINY.replace(tau=0.9)
+    thr = Case(base, a_override=8.0, noise=False).decode()
+    assert thr.steps_per_block == [base.block] * (base.gen_len // base.block)
+    ex = base.replace(commit_mode=wl.COMMIT_EARLY_EXIT, exit_tau=0.5)
+    tr = Case(ex, a_override=8.0, noise=False).decode()
+    assert tr.steps_per_block == [2] * (base.gen_len // base.block)
+    # converged rows commit the token they repeated: the same sequence
+    np.testing.assert_array_equal(tr.tokens, thr.tokens)
+
+
+def test_early_exit_at_or_above_tau_is_the_threshold_decode():
+    base = TINY
+    thr = Case(base).decode()
+    ex = Case(base.replace(commit_mode=wl.COMMIT_EARLY_EXIT, exit_tau=base.tau)).decode()
+    assert ex.steps_per_block == thr.steps_per_block
+    np.testing.assert_array_equal(ex.tokens, thr.tokens)
+
+
+def test_early_exit_decode_invariants():
+    w = TINY.replace(commit_mode=wl.COMMIT_EARLY_EXIT, exit_tau=0.3)
+    tr = Case(w).decode()
+    B = w.block
+    assert not (tr.tokens == -1).any()
+    prev_block, prev = None, None
+    for s, r in tr.steps:
+        if s != prev_block:
+            prev_block, prev = s, None
+        m = ~np.isnan(r.conf[0])
+        c = r.commit[0]
+        assert c.any() and not (c & ~m).any()
+        # every committed row cleared tau, repeated its argmax above exit_tau,
+        # or is the forced pick
+        best = int(np.argmax(np.where(m, r.conf[0], -np.inf)))
+        for i in np.where(c)[0]:
+            rep_ = prev is not None and prev[i] == r.tok[0, i]
+            assert r.conf[0, i] > w.tau or (rep_ and r.conf[0, i] > w.exit_tau) or i == best
+        prev = r.tok[0].copy()
+    assert all(1 <= n <= B for n in tr.steps_per_block)
