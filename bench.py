@@ -258,40 +258,92 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- oracle timing
-def oracle_sample(w, weights, tokens, masked, starts, plants, budget_s=20.0):
-    """Time the fp64 oracle on this host: denoising steps of the first block,
-    from the prefilled state where the workload is small enough, else from
-    zero caches (the step's arithmetic does not depend on the cache values).
-    Returns (seconds per step, steps, rows committed, threads)."""
-    import numpy as np
-    import torch
-    from oracle import dllm_oracle as O
+def _host_threads():
+    """(BLAS threads numpy uses, cores this process may run on)."""
+    import numpy  # noqa: F401  (loads the BLAS library threadpoolctl inspects)
+    from threadpoolctl import threadpool_info
+    blas = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
+    return (max(blas) if blas else 1), len(os.sched_getaffinity(0))
 
-    cfg = O.Config(batch=w.batch, n_layers=w.n_layers, hidden=w.hidden, n_q_heads=w.n_q_heads,
-                   n_kv_heads=w.n_kv_heads, head_dim=w.head_dim, vocab=w.vocab,
-                   prompt_len=w.prompt_len, gen_len=w.gen_len, block=w.block, tau=w.tau,
-                   mode=w.mode, window=w.window, rope_theta=w.rope_theta, mask_id=w.mask_id,
-                   commit_mode=w.commit_mode, steps_per_block=w.steps_per_block,
-                   exit_tau=w.exit_tau)
-    W = O.Weights(lambda l: weights.wqkv[l].cpu().double().numpy(),
-                  lambda l: weights.wo[l].cpu().double().numpy(),
-                  weights.w_lm.cpu().double().numpy())
-    st = O.new_state(cfg, tokens.numpy(), masked.numpy().astype(bool), starts.numpy())
-    small = w.n_layers * w.hidden * w.hidden <= 64 * 1024 * 1024
-    if small:
-        O.prefill(cfg, W, st)
-    plants64 = plants.h.double().cpu().numpy()
-    s = w.prompt_len
-    t0 = time.perf_counter()
-    n, committed = 0, 0
-    while st.masked[:, s:s + w.block].any():
-        r = O.decode_step(cfg, W, st, plants64, s)
-        n += 1
-        committed += int(r.commit.sum())
-        if time.perf_counter() - t0 > budget_s:
-            break
-    dt = time.perf_counter() - t0
-    return dt / n, n, committed, torch.get_num_threads()
+
+class OracleTimer:
+    """The fp64 oracle on this host's cores, timed on the workload's own
+    inputs: host copies of the weights (each layer converted to fp64 when the
+    oracle asks for it, as in the tests), the oracle's prefill of the caches,
+    then denoising steps of the first block.  Both bench legs that time the
+    oracle (our arm's cpu_baseline and the reference arm) use this, with the
+    same definition: rows the oracle commits / seconds of its steps."""
+
+    def __init__(self, w, weights, tokens, masked, starts, plants):
+        import numpy as np
+        from oracle import dllm_oracle as O
+        self.O, self.w = O, w
+        self.cfg = O.Config(batch=w.batch, n_layers=w.n_layers, hidden=w.hidden,
+                            n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads, head_dim=w.head_dim,
+                            vocab=w.vocab, prompt_len=w.prompt_len, gen_len=w.gen_len,
+                            block=w.block, tau=w.tau, mode=w.mode, window=w.window,
+                            rope_theta=w.rope_theta, mask_id=w.mask_id,
+                            commit_mode=w.commit_mode, steps_per_block=w.steps_per_block,
+                            exit_tau=w.exit_tau)
+        self.wqkv, self.wo = weights.wqkv.cpu(), weights.wo.cpu()
+        self.W = O.Weights(lambda l: self.wqkv[l].double().numpy(),
+                           lambda l: self.wo[l].double().numpy(),
+                           weights.w_lm.cpu().double().numpy())
+        self.tokens0 = tokens.numpy().copy()
+        self.masked0 = masked.numpy().astype(bool).copy()
+        self.st = O.new_state(self.cfg, self.tokens0, self.masked0, starts.numpy())
+        self.plants64 = plants.h.double().cpu().numpy()
+        t0 = time.perf_counter()
+        O.prefill(self.cfg, self.W, self.st)
+        self.prefill_s = time.perf_counter() - t0
+        self.n = 0
+        self.prev = None
+
+    def steps(self, budget_s):
+        """Denoising steps of the first block until budget_s has passed (at
+        least one); a finished block restarts from the prefilled state.
+        Returns (seconds, steps, rows committed)."""
+        O, s, B = self.O, self.w.prompt_len, self.w.block
+        t0 = time.perf_counter()
+        n = c = 0
+        while True:
+            if not self.st.masked[:, s:s + B].any():
+                self.st.tokens[:] = self.tokens0
+                self.st.masked[:] = self.masked0
+                self.n, self.prev = 0, None
+            r = O.decode_step(self.cfg, self.W, self.st, self.plants64, s,
+                              step_in_block=self.n, prev_tok=self.prev)
+            self.prev = r.tok.copy()
+            self.n += 1
+            n += 1
+            c += int(r.commit.sum())
+            if time.perf_counter() - t0 > budget_s:
+                return time.perf_counter() - t0, n, c
+
+    def one_thread_step_s(self):
+        """Seconds of one denoising step with one BLAS thread, extrapolated
+        from steps of the first one and two layers (same rows, keys and LM
+        head): L * (t2 - t1) + (2 t1 - t2); timed directly for L <= 2."""
+        import dataclasses
+        from threadpoolctl import threadpool_limits
+        O, s = self.O, self.w.prompt_len
+        t = []
+        with threadpool_limits(1):
+            if self.w.n_layers <= 2:  # short stacks: time the step itself
+                st = O.State(self.st.tokens.copy(), self.st.masked.copy(), self.st.kcache.copy(),
+                             self.st.vcache.copy(), self.st.starts)
+                t0 = time.perf_counter()
+                O.decode_step(self.cfg, self.W, st, self.plants64, s, apply=False)
+                return time.perf_counter() - t0
+            for L in (1, 2):
+                cfg = dataclasses.replace(self.cfg, n_layers=L)
+                st = O.State(self.st.tokens.copy(), self.st.masked.copy(),
+                             self.st.kcache[:L].copy(), self.st.vcache[:L].copy(), self.st.starts)
+                t0 = time.perf_counter()
+                O.decode_step(cfg, self.W, st, self.plants64, s, apply=False)
+                t.append(time.perf_counter() - t0)
+        per_layer = max(t[1] - t[0], 0.0)
+        return self.w.n_layers * per_layer + max(2 * t[0] - t[1], 0.0)
 
 
 def run_reference(args, rank, world):
@@ -301,31 +353,40 @@ def run_reference(args, rank, world):
     import torch
     from diffusion_decoding_step_b200 import workload as wl
     w = selected_workload(args)
-    weights = wl.make_weights(w, device="cpu")
+    # the same seeded draw as our arm (its generator runs on the GPU when there
+    # is one); the timed work is the oracle's alone
+    dev = "cuda" if torch.cuda.is_available() and w.name != "tiny" else "cpu"
+    weights = wl.make_weights(w, device=dev)
     tokens, masked = wl.make_tokens(w)
     starts = wl.seq_starts(w)
     plants = wl.make_plants(w, weights.w_lm)
-    step_s = []
-    commits = 0
-    steps = 0
+    timer = OracleTimer(w, weights, tokens, masked, starts, plants)
+    del weights
     for _ in range(args.warmup):
-        oracle_sample(w, weights, tokens, masked, starts, plants, budget_s=5.0)
+        timer.steps(5.0)
+    secs = commits = steps = 0
     for _ in range(args.steps):
-        sp, n, c, thr = oracle_sample(w, weights, tokens, masked, starts, plants, budget_s=20.0)
-        step_s.append(sp * n)
-        commits += c
+        t, n, c = timer.steps(20.0)
+        secs += t
         steps += n
-    total = sum(step_s)
-    value = commits / total
-    sample = (f"first block of {w.name}: {steps} oracle denoising steps over {args.steps} "
-              f"timed samples (each <= 20 s), {commits} rows committed")
+        commits += c
+    value = commits / secs
+    thr, cores = _host_threads()
+    one = timer.one_thread_step_s()
+    sample = (f"first block of {w.name} from the oracle's own prefill ({timer.prefill_s:.1f} s, "
+              f"not timed): {steps} fp64 denoising steps over {args.steps} timed samples "
+              f"(each >= 20 s of steps), {commits} rows committed; {thr} BLAS threads on "
+              f"{cores} cores; one thread: {one:.3g} s per step ("
+              + ("extrapolated from 1- and 2-layer steps" if w.n_layers > 2 else "timed") + ")")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": 1000.0 * total / args.steps, "higher_is_better": True,
+            "ms_per_step": 1000.0 * secs / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": workload_config(w, "cpu"),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": thr, "kind": "oracle",
-                             "sample": sample},
+                             "sample": sample, "s_per_step": secs / steps,
+                             "one_thread_s_per_step": one,
+                             "one_thread_tokens_per_s": (commits / steps) / one if one > 0 else None},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -493,14 +554,20 @@ def run_ours(args, rank, world, local_rank):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        wc = weights
-        sp, n, c, thr = oracle_sample(w, wc, tokens, masked, starts, plants, budget_s=20.0)
-        per_step_commit = w.batch * w.gen_len * args.steps / max(1, denoise_steps)
-        cpu = {"value": per_step_commit / sp, "unit": "tokens/s", "cores": thr,
-               "kind": "oracle",
-               "sample": (f"{n} oracle denoising steps of the first block of {w.name} "
-                          f"({sp:.2f} s each, fp64); tokens/s = the GPU run's mean commits per "
-                          f"step ({per_step_commit:.2f}) / oracle step time")}
+        timer = OracleTimer(w, weights, tokens, masked, starts, plants)
+        t, n, c = timer.steps(20.0)
+        thr, cores = _host_threads()
+        one = timer.one_thread_step_s()
+        cpu = {"value": c / t, "unit": "tokens/s", "cores": thr, "kind": "oracle",
+               "s_per_step": t / n, "one_thread_s_per_step": one,
+               "one_thread_tokens_per_s": (c / n) / one if one > 0 else None,
+               "sample": (f"{n} fp64 oracle denoising steps of the first block of {w.name} "
+                          f"from the oracle's own prefill ({timer.prefill_s:.1f} s, not timed), "
+                          f"{c} rows committed; tokens/s = rows the oracle committed / seconds "
+                          f"of its steps; {thr} BLAS threads on {cores} cores; one thread "
+                          + ("extrapolated from 1- and 2-layer steps" if w.n_layers > 2
+                             else "timed"))}
+        del timer
 
     if rank == 0:
         line = {
