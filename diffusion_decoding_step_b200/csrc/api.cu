@@ -338,7 +338,24 @@ std::vector<int> row_counts(const Shape& s) {
   return r;
 }
 
+Layout compute_layout(const Shape& s);
+
+// The workspace layout of a shape, computed once and then looked up: every
+// entry point needs it, and planning the layer-stack partition for every block
+// costs more host time than a projection kernel takes on the GPU.
 Layout layout(const Shape& s) {
+  static std::mutex mu;
+  static std::vector<std::pair<Shape, Layout>> memo;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const auto& e : memo)
+    if (memcmp(&e.first, &s, sizeof(Shape)) == 0) return e.second;
+  const Layout l = compute_layout(s);
+  if (memo.size() >= 64) memo.erase(memo.begin());
+  memo.emplace_back(s, l);
+  return l;
+}
+
+Layout compute_layout(const Shape& s) {
   Layout l{};
   size_t off = 0;
   auto take = [&](size_t bytes) {

@@ -37,11 +37,15 @@ struct GemmCfg {
   // one CTA per SM and a deep ring.  The O-projection (one CTA per SM) takes
   // four stages (about 90 KB), which still fits beside the attention kernel
   // before it; the Q/K/V projection keeps about 70 KB per CTA so that it runs
-  // two or three CTAs per SM.  (Three O-projection stages, which would let
-  // two Q/K/V CTAs start beside it, measured slower.)
+  // two or three CTAs per SM; split across more CTAs than SMs it takes five
+  // stages (about 110 KB with the receive buffer in the ring), which still fit
+  // beside the O-projection and measured 1.4 % faster per LLaDA-8B-shaped step
+  // than four.  (Three O-projection stages, which would let two Q/K/V CTAs
+  // start beside it, measured slower; six Q/K/V stages no longer fit beside
+  // it and measured 20 % slower.)
   static constexpr int kStages = EPI == EPI_LMHEAD     ? (NT <= 64 ? 8 : NT <= 128 ? 6 : 4)
                                  : EPI == EPI_OPROJ   ? 4
-                                 : EPI == EPI_QKV_DEEP ? 4
+                                 : EPI == EPI_QKV_DEEP ? (NT <= 64 ? 5 : 4)
                                                       : (NT <= 64 ? 3 : 4);
   static constexpr int kWBytes = 128 * 64 * 2;
   static constexpr int kXBytes = NT * 64 * 2;

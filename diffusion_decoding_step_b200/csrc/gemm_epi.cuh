@@ -2,9 +2,9 @@
 // and cache store; O-projection with residual add and per-slice sums of
 // squares; LM head with a running max / sum-exp / argmax / second max),
 // shared by the per-projection GEMM kernel and the persistent layer-stack
-// kernel.  Values another CTA of the same launch may have written (the
-// residual, its sums of squares) are read with L2-only loads, so that no
-// stale L1 line is used inside a persistent kernel.
+// kernel.  In the persistent kernel (XCTA = true) values another CTA of the
+// same launch may have written (the residual, its sums of squares) are read
+// with L2-only loads, so that no stale L1 line is used.
 #pragma once
 #include <float.h>
 #include <limits.h>
@@ -58,7 +58,14 @@ __device__ __forceinline__ float column_sum16(const float* stage, int et) {
 // (from the partial sums of squares), rp[c] = rotary position, and the row
 // parts of the destination offsets in units of head_dim, qoff[c] into q and
 // koff[c] into the caches (the head / kv-head parts are added per weight row).
-template <int NT, int EPI>
+// Load of a value another CTA of the same launch may have written.
+template <bool XCTA>
+__device__ __forceinline__ float ld_shared_f32(const float* p) {
+  if constexpr (XCTA) return __ldcg(p);
+  return *p;
+}
+
+template <int NT, int EPI, bool XCTA = false>
 __device__ __forceinline__ void epi_prepare(const GemmParams& p, int layer, int n, int et,
                                             float* inv, int* rp) {
   if constexpr (EPI == EPI_QKV) {
@@ -72,7 +79,7 @@ __device__ __forceinline__ void epi_prepare(const GemmParams& p, int layer, int 
       if (p.sumsq_in != nullptr && xrow < p.R) {
         const float* src = p.sumsq_in + (size_t)xrow * p.npart;
 #pragma unroll 8
-        for (int k = sub; k < p.npart; k += TPC) s += __ldcg(src + k);
+        for (int k = sub; k < p.npart; k += TPC) s += ld_shared_f32<XCTA>(src + k);
       }
 #pragma unroll
       for (int o = 1; o < TPC; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
@@ -99,14 +106,14 @@ __device__ __forceinline__ void epi_prepare(const GemmParams& p, int layer, int 
 // O-projection: the residual entries x[n*NT + c0 + i][m*128 + wl] a chunk
 // adds to.  The previous kernels are complete once the dependency wait has
 // returned, so these loads may run while the mainloop is still streaming.
-template <int NT>
+template <int NT, bool XCTA = false>
 __device__ __forceinline__ void oproj_load_x(const GemmParams& p, int m, int n, int c0, int wl,
                                              float (&xo)[16]) {
   const int wrow = m * 128 + wl;
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const int xrow = n * NT + c0 + i;
-    xo[i] = xrow < p.R ? __ldcg(p.x + (size_t)xrow * p.d_model + wrow) : 0.f;
+    xo[i] = xrow < p.R ? ld_shared_f32<XCTA>(p.x + (size_t)xrow * p.d_model + wrow) : 0.f;
   }
 }
 

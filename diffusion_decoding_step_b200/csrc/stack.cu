@@ -554,7 +554,8 @@ __global__ void __launch_bounds__(kStackThreads, 1)
           if (last) {
             // the tile is complete: add the contributors' partials in k order
             float* inv = reinterpret_cast<float*>(run);
-            if (ph == 0) epi_prepare<NT, EPI_QKV>(gp, l, 0, et, inv, reinterpret_cast<int*>(inv + NT));
+            if (ph == 0)
+              epi_prepare<NT, EPI_QKV, true>(gp, l, 0, et, inv, reinterpret_cast<int*>(inv + NT));
 #pragma unroll 1
             for (int c0 = 0; c0 < NT; c0 += 16) {
               float own[16], v[16], xo[16];
@@ -597,7 +598,7 @@ __global__ void __launch_bounds__(kStackThreads, 1)
               if (ph == 0) {
                 epi_chunk<NT, EPI_QKV>(gp, sg.tile, 0, c0, wl, et, v, xo, stage, run);
               } else {
-                oproj_load_x<NT>(gp, sg.tile, 0, c0, wl, xo);
+                oproj_load_x<NT, true>(gp, sg.tile, 0, c0, wl, xo);
                 epi_chunk<NT, EPI_OPROJ>(gp, sg.tile, 0, c0, wl, et, v, xo, stage, run);
               }
             }
