@@ -180,7 +180,7 @@ def gemm_source_sha1():
     """Digest of the GEMM kernel's sources, to tie stored ncu counters to them."""
     import hashlib
     h = hashlib.sha1()
-    for name in ("gemm.cu", "kernels.cuh", "ptx.cuh"):
+    for name in ("gemm.cu", "gemm_epi.cuh", "kernels.cuh", "ptx.cuh"):
         with open(os.path.join(ROOT, "diffusion_decoding_step_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
