@@ -196,30 +196,37 @@ GemmPlan plan_lmhead(int V, int R, int K) {
   return g;
 }
 
+// Extra plan cost (in key tiles) that 32-row attention tiles may have over
+// 128-row tiles and still be chosen for groups of more than 32 rows.
+constexpr int kAttnSgSlack = 1;
+// SMs a key-chunk plan counts as one wave.  Fewer than the 148 SMs: the
+// O-projection that follows starts its CTAs on the SMs that attention leaves
+// free and streams its weights before its dependency wait.  Measured on the
+// Dream-7B-shaped first block: 7 x 4 row tiles x 5 chunks (140 CTAs) 1171 us
+// per step, x 3 chunks of 2 tiles (84 CTAs) 1026 us.
+constexpr int kAttnSMs = 128;
+
 struct AttnPlan {
   int row_tiles, chunks, tpc;
+  bool sg;  // row tiles of 32 rows (the attention kernel's small-group mode)
 };
 
-AttnPlan plan_attn(const Shape& s, int n_rows, int ntile_bound) {
-  AttnPlan a;
-  const int g = s.Hq / s.Hkv;
-  a.row_tiles = cdiv(g * n_rows, 128);
-  const int base = s.b * s.Hkv * a.row_tiles;
-  // Key chunks per row tile: the chunks form one cluster and merge on chip.
-  // At most 8 for head_dim 128 and 6 for head_dim 32 (the merge buffer must
-  // fit in the K/V/P region).  Seven head_dim-128 chunks would not fit either,
-  // so they run as eight, the last one without keys.
-  // While the row tiles alone leave SMs idle, the chunk count minimises
-  // waves x key tiles per chunk (one CTA per SM: the K/V ring and P take
-  // most of the shared memory), counting each merge as one more tile, so a
-  // second wave of CTAs costs as much as the first.  Once the row tiles fill
-  // the SMs, splitting the keys only adds merges (measured +15 % on a
-  // 16-sequence batch).
+// Key chunks per row tile for `base` row tiles: the chunks form one cluster
+// and merge on chip.  At most 8 for head_dim 128 and 6 for head_dim 32 (the
+// merge buffer must fit in the K/V/P region).  Seven head_dim-128 chunks would
+// not fit either, so they run as eight, the last one without keys.
+// While the row tiles alone leave SMs idle, the chunk count minimises
+// waves x key tiles per chunk (one CTA per SM: the K/V ring and P take most
+// of the shared memory), counting each merge as one more tile, so a second
+// wave of CTAs costs as much as the first.  Once the row tiles fill the SMs,
+// splitting the keys only adds merges (measured +15 % on a 16-sequence batch).
+AttnPlan plan_chunks(const Shape& s, int base, int ntile_bound, long long* cost_out) {
+  AttnPlan a{};
   const int cap = base >= kNumSMs ? 1 : s.D == 128 ? 8 : 6;
   int chunks = 1;
   long long best = 1ll << 62;
   for (int c = 1; c <= std::min(ntile_bound, cap); ++c) {
-    const long long waves = cdiv(base * c, kNumSMs);
+    const long long waves = cdiv((long long)base * c, kAttnSMs);
     const long long cost = waves * cdiv(ntile_bound, c) + (c > 1 ? 1 : 0);
     if (cost < best) {
       best = cost;
@@ -229,6 +236,30 @@ AttnPlan plan_attn(const Shape& s, int n_rows, int ntile_bound) {
   a.tpc = cdiv(ntile_bound, chunks);
   a.chunks = cdiv(ntile_bound, a.tpc);
   if (a.chunks == 7) a.chunks = 8;
+  *cost_out = best;
+  return a;
+}
+
+AttnPlan plan_attn(const Shape& s, int n_rows, int ntile_bound) {
+  const int g = s.Hq / s.Hkv;
+  const int gr = g * n_rows;
+  long long cost128 = 0, cost32 = 0;
+  AttnPlan a = plan_chunks(s, s.b * s.Hkv * cdiv(gr, 128), ntile_bound, &cost128);
+  a.row_tiles = cdiv(gr, 128);
+  a.sg = false;
+  if (s.D != 128) return a;
+  // Row tiles of 32 rows, each loaded four times so that every warp takes a
+  // quarter of the keys and of the output columns: always for groups of at
+  // most 32 rows (same grid, a quarter of the softmax per thread); for larger
+  // groups while their plan costs at most one tile more than 128-row tiles
+  // (its tiles and merges are the cheaper ones).
+  const int rt32 = cdiv(gr, 32);
+  const AttnPlan b = plan_chunks(s, s.b * s.Hkv * rt32, ntile_bound, &cost32);
+  if (gr <= 32 || cost32 <= cost128 + kAttnSgSlack) {
+    a = b;
+    a.row_tiles = rt32;
+    a.sg = true;
+  }
   return a;
 }
 
@@ -639,7 +670,8 @@ dllm_status run_attn(const Ctx& c, int layer, int n_rows, const void* q, const v
   const int box_d = s.D >= 64 ? 64 : s.D;
   const CUtensorMapSwizzle sw = s.D >= 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   CUtensorMap qm, km, vm;
-  if (!make_map(&qm, q, s.D, (uint64_t)g * n_rows, (uint64_t)s.b * s.Hkv, box_d, 128, sw) ||
+  const uint32_t q_box = a.sg ? 32 : 128;
+  if (!make_map(&qm, q, s.D, (uint64_t)g * n_rows, (uint64_t)s.b * s.Hkv, box_d, q_box, sw) ||
       !make_map(&km, kc, s.D, s.S, (uint64_t)s.L * s.b * s.Hkv, box_d, kKeyTile, sw) ||
       !make_map(&vm, vc, s.D, s.S, (uint64_t)s.L * s.b * s.Hkv, box_d, kKeyTile, sw))
     return DLLM_ERR_CUDA;
@@ -653,6 +685,7 @@ dllm_status run_attn(const Ctx& c, int layer, int n_rows, const void* q, const v
   p.n_rows = n_rows;
   p.group_rows = g * n_rows;
   p.row_tiles = a.row_tiles;
+  p.small_group = a.sg ? 1 : 0;
   p.chunks = a.chunks;
   p.tiles_per_chunk = a.tpc;
   p.segs = keys.segs;

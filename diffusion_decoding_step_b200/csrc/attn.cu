@@ -24,6 +24,15 @@
 // its O by its share of the merged softmax and sends each 16-column group to
 // the CTA that owns the group, which adds the chunks' contributions in chunk
 // order and writes the bf16 output.  No partial goes through global memory.
+//
+// Small row tiles (32 query rows of a kv head's group, head_dim 128): the 32
+// rows are loaded four times into the 128-row Q tile, so S holds each row in
+// four TMEM lanes 32w + i, one per warp w.  Warp w takes keys [32w, 32w+32)
+// of every row in the softmax (the row max is exchanged once per tile through
+// shared memory) and writes its quarter of P into all four copies of the row,
+// so every lane of O = P V holds its full row and warp w reads, scales and
+// stores output columns [32w, 32w+32).  Each thread then works on 32 keys and
+// 32 output columns instead of 128, and all four warps share the merge.
 #include <float.h>
 
 #include "kernels.cuh"
@@ -46,8 +55,9 @@ struct AttnCfg {
   static constexpr int kPBytes = 128 * kKeys * 2;     // two 128B-swizzle atom columns
   static constexpr int kTmemCols = 256;               // S [0,128), O [128,128+D)
   static constexpr int kMlBytes = kMaxMerge * 128 * 8;  // (max, sum) of every chunk's rows
+  static constexpr int kXBytes = 2 * 128 * 4;  // small groups: quarter maxima and sums
   static constexpr size_t kSmem =
-      1024 + kQBytes + ST * 2 * kKVBytes + kPBytes + kMlBytes + 128 + 64;
+      1024 + kQBytes + ST * 2 * kKVBytes + kPBytes + kMlBytes + kXBytes + 128 + 64;
   // The merge reuses the K/V/P region once every chunk's last P V is done:
   // [src chunk][owned group][4 float4][128 rows] fp32 for up to kMaxMerge chunks.
   static constexpr int kGroups = D / 16;
@@ -114,11 +124,12 @@ __device__ __forceinline__ void tile_of(const int* sg, int t, int& start, int& n
   }
 }
 
-template <int D, int ST>
+template <int D, int ST, bool SG>
 __global__ void __launch_bounds__(128, 1)
     attn_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                 const __grid_constant__ CUtensorMap vmap, const AttnParams p) {
   using C = AttnCfg<D, ST>;
+  static_assert(!SG || D == 128, "small groups: one 32-key quarter and 32 columns per warp");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -127,7 +138,8 @@ __global__ void __launch_bounds__(128, 1)
   uint8_t* v_s = k_s + ST * C::kKVBytes;           // [ST]
   uint8_t* p_s = v_s + ST * C::kKVBytes;
   float2* ml_s = reinterpret_cast<float2*>(p_s + C::kPBytes);  // [kMaxMerge][128]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(p_s + C::kPBytes + C::kMlBytes);
+  float* x_s = reinterpret_cast<float*>(p_s + C::kPBytes + C::kMlBytes);  // [2][4 warps][32]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(p_s + C::kPBytes + C::kMlBytes + C::kXBytes);
   uint64_t* bar_q = bars;
   uint64_t* bar_s = bars + 1;
   uint64_t* bar_o = bars + 2;
@@ -228,8 +240,16 @@ __global__ void __launch_bounds__(128, 1)
   if (t == 0 && my_tiles > 0) {
     mbar_arrive_expect_tx(bar_q, C::kQBytes);
 #pragma unroll
-    for (int bx = 0; bx < C::kNBox; ++bx)
-      tma_load_3d(q_s + bx * C::kBoxBytes, &qmap, bar_q, bx * C::kBoxD, rt * 128, zq);
+    for (int bx = 0; bx < C::kNBox; ++bx) {
+      if constexpr (SG) {  // four copies of the (at most) 32 rows; the map's box is 32 rows
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          tma_load_3d(q_s + bx * C::kBoxBytes + c * 32 * C::kRowBytes, &qmap, bar_q,
+                      bx * C::kBoxD, rt * 32, zq);
+      } else {
+        tma_load_3d(q_s + bx * C::kBoxBytes, &qmap, bar_q, bx * C::kBoxD, rt * 128, zq);
+      }
+    }
     for (int j = 0; j < min(my_tiles, ST); ++j) {
       if (pre & (1u << j)) continue;
       int start, nv;
@@ -270,54 +290,109 @@ __global__ void __launch_bounds__(128, 1)
       break;
     }
     tc_fence_after();
-    // ---- softmax of row t over the tile (log2 domain), one TMEM read
-    float s[kKeys];
+    if constexpr (SG) {
+      // ---- softmax of row (t & 31) over keys [32w, 32w+32) of the tile
+      const int kq = warp * 32;
+      float s[32];
+      tmem_ld32(s_tmem + lane_off + kq, s);
+      tmem_ld_wait();
+      float tm[4] = {-FLT_MAX, -FLT_MAX, -FLT_MAX, -FLT_MAX};
 #pragma unroll
-    for (int c = 0; c < kKeys / 32; ++c) tmem_ld32(s_tmem + lane_off + c * 32, s + c * 32);
-    tmem_ld_wait();
-    // independent partial maxima and sums: one warp per scheduler has no
-    // other work to hide a serial dependency chain behind
-    float tm[4] = {-FLT_MAX, -FLT_MAX, -FLT_MAX, -FLT_MAX};
+      for (int i = 0; i < 32; ++i)
+        if (kq + i < nvalid) tm[i & 3] = fmaxf(tm[i & 3], s[i]);
+      x_s[t] = fmaxf(fmaxf(tm[0], tm[1]), fmaxf(tm[2], tm[3]));
+      __syncthreads();
+      const int i0 = t & 31;
+      const float tmax = fmaxf(fmaxf(x_s[i0], x_s[32 + i0]), fmaxf(x_s[64 + i0], x_s[96 + i0]));
+      const float m_new = fmaxf(m_run, tmax * p.scale_log2);
+      const float alpha = fast_exp2(m_run - m_new);
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int i = 0; i < kKeys; ++i)
-      if (i < nvalid) tm[i & 3] = fmaxf(tm[i & 3], s[i]);
-    const float tmax = fmaxf(fmaxf(tm[0], tm[1]), fmaxf(tm[2], tm[3]));
-    const float m_new = fmaxf(m_run, tmax * p.scale_log2);
-    const float alpha = fast_exp2(m_run - m_new);
-    float ls[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int c = 0; c < 4; ++c) {  // 8 keys = one 16-byte chunk of P
+        uint32_t pk[4];
 #pragma unroll
-    for (int c = 0; c < kKeys / 8; ++c) {  // 8 keys = one 16-byte chunk of P
-      uint32_t pk[4];
+        for (int i = 0; i < 8; i += 2) {
+          const int k0 = c * 8 + i;
+          const float p0 = kq + k0 < nvalid ? fast_exp2(s[k0] * p.scale_log2 - m_new) : 0.f;
+          const float p1 =
+              kq + k0 + 1 < nvalid ? fast_exp2(s[k0 + 1] * p.scale_log2 - m_new) : 0.f;
+          const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+          ls[c] += __low2float(h2) + __high2float(h2);
+          pk[i >> 1] = *reinterpret_cast<const uint32_t*>(&h2);
+        }
+        // the chunk goes into all four copies 32r + i0 of the row (same swizzle phase)
+        const int key = kq + c * 8;
+        uint8_t* pcol = p_s + (key >> 6) * (128 * 128) + ((((key & 63) >> 3) ^ (i0 & 7)) << 4);
 #pragma unroll
-      for (int i = 0; i < 8; i += 2) {
-        const int k0 = c * 8 + i;
-        const float p0 = k0 < nvalid ? fast_exp2(s[k0] * p.scale_log2 - m_new) : 0.f;
-        const float p1 = k0 + 1 < nvalid ? fast_exp2(s[k0 + 1] * p.scale_log2 - m_new) : 0.f;
-        const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-        ls[c & 3] += __low2float(h2) + __high2float(h2);
-        pk[i >> 1] = *reinterpret_cast<const uint32_t*>(&h2);
+        for (int r = 0; r < 4; ++r)
+          *reinterpret_cast<uint4*>(pcol + (r * 32 + i0) * 128) =
+              make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
-      // keys 64h..64h+63 form atom column h; row t holds 8 chunks of 16 bytes
-      uint8_t* prow = p_s + (c >> 3) * (128 * 128) + t * 128;
-      *reinterpret_cast<uint4*>(prow + (((c & 7) ^ (t & 7)) << 4)) =
-          make_uint4(pk[0], pk[1], pk[2], pk[3]);
-    }
-    // O (from earlier tiles) is rescaled in TMEM when the running max grew;
-    // the previous P V finished before this tile's S was committed.
-    if (j > 0 && __any_sync(0xffffffffu, alpha < 1.f)) {
+      // this warp only ever reads O columns [32w, 32w+32) of its lanes
+      if (j > 0 && __any_sync(0xffffffffu, alpha < 1.f)) {
 #pragma unroll
-      for (int c = 0; c < D / 16; ++c) {
-        float v[16];
-        tmem_ld16(o_tmem + lane_off + c * 16, v);
-        tmem_ld_wait();
+        for (int c = 0; c < 2; ++c) {
+          float v[16];
+          tmem_ld16(o_tmem + lane_off + kq + c * 16, v);
+          tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] *= alpha;
-        tmem_st16(o_tmem + lane_off + c * 16, v);
+          for (int i = 0; i < 16; ++i) v[i] *= alpha;
+          tmem_st16(o_tmem + lane_off + kq + c * 16, v);
+        }
+        tmem_st_wait();
       }
-      tmem_st_wait();
+      l_run = l_run * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));  // this quarter's share
+      m_run = m_new;
+    } else {
+      // ---- softmax of row t over the tile (log2 domain), one TMEM read
+      float s[kKeys];
+#pragma unroll
+      for (int c = 0; c < kKeys / 32; ++c) tmem_ld32(s_tmem + lane_off + c * 32, s + c * 32);
+      tmem_ld_wait();
+      // independent partial maxima and sums: one warp per scheduler has no
+      // other work to hide a serial dependency chain behind
+      float tm[4] = {-FLT_MAX, -FLT_MAX, -FLT_MAX, -FLT_MAX};
+#pragma unroll
+      for (int i = 0; i < kKeys; ++i)
+        if (i < nvalid) tm[i & 3] = fmaxf(tm[i & 3], s[i]);
+      const float tmax = fmaxf(fmaxf(tm[0], tm[1]), fmaxf(tm[2], tm[3]));
+      const float m_new = fmaxf(m_run, tmax * p.scale_log2);
+      const float alpha = fast_exp2(m_run - m_new);
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int c = 0; c < kKeys / 8; ++c) {  // 8 keys = one 16-byte chunk of P
+        uint32_t pk[4];
+#pragma unroll
+        for (int i = 0; i < 8; i += 2) {
+          const int k0 = c * 8 + i;
+          const float p0 = k0 < nvalid ? fast_exp2(s[k0] * p.scale_log2 - m_new) : 0.f;
+          const float p1 = k0 + 1 < nvalid ? fast_exp2(s[k0 + 1] * p.scale_log2 - m_new) : 0.f;
+          const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+          ls[c & 3] += __low2float(h2) + __high2float(h2);
+          pk[i >> 1] = *reinterpret_cast<const uint32_t*>(&h2);
+        }
+        // keys 64h..64h+63 form atom column h; row t holds 8 chunks of 16 bytes
+        uint8_t* prow = p_s + (c >> 3) * (128 * 128) + t * 128;
+        *reinterpret_cast<uint4*>(prow + (((c & 7) ^ (t & 7)) << 4)) =
+            make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+      // O (from earlier tiles) is rescaled in TMEM when the running max grew;
+      // the previous P V finished before this tile's S was committed.
+      if (j > 0 && __any_sync(0xffffffffu, alpha < 1.f)) {
+#pragma unroll
+        for (int c = 0; c < D / 16; ++c) {
+          float v[16];
+          tmem_ld16(o_tmem + lane_off + c * 16, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] *= alpha;
+          tmem_st16(o_tmem + lane_off + c * 16, v);
+        }
+        tmem_st_wait();
+      }
+      l_run = l_run * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
+      m_run = m_new;
     }
-    l_run = l_run * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
-    m_run = m_new;
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -354,8 +429,18 @@ __global__ void __launch_bounds__(128, 1)
   tc_fence_after();
 
   // ---- output
+  // A small group's thread (w, i) holds row i and output columns [32w, 32w+32);
+  // otherwise thread t holds row t of the tile and every column.
+  constexpr int kCols = SG ? 32 : D;
+  const int lrow = SG ? (t & 31) : t;  // row within the tile
+  const int c0 = SG ? warp * 32 : 0;
+  if constexpr (SG) {  // the row's softmax sum is split over its four quarter threads
+    x_s[128 + t] = l_run;
+    __syncthreads();
+    l_run = (x_s[128 + lrow] + x_s[160 + lrow]) + (x_s[192 + lrow] + x_s[224 + lrow]);
+  }
   const int g = p.Hq / p.Hkv;
-  const int r = rt * 128 + t;
+  const int r = rt * (SG ? 32 : 128) + lrow;
   const bool row_ok = r < p.group_rows;
   const int hl = r / p.n_rows;
   const int ii = r - hl * p.n_rows;
@@ -381,11 +466,11 @@ __global__ void __launch_bounds__(128, 1)
     if (ok) {
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
 #pragma unroll
-      for (int c = 0; c < D / 16; ++c) {
+      for (int c = 0; c < kCols / 16; ++c) {
         float v[16];
-        tmem_ld16(o_tmem + lane_off + c * 16, v);
+        tmem_ld16(o_tmem + lane_off + c0 + c * 16, v);
         tmem_ld_wait();
-        if (row_ok && my_tiles > 0) store16(c * 16, v, inv);
+        if (row_ok && my_tiles > 0) store16(c0 + c * 16, v, inv);
       }
     }
   } else {
@@ -395,18 +480,19 @@ __global__ void __launch_bounds__(128, 1)
     const uint32_t rank = (uint32_t)chunk;
     const bool have = ok && my_tiles > 0 && l_run > 0.f;
     const float2 mine = have ? make_float2(m_run, l_run) : make_float2(-FLT_MAX, 0.f);
-    const uint32_t ml_addr = smem_u32(&ml_s[rank * 128 + t]);
-    for (int q = 0; q < nch; ++q)
-      st_cluster_v2(map_to_rank(ml_addr, (uint32_t)q), mine.x, mine.y);
+    const uint32_t ml_addr = smem_u32(&ml_s[rank * 128 + lrow]);
+    if (!SG || warp == 0)
+      for (int q = 0; q < nch; ++q)
+        st_cluster_v2(map_to_rank(ml_addr, (uint32_t)q), mine.x, mine.y);
     cluster_sync();  // (max, sum) everywhere; every chunk's P V is done
     float mx = -FLT_MAX;
     for (int c = 0; c < nch; ++c) {
-      const float2 e = ml_s[c * 128 + t];
+      const float2 e = ml_s[c * 128 + lrow];
       if (e.y > 0.f) mx = fmaxf(mx, e.x);
     }
     float lt = 0.f;
     for (int c = 0; c < nch; ++c) {
-      const float2 e = ml_s[c * 128 + t];
+      const float2 e = ml_s[c * 128 + lrow];
       if (e.y > 0.f) lt += fast_exp2(e.x - mx) * e.y;
     }
     const float wmine = have && lt > 0.f ? fast_exp2(mine.x - mx) / lt : 0.f;
@@ -415,21 +501,22 @@ __global__ void __launch_bounds__(128, 1)
     const int gpo = (C::kGroups + nch - 1) / nch;
     float4* red = reinterpret_cast<float4*>(k_s);
     const uint32_t red_addr = smem_u32(red);
-    // the whole O row is read from TMEM with one wait, then sent out
-    float o[D];
+    // this thread's columns of the O row are read from TMEM with one wait, then sent out
+    float o[kCols];
 #pragma unroll
-    for (int c = 0; c < D / 32; ++c) tmem_ld32(o_tmem + lane_off + c * 32, o + c * 32);
+    for (int c = 0; c < kCols / 32; ++c) tmem_ld32(o_tmem + lane_off + c0 + c * 32, o + c * 32);
     tmem_ld_wait();
     if (row_ok) {
 #pragma unroll
-      for (int gi = 0; gi < C::kGroups; ++gi) {
+      for (int gg = 0; gg < kCols / 16; ++gg) {
+        const int gi = c0 / 16 + gg;
         const uint32_t owner = (uint32_t)(gi % nch);
         const int lg = gi / nch;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const int slot = ((int)(rank * gpo + lg) * 4 + q) * 128 + t;
+          const int slot = ((int)(rank * gpo + lg) * 4 + q) * 128 + lrow;
           const uint32_t dst = map_to_rank(red_addr + slot * 16, owner);
-          const float* v = o + gi * 16 + 4 * q;
+          const float* v = o + gg * 16 + 4 * q;
           if (wmine != 0.f)
             st_cluster_v4(dst, v[0] * wmine, v[1] * wmine, v[2] * wmine, v[3] * wmine);
           else
@@ -439,7 +526,8 @@ __global__ void __launch_bounds__(128, 1)
     }
     cluster_sync();  // every contribution has landed
     if (ok && row_ok) {
-      for (int lg = 0; lg < gpo; ++lg) {
+      // a small group's four warps share the owned groups of the row
+      for (int lg = SG ? warp : 0; lg < gpo; lg += SG ? 4 : 1) {
         const int gi = lg * nch + (int)rank;
         if (gi >= C::kGroups) break;
         float v[16];
@@ -448,7 +536,7 @@ __global__ void __launch_bounds__(128, 1)
         for (int c = 0; c < nch; ++c) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const float4 x = red[((c * gpo + lg) * 4 + q) * 128 + t];
+            const float4 x = red[((c * gpo + lg) * 4 + q) * 128 + lrow];
             v[4 * q] += x.x;
             v[4 * q + 1] += x.y;
             v[4 * q + 2] += x.z;
@@ -470,12 +558,12 @@ __global__ void __launch_bounds__(128, 1)
   }
 }
 
-template <int D, int ST>
+template <int D, int ST, bool SG>
 static cudaError_t launch_attn_t(const CUtensorMap& qmap, const CUtensorMap& kmap,
                                  const CUtensorMap& vmap, const AttnParams& p, bool pdl,
                                  cudaStream_t s) {
   using C_ = AttnCfg<D, ST>;
-  auto kern = attn_kernel<D, ST>;
+  auto kern = attn_kernel<D, ST, SG>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.batch * p.Hkv * p.row_tiles * p.chunks);
   cfg.blockDim = dim3(128);
@@ -505,11 +593,13 @@ static cudaError_t launch_attn_t(const CUtensorMap& qmap, const CUtensorMap& kma
 
 cudaError_t attn_prepare() {
   cudaError_t e = cudaSuccess;
-#define DLLM_SET(D, ST)                                                                   \
-  if (e == cudaSuccess)                                                                  \
-    e = cudaFuncSetAttribute(attn_kernel<D, ST>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+#define DLLM_SET(D, ST, SG)                                                   \
+  if (e == cudaSuccess)                                                      \
+    e = cudaFuncSetAttribute(attn_kernel<D, ST, SG>,                         \
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,    \
                              (int)AttnCfg<D, ST>::kSmem);
-  DLLM_SET(128, 1) DLLM_SET(128, 2) DLLM_SET(32, 1) DLLM_SET(32, 2)
+  DLLM_SET(128, 1, false) DLLM_SET(128, 2, false) DLLM_SET(32, 1, false) DLLM_SET(32, 2, false)
+  DLLM_SET(128, 1, true) DLLM_SET(128, 2, true)
 #undef DLLM_SET
   return e;
 }
@@ -519,16 +609,22 @@ size_t attn_smem_bytes(int head_dim) {
 }
 
 // One key tile per CTA keeps a single stage; longer chunks double-buffer.
+// A small group's Q map has a 32-row box (it is loaded four times).
 cudaError_t launch_attn(int head_dim, const CUtensorMap& qmap, const CUtensorMap& kmap,
                         const CUtensorMap& vmap, const AttnParams& p, bool pdl,
                         cudaStream_t s) {
   const bool one = p.tiles_per_chunk <= 1;
+  if (p.small_group) {
+    if (head_dim != 128 || p.row_tiles * 32 < p.group_rows) return cudaErrorInvalidValue;
+    return one ? launch_attn_t<128, 1, true>(qmap, kmap, vmap, p, pdl, s)
+               : launch_attn_t<128, 2, true>(qmap, kmap, vmap, p, pdl, s);
+  }
   if (head_dim == 128)
-    return one ? launch_attn_t<128, 1>(qmap, kmap, vmap, p, pdl, s)
-               : launch_attn_t<128, 2>(qmap, kmap, vmap, p, pdl, s);
+    return one ? launch_attn_t<128, 1, false>(qmap, kmap, vmap, p, pdl, s)
+               : launch_attn_t<128, 2, false>(qmap, kmap, vmap, p, pdl, s);
   if (head_dim == 32)
-    return one ? launch_attn_t<32, 1>(qmap, kmap, vmap, p, pdl, s)
-               : launch_attn_t<32, 2>(qmap, kmap, vmap, p, pdl, s);
+    return one ? launch_attn_t<32, 1, false>(qmap, kmap, vmap, p, pdl, s)
+               : launch_attn_t<32, 2, false>(qmap, kmap, vmap, p, pdl, s);
   return cudaErrorInvalidValue;
 }
 

@@ -68,7 +68,8 @@ struct AttnParams {
   int batch, Hq, Hkv, D, S, layer;
   int n_rows;       // query rows per sequence and head
   int group_rows;   // (Hq/Hkv) * n_rows
-  int row_tiles;    // ceil(group_rows / 128)
+  int row_tiles;    // ceil(group_rows / 128), or ceil(group_rows / 32) with small_group
+  int small_group;  // 1: row tiles of 32 rows, loaded four times (Q map box of 32 rows)
   int chunks;       // key chunks per (sequence, kv head, row tile) = cluster size
   int tiles_per_chunk;
   const int* segs;  // [b][2][2] (start, len), or null: derived from the fields below

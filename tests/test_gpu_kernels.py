@@ -282,11 +282,21 @@ ATTN_CASES = [  # (Hq, Hkv, D, batch, n_rows, S, segs per sequence, layer)
     (8, 8, 128, 3, 32, 1280, [[(300, 980), (0, 0)], [(0, 1280), (0, 0)], [(512, 768), (0, 0)]], 1),
     (4, 2, 128, 1, 700, 700, [[(0, 700), (0, 0)]], 0),
     (32, 32, 128, 1, 512, 512, [[(0, 512), (0, 0)]], 1),   # prefill shape
-    (28, 4, 128, 1, 32, 640, [[(0, 544), (639, 1)]], 0),   # 6 key chunks
-    (28, 4, 128, 1, 32, 1024, [[(5, 539), (0, 0)]], 1),    # 5 chunks of 2 tiles
+    (28, 4, 128, 1, 32, 640, [[(0, 544), (639, 1)]], 0),   # 32-row tiles: 7 per kv head, 3 chunks
+    (28, 4, 128, 1, 32, 1024, [[(5, 539), (0, 0)]], 1),    # 32-row tiles, 3 chunks of 3 tiles
     (8, 8, 32, 1, 16, 640, [[(0, 600), (0, 0)]], 0),       # head_dim 32, 6 chunks
-    (28, 4, 128, 1, 32, 896, [[(0, 880), (895, 1)]], 0),   # 8 key chunks
-    (28, 4, 128, 1, 32, 768, [[(3, 700), (0, 0)]], 1),     # 7 tiles: 8 chunks, the last empty
+    (28, 4, 128, 1, 32, 896, [[(0, 880), (895, 1)]], 0),   # 32-row tiles, 4 chunks
+    (28, 4, 128, 1, 32, 768, [[(3, 700), (0, 0)]], 1),     # 32-row tiles, 4 chunks
+    # 128-row tiles (groups of 448 rows)
+    (28, 4, 128, 1, 64, 640, [[(0, 544), (639, 1)]], 0),   # 6 key chunks
+    (28, 4, 128, 1, 64, 896, [[(0, 880), (895, 1)]], 0),   # 8 key chunks
+    (28, 4, 128, 1, 64, 768, [[(3, 700), (0, 0)]], 1),     # 7 tiles: 8 chunks, the last empty
+    # one 32-row tile per kv head
+    (4, 4, 128, 1, 8, 768, [[(3, 700), (0, 0)]], 0),       # 7 tiles: 8 chunks, the last empty
+    (4, 4, 128, 1, 8, 640, [[(0, 544), (639, 1)]], 1),     # 6 key chunks
+    (4, 4, 128, 1, 1, 96, [[(0, 96), (0, 0)]], 0),         # one row, two tiles in one CTA
+    (1, 1, 128, 1, 16, 64, [[(0, 64), (0, 0)]], 1),        # one tile, no chunks
+    (16, 2, 128, 2, 4, 200, [[(0, 150), (199, 1)], [(20, 100), (0, 0)]], 0),  # GQA, 32 rows
 ]
 
 
