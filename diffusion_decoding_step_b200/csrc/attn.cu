@@ -125,7 +125,7 @@ __device__ __forceinline__ void tile_of(const int* sg, int t, int& start, int& n
 }
 
 template <int D, int ST, bool SG>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(SG ? 128 : 256, 1)
     attn_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                 const __grid_constant__ CUtensorMap vmap, const AttnParams p) {
   using C = AttnCfg<D, ST>;
@@ -232,7 +232,11 @@ __global__ void __launch_bounds__(128, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t s_tmem = tmem;
   const uint32_t o_tmem = tmem + 128;
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;  // a warp reads lanes 32(w%4)..
+  // 128-row tiles run 8 warps: thread t holds row t % 128 and key half
+  // t / 128 in the softmax, and the same half of the output columns.
+  const int half = SG ? 0 : t >> 7;
+  const int trow = t & 127;
 
   constexpr uint32_t kIdescS = idesc_bf16(128, kKeys, 0, 0);
   constexpr uint32_t kIdescO = idesc_bf16(128, D, 0, 1);
@@ -344,53 +348,60 @@ __global__ void __launch_bounds__(128, 1)
       l_run = l_run * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));  // this quarter's share
       m_run = m_new;
     } else {
-      // ---- softmax of row t over the tile (log2 domain), one TMEM read
-      float s[kKeys];
+      // ---- softmax of row trow over key half `half` of the tile (log2
+      // domain); the row max crosses the two halves through shared memory
+      constexpr int kH = kKeys / 2;
+      const int kb = half * kH;
+      float s[kH];
 #pragma unroll
-      for (int c = 0; c < kKeys / 32; ++c) tmem_ld32(s_tmem + lane_off + c * 32, s + c * 32);
+      for (int c = 0; c < kH / 32; ++c) tmem_ld32(s_tmem + lane_off + kb + c * 32, s + c * 32);
       tmem_ld_wait();
-      // independent partial maxima and sums: one warp per scheduler has no
-      // other work to hide a serial dependency chain behind
+      // independent partial maxima and sums: two warps per scheduler still
+      // leave little other work to hide a serial dependency chain behind
       float tm[4] = {-FLT_MAX, -FLT_MAX, -FLT_MAX, -FLT_MAX};
 #pragma unroll
-      for (int i = 0; i < kKeys; ++i)
-        if (i < nvalid) tm[i & 3] = fmaxf(tm[i & 3], s[i]);
-      const float tmax = fmaxf(fmaxf(tm[0], tm[1]), fmaxf(tm[2], tm[3]));
+      for (int i = 0; i < kH; ++i)
+        if (kb + i < nvalid) tm[i & 3] = fmaxf(tm[i & 3], s[i]);
+      x_s[t] = fmaxf(fmaxf(tm[0], tm[1]), fmaxf(tm[2], tm[3]));
+      __syncthreads();
+      const float tmax = fmaxf(x_s[trow], x_s[128 + trow]);
       const float m_new = fmaxf(m_run, tmax * p.scale_log2);
       const float alpha = fast_exp2(m_run - m_new);
       float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < kKeys / 8; ++c) {  // 8 keys = one 16-byte chunk of P
+      for (int c = 0; c < kH / 8; ++c) {  // 8 keys = one 16-byte chunk of P
         uint32_t pk[4];
 #pragma unroll
         for (int i = 0; i < 8; i += 2) {
           const int k0 = c * 8 + i;
-          const float p0 = k0 < nvalid ? fast_exp2(s[k0] * p.scale_log2 - m_new) : 0.f;
-          const float p1 = k0 + 1 < nvalid ? fast_exp2(s[k0 + 1] * p.scale_log2 - m_new) : 0.f;
+          const float p0 = kb + k0 < nvalid ? fast_exp2(s[k0] * p.scale_log2 - m_new) : 0.f;
+          const float p1 =
+              kb + k0 + 1 < nvalid ? fast_exp2(s[k0 + 1] * p.scale_log2 - m_new) : 0.f;
           const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
           ls[c & 3] += __low2float(h2) + __high2float(h2);
           pk[i >> 1] = *reinterpret_cast<const uint32_t*>(&h2);
         }
-        // keys 64h..64h+63 form atom column h; row t holds 8 chunks of 16 bytes
-        uint8_t* prow = p_s + (c >> 3) * (128 * 128) + t * 128;
-        *reinterpret_cast<uint4*>(prow + (((c & 7) ^ (t & 7)) << 4)) =
+        // keys 64h..64h+63 form atom column h; row trow holds 8 chunks of 16 bytes
+        uint8_t* prow = p_s + half * (128 * 128) + trow * 128;
+        *reinterpret_cast<uint4*>(prow + ((c ^ (trow & 7)) << 4)) =
             make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
       // O (from earlier tiles) is rescaled in TMEM when the running max grew;
-      // the previous P V finished before this tile's S was committed.
+      // the previous P V finished before this tile's S was committed.  Each
+      // thread rescales the half of the row's columns that it later reads.
       if (j > 0 && __any_sync(0xffffffffu, alpha < 1.f)) {
 #pragma unroll
-        for (int c = 0; c < D / 16; ++c) {
+        for (int c = 0; c < D / 32; ++c) {
           float v[16];
-          tmem_ld16(o_tmem + lane_off + c * 16, v);
+          tmem_ld16(o_tmem + lane_off + half * (D / 2) + c * 16, v);
           tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < 16; ++i) v[i] *= alpha;
-          tmem_st16(o_tmem + lane_off + c * 16, v);
+          tmem_st16(o_tmem + lane_off + half * (D / 2) + c * 16, v);
         }
         tmem_st_wait();
       }
-      l_run = l_run * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
+      l_run = l_run * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));  // this half's share
       m_run = m_new;
     }
     fence_proxy_async_smem();
@@ -431,13 +442,19 @@ __global__ void __launch_bounds__(128, 1)
   // ---- output
   // A small group's thread (w, i) holds row i and output columns [32w, 32w+32);
   // otherwise thread t holds row t of the tile and every column.
-  constexpr int kCols = SG ? 32 : D;
-  const int lrow = SG ? (t & 31) : t;  // row within the tile
-  const int c0 = SG ? warp * 32 : 0;
-  if constexpr (SG) {  // the row's softmax sum is split over its four quarter threads
+  constexpr int kCols = SG ? 32 : D / 2;
+  const int lrow = SG ? (t & 31) : trow;  // row within the tile
+  const int c0 = SG ? warp * 32 : half * (D / 2);
+  // the row's softmax sum is split over its four quarter (or two half) threads
+  if constexpr (SG) {
     x_s[128 + t] = l_run;
     __syncthreads();
     l_run = (x_s[128 + lrow] + x_s[160 + lrow]) + (x_s[192 + lrow] + x_s[224 + lrow]);
+  } else {
+    __syncthreads();  // the last tile's maxima have been read
+    x_s[t] = l_run;
+    __syncthreads();
+    l_run = x_s[trow] + x_s[128 + trow];
   }
   const int g = p.Hq / p.Hkv;
   const int r = rt * (SG ? 32 : 128) + lrow;
@@ -481,7 +498,7 @@ __global__ void __launch_bounds__(128, 1)
     const bool have = ok && my_tiles > 0 && l_run > 0.f;
     const float2 mine = have ? make_float2(m_run, l_run) : make_float2(-FLT_MAX, 0.f);
     const uint32_t ml_addr = smem_u32(&ml_s[rank * 128 + lrow]);
-    if (!SG || warp == 0)
+    if (SG ? warp == 0 : half == 0)
       for (int q = 0; q < nch; ++q)
         st_cluster_v2(map_to_rank(ml_addr, (uint32_t)q), mine.x, mine.y);
     cluster_sync();  // (max, sum) everywhere; every chunk's P V is done
@@ -503,8 +520,12 @@ __global__ void __launch_bounds__(128, 1)
     const uint32_t red_addr = smem_u32(red);
     // this thread's columns of the O row are read from TMEM with one wait, then sent out
     float o[kCols];
+    if constexpr (kCols % 32 == 0) {
 #pragma unroll
-    for (int c = 0; c < kCols / 32; ++c) tmem_ld32(o_tmem + lane_off + c0 + c * 32, o + c * 32);
+      for (int c = 0; c < kCols / 32; ++c) tmem_ld32(o_tmem + lane_off + c0 + c * 32, o + c * 32);
+    } else {
+      tmem_ld16(o_tmem + lane_off + c0, *reinterpret_cast<float(*)[16]>(o));
+    }
     tmem_ld_wait();
     if (row_ok) {
 #pragma unroll
@@ -526,8 +547,8 @@ __global__ void __launch_bounds__(128, 1)
     }
     cluster_sync();  // every contribution has landed
     if (ok && row_ok) {
-      // a small group's four warps share the owned groups of the row
-      for (int lg = SG ? warp : 0; lg < gpo; lg += SG ? 4 : 1) {
+      // the row's four quarter (two half) threads share its owned groups
+      for (int lg = SG ? warp : half; lg < gpo; lg += SG ? 4 : 2) {
         const int gi = lg * nch + (int)rank;
         if (gi >= C::kGroups) break;
         float v[16];
@@ -566,7 +587,7 @@ static cudaError_t launch_attn_t(const CUtensorMap& qmap, const CUtensorMap& kma
   auto kern = attn_kernel<D, ST, SG>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.batch * p.Hkv * p.row_tiles * p.chunks);
-  cfg.blockDim = dim3(128);
+  cfg.blockDim = dim3(SG ? 128 : 256);
   cfg.dynamicSmemBytes = AttnCfg<D, ST>::kSmem;
   cfg.stream = s;
   cudaLaunchAttribute attr[2];

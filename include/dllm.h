@@ -373,7 +373,7 @@ void dllm_graph_cache_clear(void);
  * or the LM head after the last layer of a step); layer l's O-projection asks
  * for the following oproj_next_bytes.  Only the cache is affected, never a
  * result.  Process-wide; clears the graph cache.  Negative sizes are
- * rejected (DLLM_ERR_INVALID).  Defaults: 0, 0, off. */
+ * rejected (DLLM_ERR_INVALID).  Defaults: 8 MiB, 0, off. */
 dllm_status dllm_set_l2_prefetch(int64_t attn_next_bytes, int64_t oproj_next_bytes,
                                  int32_t attn_prefetch_wo);
 
