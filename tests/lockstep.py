@@ -201,10 +201,17 @@ def lockstep_incremental(dec, case, max_blocks=None, log=None) -> Report:
     end = cfg.prompt_len if cfg.mode == O.MODE_PREFIX else cfg.seq_len
     ref = O.new_state(cfg, st.tokens, st.masked, st.starts)
     O.prefill(cfg, W, ref)
+    # Both prefills run free through every layer: unlike a step or a refresh,
+    # the keys the attention reads are each side's own, so the two sides'
+    # bf16 roundings decorrelate with depth.  Layer 0 (same inputs up to
+    # rounding) keeps 5e-3; all layers together get 1e-2, about 1.3 bf16 ulps
+    # of relative spacing (2^-7).  On the 32-layer shape the per-layer rel-L2
+    # rises from 1e-4 at layer 0 to 5.7e-3 at layer 31.
     for bi in range(cfg.batch):
         a = int(st.starts[bi])
         for got, want in ((st.kcache, ref.kcache), (st.vcache, ref.vcache)):
-            assert rel_l2(got[:, bi, :, a:end], want[:, bi, :, a:end]) <= 5e-3
+            assert rel_l2(got[0, bi, :, a:end], want[0, bi, :, a:end]) <= 5e-3
+            assert rel_l2(got[:, bi, :, a:end], want[:, bi, :, a:end]) <= 1e-2
     del ref
     blocks = list(range(cfg.prompt_len, cfg.seq_len, B))[:max_blocks]
     t0 = time.time()

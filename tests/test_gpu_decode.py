@@ -270,7 +270,8 @@ def test_full_size_generation_lockstep(name, blocks):
     oracle in the launch configuration bench.py times: confidences within
     2e-3, tokens and commits bit-exact outside flagged rows, the block's
     keys/values after every step and refresh within rel-L2 5e-3, prefill of
-    all layers within rel-L2 5e-3."""
+    layer 0 within rel-L2 5e-3 and of all layers within 1e-2 (both sides run
+    the prefill free through every layer)."""
     from tests.lockstep import lockstep_incremental
     w = wl.WORKLOADS[name]
     ensure_lib()
