@@ -90,11 +90,14 @@ constexpr int gemm_min_blocks() {
   return (EPI == EPI_OPROJ && NT <= 32) ? 2 : NT <= 32 ? 3 : NT <= 64 ? 2 : 1;
 }
 
-template <int NT, int EPI>
+// CW: width of the split-K chunks dealt to a cluster's ranks (16 columns,
+// or 8 so that all ranks of a 3- or 4-way split of a 32-column tile own one).
+template <int NT, int EPI, int CW>
 __global__ void __launch_bounds__(192, gemm_min_blocks<NT, EPI>())
     gemm_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap xmap,
                 const GemmParams p) {
   using C = GemmCfg<NT, EPI>;
+  static_assert(CW == 16 || (CW == 8 && NT == 32 && EPI != EPI_LMHEAD), "chunk width");
   constexpr int ST = C::kStages;
   constexpr int kEpi = EPI == EPI_QKV_DEEP ? EPI_QKV : EPI;  // epilogue kind
   constexpr uint32_t kIdesc = idesc_bf16(128, NT, 0, 0);
@@ -125,10 +128,11 @@ __global__ void __launch_bounds__(192, gemm_min_blocks<NT, EPI>())
   // Split K is reduced inside a thread-block cluster for decode tiles.
   constexpr bool kClusterSplit = NT <= 64;
   float part[kClusterSplit ? NT : 1];
-  // 16-column chunks of a split tile are dealt round robin to the cluster's
+  // CW-column chunks of a split tile are dealt round robin to the cluster's
   // ranks; at most kOwnMax per rank (splits >= 2)
-  constexpr int kOwnMax = kClusterSplit ? (NT / 16 + 1) / 2 : 1;
-  float xpre[kOwnMax][16];
+  constexpr int kNChunk = NT / CW;
+  constexpr int kOwnMax = kClusterSplit ? (kNChunk + 1) / 2 : 1;
+  float xpre[kOwnMax][CW];
   if (threadIdx.x == 0) {
     for (int s = 0; s < ST; ++s) {
       mbar_init(&full[s], 1);
@@ -160,9 +164,9 @@ __global__ void __launch_bounds__(192, gemm_min_blocks<NT, EPI>())
       // Owners of split-K chunks expect the other ranks' partials; the
       // cluster barrier (waited for in the tail) publishes the armed barriers.
       const int rank = (int)cluster_ctarank();
-      const int owned = (NT / 16 - rank + p.splits - 1) / p.splits;
+      const int owned = (kNChunk - rank + p.splits - 1) / p.splits;
       if (threadIdx.x == 0 && owned > 0)
-        mbar_arrive_expect_tx(red_bar, (uint32_t)((p.splits - 1) * owned * 128 * 64));
+        mbar_arrive_expect_tx(red_bar, (uint32_t)((p.splits - 1) * owned * 128 * CW * 4));
       cluster_arrive_relaxed();
     }
   }
@@ -293,7 +297,7 @@ __global__ void __launch_bounds__(192, gemm_min_blocks<NT, EPI>())
 #pragma unroll
           for (int lq = 0; lq < kOwnMax; ++lq) {
             const int q = lq * p.splits + rank;
-            if (q < NT / 16) oproj_load_x<NT>(p, m, n, q * 16, wl, xpre[lq]);
+            if (q < kNChunk) oproj_load_x<NT, false, CW>(p, m, n, q * CW, wl, xpre[lq]);
           }
         }
       }
@@ -324,7 +328,7 @@ __global__ void __launch_bounds__(192, gemm_min_blocks<NT, EPI>())
         if constexpr (kEpi == EPI_OPROJ) oproj_load_x<NT>(p, m, n, c0, wl, xo);
         tmem_ld16(tmem + ((uint32_t)lane_base << 16) + acc * NT + c0, v);
         tmem_ld_wait();
-        epi_chunk<NT, kEpi>(p, m, n, c0, wl, et, v, xo, stage, run);
+        epi_chunk<NT, kEpi, 16>(p, m, n, c0, wl, et, v, xo, stage, run);
       }
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
@@ -346,7 +350,7 @@ __global__ void __launch_bounds__(192, gemm_min_blocks<NT, EPI>())
   if constexpr (kClusterSplit) {
     if (p.splits > 1) {
       // The splits of a tile form one cluster (one unit per CTA).  The tile's
-      // 16-column chunks are dealt round robin to the ranks; every rank sends
+      // CW-column chunks are dealt round robin to the ranks; every rank sends
       // its partial of each chunk it does not own to the owner's receive
       // buffer with a bulk copy (the bytes complete on the owner's red_bar), and
       // each owner adds the partials of its chunks in rank order and runs
@@ -362,21 +366,22 @@ __global__ void __launch_bounds__(192, gemm_min_blocks<NT, EPI>())
       const int et = threadIdx.x - 64;
       const int wl = 32 * (warp & 3) + (threadIdx.x & 31);
       const int sp = p.splits;
-      const int own = (NT / 16 + sp - 1) / sp;  // chunk slots per owner
-      const int sw = (wl >> 1) & 3;              // float4 j of a lane sits at j ^ sw
+      const int own = (kNChunk + sp - 1) / sp;  // chunk slots per owner
+      // float4 j of a lane's chunk row sits at j ^ sw (bank spread of the staging stores)
+      const int sw = CW == 16 ? (wl >> 1) & 3 : (wl >> 2) & 1;
       if (epi) {
         // Each chunk this rank does not own is staged in the (idle) ring in
         // the owner's layout, then sent with one bulk copy.
         float* stg = reinterpret_cast<float*>(w_st + (p.recv_in_ring ? C::kRecvBytes : 0));
         int k = 0;
 #pragma unroll
-        for (int q = 0; q < NT / 16; ++q) {
+        for (int q = 0; q < kNChunk; ++q) {
           if (q % sp == rank) continue;
-          float4* row = reinterpret_cast<float4*>(stg + ((size_t)k * 128 + wl) * 16);
+          float4* row = reinterpret_cast<float4*>(stg + ((size_t)k * 128 + wl) * CW);
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            row[j ^ sw] = make_float4(part[q * 16 + 4 * j], part[q * 16 + 4 * j + 1],
-                                      part[q * 16 + 4 * j + 2], part[q * 16 + 4 * j + 3]);
+          for (int j = 0; j < CW / 4; ++j)
+            row[j ^ sw] = make_float4(part[q * CW + 4 * j], part[q * CW + 4 * j + 1],
+                                      part[q * CW + 4 * j + 2], part[q * CW + 4 * j + 3]);
           ++k;
         }
         fence_proxy_async_smem();
@@ -384,13 +389,13 @@ __global__ void __launch_bounds__(192, gemm_min_blocks<NT, EPI>())
         if (et == 0) {
           k = 0;
 #pragma unroll
-          for (int q = 0; q < NT / 16; ++q) {
+          for (int q = 0; q < kNChunk; ++q) {
             const int owner = q % sp;
             if (owner == rank) continue;
             const int slot = rank < owner ? rank : rank - 1;
             const uint32_t dst = map_to_rank(
-                smem_u32(recv + (size_t)(slot * own + q / sp) * 128 * 16), (uint32_t)owner);
-            bulk_copy_to_cluster(dst, smem_u32(stg + (size_t)k * 128 * 16), 128 * 16 * 4,
+                smem_u32(recv + (size_t)(slot * own + q / sp) * 128 * CW), (uint32_t)owner);
+            bulk_copy_to_cluster(dst, smem_u32(stg + (size_t)k * 128 * CW), 128 * CW * 4,
                                  map_to_rank(smem_u32(red_bar), (uint32_t)owner));
             ++k;
           }
@@ -399,7 +404,7 @@ __global__ void __launch_bounds__(192, gemm_min_blocks<NT, EPI>())
       // The closing cluster barrier only keeps every CTA alive until the
       // partials sent to it have landed; the partials themselves are ordered
       // by red_bar, so the arrivals need no release.
-      if (epi && rank < NT / 16) {
+      if (epi && rank < kNChunk) {
         const bool got = mbar_wait_cluster(red_bar, 0, p.status);
         cluster_arrive_relaxed();
         if (got && !flags[0]) {
@@ -408,28 +413,28 @@ __global__ void __launch_bounds__(192, gemm_min_blocks<NT, EPI>())
 #pragma unroll
           for (int lq = 0; lq < kOwnMax; ++lq) {
             const int q = lq * sp + rank;
-            if (q >= NT / 16) break;
-            float mine[16];
+            if (q >= kNChunk) break;
+            float mine[CW];
 #pragma unroll
-            for (int qq = 0; qq < NT / 16; ++qq)
+            for (int qq = 0; qq < kNChunk; ++qq)
               if (qq == q) {
 #pragma unroll
-                for (int i = 0; i < 16; ++i) mine[i] = part[qq * 16 + i];
+                for (int i = 0; i < CW; ++i) mine[i] = part[qq * CW + i];
               }
-            float v[16];
+            float v[CW];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] = 0.f;
+            for (int i = 0; i < CW; ++i) v[i] = 0.f;
             for (int r = 0; r < sp; ++r) {
               if (r == rank) {
 #pragma unroll
-                for (int i = 0; i < 16; ++i) v[i] += mine[i];
+                for (int i = 0; i < CW; ++i) v[i] += mine[i];
                 continue;
               }
               const int slot = r < rank ? r : r - 1;
               const float4* src = reinterpret_cast<const float4*>(
-                  recv + ((size_t)(slot * own + lq) * 128 + wl) * 16);
+                  recv + ((size_t)(slot * own + lq) * 128 + wl) * CW);
 #pragma unroll
-              for (int j = 0; j < 4; ++j) {
+              for (int j = 0; j < CW / 4; ++j) {
                 const float4 x = src[j ^ sw];
                 v[4 * j] += x.x;
                 v[4 * j + 1] += x.y;
@@ -437,7 +442,7 @@ __global__ void __launch_bounds__(192, gemm_min_blocks<NT, EPI>())
                 v[4 * j + 3] += x.w;
               }
             }
-            epi_chunk<NT, kEpi>(p, m, n, q * 16, wl, et, v, xpre[lq], stage, run);
+            epi_chunk<NT, kEpi, CW>(p, m, n, q * CW, wl, et, v, xpre[lq], stage, run);
           }
         }
       } else {
@@ -453,10 +458,10 @@ __global__ void __launch_bounds__(192, gemm_min_blocks<NT, EPI>())
   }
 }
 
-template <int NT, int EPI>
+template <int NT, int EPI, int CW = 16>
 static cudaError_t launch_t(const CUtensorMap& wmap, const CUtensorMap& xmap, const GemmParams& p,
                             int grid, bool pdl, cudaStream_t s) {
-  auto kern = gemm_kernel<NT, EPI>;
+  auto kern = gemm_kernel<NT, EPI, CW>;
   const size_t smem = p.recv_in_ring ? GemmCfg<NT, EPI>::kSmemBase : GemmCfg<NT, EPI>::kSmem;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
@@ -491,14 +496,16 @@ static cudaError_t launch_t(const CUtensorMap& wmap, const CUtensorMap& xmap, co
 // that no attribute call happens while a launch sequence is being captured.
 cudaError_t gemm_prepare() {
   cudaError_t e = cudaSuccess;
-#define DLLM_SET(NT, EPI)                                                                      \
-  if (e == cudaSuccess)                                                                       \
-    e = cudaFuncSetAttribute(gemm_kernel<NT, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+#define DLLM_SET(NT, EPI, CW)                                             \
+  if (e == cudaSuccess)                                                  \
+    e = cudaFuncSetAttribute(gemm_kernel<NT, EPI, CW>,                   \
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, \
                              (int)GemmCfg<NT, EPI>::kSmem);
-  DLLM_SET(32, 0) DLLM_SET(32, 1) DLLM_SET(32, 2) DLLM_SET(32, 3)
-  DLLM_SET(64, 0) DLLM_SET(64, 1) DLLM_SET(64, 2) DLLM_SET(64, 3)
-  DLLM_SET(128, 0) DLLM_SET(128, 1) DLLM_SET(128, 2)
-  DLLM_SET(256, 0) DLLM_SET(256, 1) DLLM_SET(256, 2)
+  DLLM_SET(32, 0, 16) DLLM_SET(32, 1, 16) DLLM_SET(32, 2, 16) DLLM_SET(32, 3, 16)
+  DLLM_SET(32, 0, 8) DLLM_SET(32, 1, 8) DLLM_SET(32, 3, 8)
+  DLLM_SET(64, 0, 16) DLLM_SET(64, 1, 16) DLLM_SET(64, 2, 16) DLLM_SET(64, 3, 16)
+  DLLM_SET(128, 0, 16) DLLM_SET(128, 1, 16) DLLM_SET(128, 2, 16)
+  DLLM_SET(256, 0, 16) DLLM_SET(256, 1, 16) DLLM_SET(256, 2, 16)
 #undef DLLM_SET
   return e;
 }
@@ -507,6 +514,10 @@ cudaError_t gemm_prepare() {
 template <int EPI>
 static cudaError_t launch_e(int nt, const CUtensorMap& wmap, const CUtensorMap& xmap,
                             const GemmParams& p, int grid, bool pdl, cudaStream_t s) {
+  // 3- and 4-way splits of a 32-column tile deal 8-column chunks, so that
+  // every rank owns part of the reduction and the epilogue
+  if constexpr (EPI != EPI_LMHEAD)
+    if (nt == 32 && p.splits >= 3) return launch_t<32, EPI, 8>(wmap, xmap, p, grid, pdl, s);
   if constexpr (EPI == EPI_QKV_DEEP) {
     switch (nt) {
       case 32: return launch_t<32, EPI>(wmap, xmap, p, grid, pdl, s);

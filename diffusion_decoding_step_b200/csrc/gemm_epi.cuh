@@ -35,20 +35,24 @@ __device__ __forceinline__ LmStat lm_shfl_xor(const LmStat& a, int mask) {
   return r;
 }
 
-// Sum over the 128 lanes of each of the chunk's 16 columns staged as
-// stage[col][lane]: 8 threads per column, 16 lanes each, then a shuffle
-// tree.  Returns the column sum in the thread with (et & 7) == 0.  Each
-// thread starts its 16 lanes at a rotation that puts the warp's 32 threads
-// (4 columns x 8 subs) on 32 distinct banks at every step.
-__device__ __forceinline__ float column_sum16(const float* stage, int et) {
-  const int col = et >> 3, sub = et & 7;
-  const float* cv = stage + col * 128 + sub * 16;
-  const int rot = 4 * (col & 3) + (sub >> 1);
+// Sum over the 128 lanes of each of the chunk's CW columns staged as
+// stage[col][lane]: 128 / CW threads per column, CW lanes each, then a
+// shuffle tree.  Returns the column sum in the column's first thread.  Each
+// thread starts its CW lanes at a rotation that puts the warp's 32 threads on
+// 32 distinct banks at every step (16 columns: 4 columns x 8 subs; 8
+// columns: 2 columns x 16 subs).
+template <int CW>
+__device__ __forceinline__ float column_sum(const float* stage, int et) {
+  static_assert(CW == 16 || CW == 8, "chunk width");
+  constexpr int TPC = 128 / CW;  // threads per column
+  const int col = et / TPC, sub = et % TPC;
+  const float* cv = stage + col * 128 + sub * CW;
+  const int rot = CW == 16 ? 4 * (col & 3) + (sub >> 1) : (sub >> 2) + 4 * (col & 1);
   float s = 0.f;
 #pragma unroll
-  for (int q = 0; q < 16; ++q) s += cv[(q + rot) & 15];
+  for (int q = 0; q < CW; ++q) s += cv[(q + rot) & (CW - 1)];
 #pragma unroll
-  for (int mask = 1; mask < 8; mask <<= 1) s += __shfl_xor_sync(0xffffffffu, s, mask);
+  for (int mask = 1; mask < TPC; mask <<= 1) s += __shfl_xor_sync(0xffffffffu, s, mask);
   return s;
 }
 
@@ -106,27 +110,29 @@ __device__ __forceinline__ void epi_prepare(const GemmParams& p, int layer, int 
 // O-projection: the residual entries x[n*NT + c0 + i][m*128 + wl] a chunk
 // adds to.  The previous kernels are complete once the dependency wait has
 // returned, so these loads may run while the mainloop is still streaming.
-template <int NT, bool XCTA = false>
+template <int NT, bool XCTA = false, int CW = 16>
 __device__ __forceinline__ void oproj_load_x(const GemmParams& p, int m, int n, int c0, int wl,
-                                             float (&xo)[16]) {
+                                             float (&xo)[CW]) {
   const int wrow = m * 128 + wl;
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
+  for (int i = 0; i < CW; ++i) {
     const int xrow = n * NT + c0 + i;
     xo[i] = xrow < p.R ? ld_shared_f32<XCTA>(p.x + (size_t)xrow * p.d_model + wrow) : 0.f;
   }
 }
 
-// Epilogue of one 16-column chunk; v[i] = D^T[m*128 + wl][n*NT + c0 + i].
+// Epilogue of one CW-column chunk; v[i] = D^T[m*128 + wl][n*NT + c0 + i].
 // xo: the O-projection's residual entries of the chunk (oproj_load_x).
-template <int NT, int EPI>
+// The LM head takes 16-column chunks only.
+template <int NT, int EPI, int CW = 16>
 __device__ __forceinline__ void epi_chunk(const GemmParams& p, int m, int n, int c0, int wl,
-                                          int et, const float (&v)[16], const float (&xo)[16],
+                                          int et, const float (&v)[CW], const float (&xo)[CW],
                                           float* stage, LmStat* run) {
+  static_assert(EPI != EPI_LMHEAD || CW == 16, "LM-head chunks are 16 columns");
   if constexpr (EPI == EPI_OPROJ) {
     const int wrow = m * 128 + wl;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
+    for (int i = 0; i < CW; ++i) {
       const int xrow = n * NT + c0 + i;
       float sq = 0.f;
       if (xrow < p.R) {
@@ -140,9 +146,9 @@ __device__ __forceinline__ void epi_chunk(const GemmParams& p, int m, int n, int
     }
     if (p.sumsq_out != nullptr) {
       named_bar_sync(1, 128);
-      const float s = column_sum16(stage, et);
-      const int xrow = n * NT + c0 + (et >> 3);
-      if ((et & 7) == 0 && xrow < p.R) p.sumsq_out[(size_t)xrow * p.npart + m] = s;
+      const float s = column_sum<CW>(stage, et);
+      const int xrow = n * NT + c0 + et / (128 / CW);
+      if (et % (128 / CW) == 0 && xrow < p.R) p.sumsq_out[(size_t)xrow * p.npart + m] = s;
       named_bar_sync(1, 128);
     }
   } else if constexpr (EPI == EPI_QKV) {
@@ -157,22 +163,22 @@ __device__ __forceinline__ void epi_chunk(const GemmParams& p, int m, int n, int
     const bool is_q = head < p.Hq;
     const bool is_k = !is_q && head < p.Hq + p.Hkv;
     const bool has_rope = p.rope_tab != nullptr;  // uniform over the CTA
-    float val[16];
+    float val[CW];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) val[i] = v[i] * inv[c0 + i];
+    for (int i = 0; i < CW; ++i) val[i] = v[i] * inv[c0 + i];
     if (has_rope) {
       // rotate-half pairs live in lanes dd and dd +- D/2 of the same tile
 #pragma unroll
-      for (int i = 0; i < 16; ++i) stage[i * 128 + wl] = val[i];
+      for (int i = 0; i < CW; ++i) stage[i * 128 + wl] = val[i];
       named_bar_sync(1, 128);
       if (is_q || is_k) {
         const int partner = wl + (dd < half ? half : -half);
         const int j = dd < half ? dd : dd - half;
-        float2 cs[16];
+        float2 cs[CW];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) cs[i] = p.rope_tab[(size_t)rpos[c0 + i] * half + j];
+        for (int i = 0; i < CW; ++i) cs[i] = p.rope_tab[(size_t)rpos[c0 + i] * half + j];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
+        for (int i = 0; i < CW; ++i) {
           const float o = stage[i * 128 + partner];
           val[i] = dd < half ? (val[i] * cs[i].x - o * cs[i].y) : (val[i] * cs[i].x + o * cs[i].y);
         }
@@ -191,7 +197,7 @@ __device__ __forceinline__ void epi_chunk(const GemmParams& p, int m, int n, int
     }
     const int* roff = is_q ? qoff : koff;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
+    for (int i = 0; i < CW; ++i) {
       if (n * NT + c0 + i < p.R)
         dst[(size_t)roff[c0 + i] * D + hoff] = __float2bfloat16_rn(val[i]);
     }
