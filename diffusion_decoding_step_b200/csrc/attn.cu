@@ -143,9 +143,10 @@ __global__ void __launch_bounds__(SG ? 128 : 256, 1)
   uint64_t* bar_q = bars;
   uint64_t* bar_s = bars + 1;
   uint64_t* bar_o = bars + 2;
-  uint64_t* bar_kv = bars + 3;  // [ST]
-  uint64_t* dep_bar = bars + 3 + ST;  // thread 0 passes the dependency wait, the rest sleep
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4 + ST);
+  uint64_t* bar_k = bars + 3;       // [ST]
+  uint64_t* bar_v = bars + 3 + ST;  // [ST]
+  uint64_t* dep_bar = bars + 3 + 2 * ST;  // thread 0 passes the dependency wait, the rest sleep
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4 + 2 * ST);
   volatile int* flags = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
   const int t = threadIdx.x;
@@ -164,7 +165,10 @@ __global__ void __launch_bounds__(SG ? 128 : 256, 1)
     mbar_init(bar_q, 1);
     mbar_init(bar_s, 1);
     mbar_init(bar_o, 1);
-    for (int s = 0; s < ST; ++s) mbar_init(&bar_kv[s], 1);
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(&bar_k[s], 1);
+      mbar_init(&bar_v[s], 1);
+    }
     mbar_init(dep_bar, 1);
     flags[0] = 0;
     flags[1] = 0;
@@ -180,15 +184,41 @@ __global__ void __launch_bounds__(SG ? 128 : 256, 1)
   int sg[4] = {0, 0, 0, 0};
   if (p.segs == nullptr) seq_segments(p, b, sg);
 
-  auto issue_kv = [&](int j, int start) {  // key tile t0 + j into stage j % ST
+  // Key tile t0 + j into stage j % ST.  On 128-row tiles K and V complete
+  // on separate barriers: a K stage is refilled as soon as its S = Q K^T is
+  // done, its V stage once P V is done.  32-row tiles load both on bar_k and
+  // refill the stage once P V is done.
+  constexpr bool kSplitKV = !SG;
+  auto issue_k = [&](int j, int start) {
     const int st = j % ST;
-    mbar_arrive_expect_tx(&bar_kv[st], 2 * C::kKVBytes);
+    mbar_arrive_expect_tx(&bar_k[st], C::kKVBytes);
 #pragma unroll
-    for (int bx = 0; bx < C::kNBox; ++bx) {
-      tma_load_3d(k_s + st * C::kKVBytes + bx * C::kBoxBytes, &kmap, &bar_kv[st],
+    for (int bx = 0; bx < C::kNBox; ++bx)
+      tma_load_3d(k_s + st * C::kKVBytes + bx * C::kBoxBytes, &kmap, &bar_k[st],
                   bx * C::kBoxD, start, zc);
-      tma_load_3d(v_s + st * C::kKVBytes + bx * C::kBoxBytes, &vmap, &bar_kv[st],
+  };
+  auto issue_v = [&](int j, int start) {
+    const int st = j % ST;
+    mbar_arrive_expect_tx(&bar_v[st], C::kKVBytes);
+#pragma unroll
+    for (int bx = 0; bx < C::kNBox; ++bx)
+      tma_load_3d(v_s + st * C::kKVBytes + bx * C::kBoxBytes, &vmap, &bar_v[st],
                   bx * C::kBoxD, start, zc);
+  };
+  auto issue_kv = [&](int j, int start) {
+    if constexpr (kSplitKV) {
+      issue_k(j, start);
+      issue_v(j, start);
+    } else {
+      const int st = j % ST;
+      mbar_arrive_expect_tx(&bar_k[st], 2 * C::kKVBytes);
+#pragma unroll
+      for (int bx = 0; bx < C::kNBox; ++bx) {
+        tma_load_3d(k_s + st * C::kKVBytes + bx * C::kBoxBytes, &kmap, &bar_k[st],
+                    bx * C::kBoxD, start, zc);
+        tma_load_3d(v_s + st * C::kKVBytes + bx * C::kBoxBytes, &vmap, &bar_k[st],
+                    bx * C::kBoxD, start, zc);
+      }
     }
   };
   auto chunk_range = [&](int& first, int& n) {
@@ -262,31 +292,47 @@ __global__ void __launch_bounds__(SG ? 128 : 256, 1)
     }
   }
 
+  auto issue_s = [&](int j) {  // S = Q K^T of tile t0 + j (thread 0; Q and K are in)
+    tc_fence_after();
+    const uint32_t qa = smem_u32(q_s);
+    const uint32_t ka = smem_u32(k_s + (j % ST) * C::kKVBytes);
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint32_t off = (kk * 16 / C::kBoxD) * C::kBoxBytes + ((kk * 16) % C::kBoxD) * 2;
+      umma_bf16(s_tmem, smem_desc(qa + off, 16, 8 * C::kRowBytes, C::kSwCode),
+                smem_desc(ka + off, 16, 8 * C::kRowBytes, C::kSwCode), kIdescS,
+                kk > 0 ? 1u : 0u);
+    }
+    umma_commit(bar_s);
+  };
+  // 128-row tiles: once every thread holds tile j's S in registers (the
+  // row-max barrier), S of tile j+1 is issued at once if its K has landed,
+  // so that it runs during the rest of the softmax.  Its completion then no
+  // longer implies that P V of tile j is done: the P writes and O rescales of
+  // tile j+1 wait for that explicitly.  (On the 32-row shapes, one or two key
+  // tiles per CTA, this measured slower.)
+  bool s_next = false;  // thread 0: S of the next tile already issued
+  auto early_s = [&](int j) {
+    if (!SG && t == 0) {
+      s_next = j + 1 < my_tiles && mbar_try_wait(&bar_k[(j + 1) % ST], ((j + 1) / ST) & 1);
+      if (s_next) issue_s(j + 1);
+    }
+  };
+
   float m_run = -FLT_MAX, l_run = 0.f;
   bool ok = true;
   for (int j = 0; j < my_tiles; ++j) {
     const int st = j % ST;
     int kstart, nvalid;
     tile_of(sg, t0 + j, kstart, nvalid);
-    // ---- S = Q K^T
-    if (t == 0) {
+    // ---- S = Q K^T (unless issued early during the previous tile)
+    if (t == 0 && !s_next) {
       const bool good = (j > 0 || mbar_wait(bar_q, 0, p.status)) &&
-                        mbar_wait(&bar_kv[st], (j / ST) & 1, p.status);
-      if (good) {
-        tc_fence_after();
-        const uint32_t qa = smem_u32(q_s);
-        const uint32_t ka = smem_u32(k_s + st * C::kKVBytes);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk * 16 / C::kBoxD) * C::kBoxBytes + ((kk * 16) % C::kBoxD) * 2;
-          umma_bf16(s_tmem, smem_desc(qa + off, 16, 8 * C::kRowBytes, C::kSwCode),
-                    smem_desc(ka + off, 16, 8 * C::kRowBytes, C::kSwCode), kIdescS,
-                    kk > 0 ? 1u : 0u);
-        }
-        umma_commit(bar_s);
-      } else {
+                        mbar_wait(&bar_k[st], (j / ST) & 1, p.status);
+      if (good)
+        issue_s(j);
+      else
         flags[0] = 1;
-      }
     }
     const bool bad_s = !mbar_wait(bar_s, j & 1, p.status) || flags[0];
     if (__syncthreads_or(bad_s)) {
@@ -294,6 +340,11 @@ __global__ void __launch_bounds__(SG ? 128 : 256, 1)
       break;
     }
     tc_fence_after();
+    if (kSplitKV && t == 0 && j + ST < my_tiles) {  // S has read this K stage
+      int start, nv;
+      tile_of(sg, t0 + j + ST, start, nv);
+      issue_k(j + ST, start);
+    }
     if constexpr (SG) {
       // ---- softmax of row (t & 31) over keys [32w, 32w+32) of the tile
       const int kq = warp * 32;
@@ -363,10 +414,13 @@ __global__ void __launch_bounds__(SG ? 128 : 256, 1)
       for (int i = 0; i < kH; ++i)
         if (kb + i < nvalid) tm[i & 3] = fmaxf(tm[i & 3], s[i]);
       x_s[t] = fmaxf(fmaxf(tm[0], tm[1]), fmaxf(tm[2], tm[3]));
+      tc_fence_before();
       __syncthreads();
+      early_s(j);
       const float tmax = fmaxf(x_s[trow], x_s[128 + trow]);
       const float m_new = fmaxf(m_run, tmax * p.scale_log2);
       const float alpha = fast_exp2(m_run - m_new);
+      if (j > 0 && !mbar_wait(bar_o, (j - 1) & 1, p.status)) flags[0] = 1;  // P and O free
       float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < kH / 8; ++c) {  // 8 keys = one 16-byte chunk of P
@@ -386,8 +440,8 @@ __global__ void __launch_bounds__(SG ? 128 : 256, 1)
         *reinterpret_cast<uint4*>(prow + ((c ^ (trow & 7)) << 4)) =
             make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
-      // O (from earlier tiles) is rescaled in TMEM when the running max grew;
-      // the previous P V finished before this tile's S was committed.  Each
+      // O (from earlier tiles) is rescaled in TMEM when the running max grew
+      // (the previous P V was waited for above).  Each
       // thread rescales the half of the row's columns that it later reads.
       if (j > 0 && __any_sync(0xffffffffu, alpha < 1.f)) {
 #pragma unroll
@@ -410,23 +464,30 @@ __global__ void __launch_bounds__(SG ? 128 : 256, 1)
     // ---- O += P V
     if (t == 0) {
       tc_fence_after();
-      const uint32_t pa = smem_u32(p_s);
-      const uint32_t va = smem_u32(v_s + st * C::kKVBytes);
+      if (!kSplitKV || mbar_wait(&bar_v[st], (j / ST) & 1, p.status)) {
+        const uint32_t pa = smem_u32(p_s);
+        const uint32_t va = smem_u32(v_s + st * C::kKVBytes);
 #pragma unroll
-      for (int kk = 0; kk < kKeys / 16; ++kk) {
-        const uint32_t aoff = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-        const uint32_t boff = kk * 16 * C::kRowBytes;
-        umma_bf16(o_tmem, smem_desc(pa + aoff, 16, 1024, 2),
-                  smem_desc(va + boff, C::kBoxBytes, 8 * C::kRowBytes, C::kSwCode), kIdescO,
-                  (j > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < kKeys / 16; ++kk) {
+          const uint32_t aoff = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+          const uint32_t boff = kk * 16 * C::kRowBytes;
+          umma_bf16(o_tmem, smem_desc(pa + aoff, 16, 1024, 2),
+                    smem_desc(va + boff, C::kBoxBytes, 8 * C::kRowBytes, C::kSwCode), kIdescO,
+                    (j > 0 || kk > 0) ? 1u : 0u);
+        }
+      } else {
+        flags[0] = 1;
       }
-      umma_commit(bar_o);
+      umma_commit(bar_o);  // arrives at once when nothing was issued
       if (j + ST < my_tiles) {
-        // stage st is free once this P V has read V; the next S reads the other stage
+        // the V stage is free once this P V has read it
         if (mbar_wait(bar_o, j & 1, p.status)) {
           int start, nv;
           tile_of(sg, t0 + j + ST, start, nv);
-          issue_kv(j + ST, start);
+          if constexpr (kSplitKV)
+            issue_v(j + ST, start);
+          else
+            issue_kv(j + ST, start);
         } else {
           flags[0] = 1;
         }
