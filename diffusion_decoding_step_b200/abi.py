@@ -83,6 +83,7 @@ SIGNATURES = {
     "dllm_set_l2_prefetch": (C.c_int, [C.c_int64, C.c_int64, C.c_int32]),
     "dllm_set_layer_stack": (C.c_int, [C.c_int32, C.c_int32]),
     "dllm_layer_stack_plan": (C.c_int, [_CFG, _I, C.POINTER(C.c_int32)]),
+    "dllm_attention_plan": (C.c_int, [_CFG, _I, C.POINTER(C.c_int32)]),
     "dllm_selftest_wait_timeout": (C.c_int, [_P, C.c_int32, _P]),
     "dllm_status_string": (C.c_char_p, [C.c_int]),
 }

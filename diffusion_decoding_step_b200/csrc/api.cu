@@ -1461,6 +1461,38 @@ dllm_status dllm_set_layer_stack(int32_t enable, int32_t l2_lookahead) {
   return DLLM_OK;
 }
 
+dllm_status dllm_attention_plan(const dllm_config* cfg, int32_t block_start, int32_t* info) {
+  Shape s;
+  DLLM_TRY(check_cfg(cfg, &s));
+  if (!info) return DLLM_ERR_INVALID;
+  int n_rows, blk, seg_end;
+  if (block_start < 0) {  // the prefill
+    if (s.mode == DLLM_CACHE_NONE) return DLLM_ERR_INVALID;
+    n_rows = (s.mode == DLLM_CACHE_PREFIX || s.mode == DLLM_CACHE_PREFIX_SUFFIXQ) ? s.P : s.S;
+    if (n_rows < 1) return DLLM_ERR_INVALID;
+    blk = -1;
+    seg_end = n_rows;
+  } else {  // the rows and key range a decode step uses
+    DLLM_TRY(check_block(s, block_start));
+    const bool none = s.mode == DLLM_CACHE_NONE;
+    const bool sufq = s.mode == DLLM_CACHE_PREFIX_SUFFIXQ;
+    n_rows = none ? block_start + s.B : sufq ? s.S - block_start : s.B;
+    blk = block_start;
+    seg_end = none ? block_start + s.B : sufq ? s.S : 0;
+  }
+  const int ntb = key_tiles_bound(s, blk, seg_end);
+  const AttnPlan a = plan_attn(s, n_rows, ntb);
+  info[0] = a.sg ? 32 : 128;
+  info[1] = a.row_tiles;
+  info[2] = a.chunks;
+  info[3] = a.tpc;
+  info[4] = (int32_t)std::min<long long>((long long)s.b * s.Hkv * a.row_tiles * a.chunks, INT32_MAX);
+  info[5] = ntb;
+  info[6] = a.sg ? 128 : 256;
+  info[7] = a.tpc <= 1 ? 1 : 2;
+  return DLLM_OK;
+}
+
 dllm_status dllm_layer_stack_plan(const dllm_config* cfg, int32_t block_start, int32_t* info) {
   Shape s;
   DLLM_TRY(check_cfg(cfg, &s));

@@ -1,16 +1,15 @@
 // Non-causal GQA block attention on tcgen05.
 //
-// One CTA = (sequence b, kv head, tile of 128 query rows of that kv head's
+// One CTA = (sequence b, kv head, tile of query rows of that kv head's
 // group, chunk of key tiles).  The query rows of a kv head's group are the
 // g = Hq/Hkv heads x n_rows block rows, contiguous in the q buffer
 // [b][Hq][n_rows][D], so a row tile is one TMA box (rows past the group are
 // zero-filled).  Key/value tiles of 128 positions stream from the bf16 cache
 // [L][b][Hkv][S][D] through a TMA ring of ST stages.  Per key tile:
 //   S = Q K^T      UMMA M=128 (rows) x N=128 (keys) into TMEM columns [0,128)
-//   softmax        thread t owns query row t (TMEM lane t): the row is read
-//                  from TMEM once, max and sum run in registers in the log2
-//                  domain, P goes to shared memory in bf16 in the UMMA
-//                  K-major layout
+//   softmax        the row is read from TMEM once, max and sum run in
+//                  registers in the log2 domain, P goes to shared memory in
+//                  bf16 in the UMMA K-major layout
 //   O += P V       UMMA M=128 x N=D into TMEM columns [128,128+D); V is read
 //                  MN-major straight from its TMA tile.  O stays in TMEM; a
 //                  row is rescaled there only when its running max grows.
@@ -25,14 +24,20 @@
 // the CTA that owns the group, which adds the chunks' contributions in chunk
 // order and writes the bf16 output.  No partial goes through global memory.
 //
-// Small row tiles (32 query rows of a kv head's group, head_dim 128): the 32
-// rows are loaded four times into the 128-row Q tile, so S holds each row in
-// four TMEM lanes 32w + i, one per warp w.  Warp w takes keys [32w, 32w+32)
-// of every row in the softmax (the row max is exchanged once per tile through
-// shared memory) and writes its quarter of P into all four copies of the row,
-// so every lane of O = P V holds its full row and warp w reads, scales and
-// stores output columns [32w, 32w+32).  Each thread then works on 32 keys and
-// 32 output columns instead of 128, and all four warps share the merge.
+// Two row-tile shapes:
+// - 128 rows, 8 warps: threads t and t+128 share TMEM lane t % 128 (a warp
+//   reaches lanes 32(w % 4)..); each takes one 64-key half of the row in the
+//   softmax (the row max crosses the halves through shared memory) and the
+//   same half of the output columns.  K and V complete on separate barriers,
+//   and S of the next key tile is issued at the row-max barrier, once every
+//   thread holds this tile's S in registers, so it overlaps the softmax.
+// - 32 rows (SG, head_dim 128, 4 warps): the 32 rows are loaded four times
+//   into the 128-row Q tile, so S holds each row in four TMEM lanes 32w + i,
+//   one per warp w.  Warp w takes keys [32w, 32w+32) of every row in the
+//   softmax (the row max is exchanged once per tile through shared memory)
+//   and writes its quarter of P into all four copies of the row, so every
+//   lane of O = P V holds its full row and warp w reads, scales and stores
+//   output columns [32w, 32w+32).
 #include <float.h>
 
 #include "kernels.cuh"

@@ -400,6 +400,18 @@ dllm_status dllm_set_layer_stack(int32_t enable, int32_t l2_lookahead);
  * tile belongs to exactly one CTA share (a self-check of the partition). */
 dllm_status dllm_layer_stack_plan(const dllm_config* cfg, int32_t block_start, int32_t* info);
 
+/* Host query (no GPU work): the launch plan of the block attention
+ * (dllm_block_attn's kernel as a decode step or the prefill runs it) for the
+ * step of the block at block_start, or for the prefill when block_start < 0.
+ * info (host, 8 ints): [0] query rows per tile (32: each row tile is loaded
+ * four times and every warp takes a quarter of the keys and output columns;
+ * 128: two threads per row), [1] row tiles per (sequence, kv head), [2] key
+ * chunks per row tile (the cluster size), [3] 128-key tiles per chunk, [4]
+ * CTAs, [5] the key-tile bound the plan is made for, [6] threads per CTA, [7]
+ * K/V ring stages.  DLLM_ERR_INVALID for a block start that is not a block of
+ * the generation, or a prefill of a cache mode that has none. */
+dllm_status dllm_attention_plan(const dllm_config* cfg, int32_t block_start, int32_t* info);
+
 /* Failure-detection self-test (no counterpart on the pages).  Launches one
  * CTA whose bounded device wait has nothing to wait for: after limit_us
  * microseconds (clamped to [1, 2000000]) it gives up and ORs

@@ -200,3 +200,77 @@ def test_layer_stack_plan_partitions_every_weight_block():
         info = (C.c_int32 * 8)()
         assert abi.dllm_layer_stack_plan(C.byref(make_config(w)), w.prompt_len, info) == abi.DLLM_OK
         assert info[0] == 0
+
+
+def _attn_plan(w, block_start):
+    info = (C.c_int32 * 8)()
+    st = abi.dllm_attention_plan(C.byref(make_config(w)), block_start, info)
+    return st, list(info)
+
+
+def _cdiv(a, b):
+    return -(-a // b)
+
+
+def test_attention_plan_invariants():
+    """Host plan of the block attention: the row tiles cover the GQA group's
+    query rows with none empty, the key chunks cover the key-tile bound
+    (seven chunks run as eight, the last empty), the cluster stays within the
+    merge buffer's limit, 32-row tiles only with head_dim 128, and row tiles
+    that already fill the SMs keep one chunk."""
+    shapes = list(wl.WORKLOADS.values())
+    for mode in (wl.MODE_NONE, wl.MODE_PREFIX, wl.MODE_DUAL, wl.MODE_DUAL_PRUNED,
+                 wl.MODE_PREFIX_SUFFIXQ):
+        shapes.append(wl.WORKLOADS["dream7b_prefix"].replace(mode=mode, window=64))
+        shapes.append(wl.WORKLOADS["tiny"].replace(mode=mode, window=8))
+    for w in shapes:
+        g = w.n_q_heads // w.n_kv_heads
+        starts = list(range(w.prompt_len, w.seq_len, w.block))
+        if w.mode != wl.MODE_NONE:
+            starts.append(-1)
+        for blk in starts:
+            st, info = _attn_plan(w, blk)
+            assert st == abi.DLLM_OK, (w.name, blk)
+            rows_per_tile, row_tiles, chunks, tpc, ctas, ntb, threads, stages = info
+            if blk < 0:
+                n_rows = w.prompt_len if w.mode in (wl.MODE_PREFIX, wl.MODE_PREFIX_SUFFIXQ) \
+                    else w.seq_len
+            elif w.mode == wl.MODE_NONE:
+                n_rows = blk + w.block
+            elif w.mode == wl.MODE_PREFIX_SUFFIXQ:
+                n_rows = w.seq_len - blk
+            else:
+                n_rows = w.block
+            gr = g * n_rows
+            assert rows_per_tile in (32, 128)
+            assert rows_per_tile == 128 or w.head_dim == 128
+            assert rows_per_tile * row_tiles >= gr > rows_per_tile * (row_tiles - 1)
+            assert threads == (128 if rows_per_tile == 32 else 256)
+            assert chunks * tpc >= ntb >= 1
+            assert chunks == _cdiv(ntb, tpc) or (_cdiv(ntb, tpc) == 7 and chunks == 8)
+            assert chunks <= (8 if w.head_dim == 128 else 6)
+            assert stages == (1 if tpc <= 1 else 2)
+            assert ctas == w.batch * w.n_kv_heads * row_tiles * chunks
+            if w.batch * w.n_kv_heads * row_tiles >= 148:
+                assert chunks == 1
+
+
+def test_attention_plan_of_the_workload_shapes():
+    """The plans the design notes measure: LLaDA-8B's one-head groups take
+    32-row tiles in 4 key chunks; Dream-7B's 224-row groups 7 such tiles per
+    kv head with 3 chunks of 2 key tiles at the first block (84 CTAs, leaving
+    SMs for the O-projection); the long-context Qwen shape 128-row tiles in 2
+    chunks (one wave); the 16-sequence batch one chunk; prefills 128-row
+    tiles."""
+    W = wl.WORKLOADS
+    assert _attn_plan(W["llada8b_dual"], 256)[1][:5] == [32, 1, 4, 1, 128]
+    assert _attn_plan(W["dream7b_prefix"], 512)[1][:5] == [32, 7, 3, 2, 84]
+    assert _attn_plan(W["dream7b_prefix"], 992)[1][:4] == [32, 7, 4, 2]
+    q = _attn_plan(W["qwen7b_long_pruned"], 8192)[1]
+    assert q[:3] == [128, 4, 2] and q[4] == 128
+    assert _attn_plan(W["llada8b_dual_b16"], 1024)[1][:5] == [32, 1, 1, 10, 512]
+    assert _attn_plan(W["llada8b_dual"], -1)[1][:4] == [128, 4, 1, 4]
+    assert _attn_plan(W["tiny"], 64)[1][0] == 128                 # head_dim 32
+    # not a block of the generation; a prefill of a cache mode without one
+    assert _attn_plan(W["llada8b_dual"], 257)[0] == abi.DLLM_ERR_INVALID
+    assert _attn_plan(W["llada8b_dual"].replace(mode=wl.MODE_NONE), -1)[0] == abi.DLLM_ERR_INVALID
